@@ -1,0 +1,233 @@
+/*
+ * dash.h -- C ABI of the B200 (sm_100a) Delta-Attention Selective Halting
+ * (DASH) long-context prefill library, libdash.so.
+ *
+ * Pages cited (short name -> page title):
+ *   [DASH blog]  "DASH：基于注意力增量的Transformer令牌压缩，实现长序列推理高效加速"
+ *                §2.1 (U and Δattn_t = ||U_t||_2), §2.3 (single-shot halting
+ *                at layer L_s), §3.1 (algorithm steps, top-K, forced first /
+ *                last tokens, gather of the active set), §3.3 (pseudocode).
+ *   [DASH news]  "DASH：通过注意力动态监测实现长上下文高效预填充", sections
+ *                "层间更新动态监测" (threshold) and "选择性停止机制" (halted
+ *                tokens keep their KV-cache state).
+ *   [DASH abs]   "Stability Implies Redundancy: Delta Attention Selective
+ *                Halting for Efficient Long-Context Prefilling" (abstract).
+ *
+ * Conventions shared by every entry point:
+ *   - Every function returns dash_status; DASH_OK (0) on success.
+ *   - Argument errors (null pointers, negative or unsupported sizes, a too
+ *     small workspace) are detected on the host before anything is launched;
+ *     nothing is written then.
+ *   - Array pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them.  Scratch memory comes from the
+ *     caller's workspace (size from the matching *_workspace_size call).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; a call returns before the GPU finishes unless
+ *     its comment says it synchronises.
+ *   - Activations and weights are bf16 (raw bit patterns, dash_bf16),
+ *     row-major; scores fp32; token indices int32.
+ *   - Faults found on the device (a bounded wait that gave up, an index out
+ *     of range, a non-finite score) set a sticky device error word instead of
+ *     trapping; dash_device_error() reads and clears it.  While it is set,
+ *     the library's pipelined kernels return early.
+ */
+#ifndef DASH_H_
+#define DASH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t dash_bf16; /* bf16 bit pattern */
+
+typedef enum dash_status {
+  DASH_OK = 0,
+  DASH_ERR_INVALID_ARG = 1, /* null pointer, negative size, unknown enum */
+  DASH_ERR_SHAPE = 2,       /* a size the kernels do not support */
+  DASH_ERR_NONFINITE = 3,   /* a NaN/Inf score, or ||H_t|| = 0 in relative mode */
+  DASH_ERR_NO_MEMORY = 4,   /* workspace smaller than *_workspace_size() */
+  DASH_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed */
+  DASH_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+  DASH_ERR_INDEX = 7        /* an index list entry out of range */
+} dash_status;
+
+/* Decoder-stack dimensions.  Supported: head_dim 64 or 128; d_model and
+ * n_heads*head_dim multiples of 128 (d_model <= 4096); ffn_dim a multiple
+ * of 64; n_heads a multiple of n_kv_heads. */
+typedef struct dash_dims {
+  int32_t n_layers;
+  int32_t d_model;    /* d */
+  int32_t n_heads;    /* query heads hq */
+  int32_t n_kv_heads; /* key/value heads hkv */
+  int32_t head_dim;   /* hd */
+  int32_t ffn_dim;    /* F */
+  double rms_eps;     /* RMSNorm epsilon */
+  double rope_theta;  /* RoPE base θ (rotate-half pairs (i, i + hd/2)) */
+} dash_dims;
+
+/* Weights of one pre-norm decoder block ([DASH blog] §2.1: norm ->
+ * attention -> U, H' = H + U; then norm -> SwiGLU FFN -> residual).
+ * All bf16, row-major [out_features, in_features], no biases. */
+typedef struct dash_layer_weights {
+  const dash_bf16* attn_norm; /* [d] RMSNorm gain before attention */
+  const dash_bf16* w_qkv;     /* [(hq + 2*hkv)*hd, d]: q heads, then k heads, then v heads */
+  const dash_bf16* w_o;       /* [d, hq*hd] */
+  const dash_bf16* ffn_norm;  /* [d] RMSNorm gain before the FFN */
+  const dash_bf16* w_gate;    /* [F, d] */
+  const dash_bf16* w_up;      /* [F, d] */
+  const dash_bf16* w_down;    /* [d, F] */
+} dash_layer_weights;
+
+typedef enum dash_mode {
+  DASH_MODE_PRUNE = 0, /* halted tokens leave the sequence ([DASH blog] §3.1) */
+  DASH_MODE_HALT = 1,  /* halted tokens stay frozen, their K/V visible ([DASH news]) */
+  DASH_MODE_DENSE = 2  /* no halting: every layer on every token */
+} dash_mode;
+
+typedef enum dash_select_kind {
+  DASH_SELECT_TOPK = 0,     /* top floor(keep_ratio * n) by score ([DASH blog] §3.1) */
+  DASH_SELECT_THRESHOLD = 1 /* score >= threshold ([DASH news] "层间更新动态监测") */
+} dash_select_kind;
+
+typedef enum dash_score_kind {
+  DASH_SCORE_ABS = 0, /* Δ_t = ||U_t||_2 ([DASH blog] §2.1) */
+  DASH_SCORE_REL = 1  /* Δ_t = ||U_t||_2 / ||H_t||_2, H = the layer's input residual */
+} dash_score_kind;
+
+typedef struct dash_config {
+  int32_t halt_layer; /* L_s, 0-based: layers 0..L_s run on all T tokens ([DASH blog] §2.3) */
+  int32_t mode;       /* dash_mode */
+  int32_t select;     /* dash_select_kind */
+  int32_t score;      /* dash_score_kind */
+  double keep_ratio;  /* top-k: keep = 1 - ρ */
+  float threshold;    /* threshold mode: keep t iff Δ_t >= threshold */
+  int32_t keep_first; /* first tokens always kept (0 = none) */
+  int32_t keep_last;  /* last tokens always kept (0 = none) */
+} dash_config;
+
+/* Human-readable name of a status code (static string). */
+const char* dash_status_string(dash_status s);
+
+/* Reads and clears the sticky device error word.  Synchronises the device.
+ * Returns DASH_OK, DASH_ERR_TIMEOUT, DASH_ERR_INDEX or DASH_ERR_NONFINITE
+ * (the first one found, in that order of priority: TIMEOUT, INDEX, NONFINITE). */
+dash_status dash_device_error(void);
+
+/* ---------------------------------------------------------------- score --
+ * Δattn per token ([DASH blog] §2.1: Δattn_t = ||U_t||_2; relative form
+ * ||U_t||_2 / ||H_t||_2 when relative != 0).
+ *   U, H:  [T, d] bf16 (H may be NULL when relative == 0).
+ *   delta: [T] fp32 out; sums of squares accumulate in fp32.
+ * In relative mode a row with ||H_t|| = 0 yields Inf/NaN and sets the
+ * NONFINITE device error.  Requires d % 8 == 0. */
+dash_status dash_score(const dash_bf16* U, const dash_bf16* H, int64_t T, int32_t d,
+                       int32_t relative, float* delta, void* stream);
+
+/* --------------------------------------------------------------- select --
+ * Number of active tokens in top-k mode ([DASH blog] §3.1):
+ * |forced| + floor(keep_ratio * (T - |forced|)), forced = the first
+ * keep_first and the last keep_last tokens.  Host-only arithmetic in double. */
+int64_t dash_topk_count(int64_t T, double keep_ratio, int32_t keep_first, int32_t keep_last);
+
+/* Workspace bytes dash_select needs for T scores (currently 0: all scratch
+ * lives in shared memory). */
+size_t dash_select_workspace_size(int64_t T);
+
+/* Active-set selection ([DASH blog] §3.1 and the final sort of §3.3;
+ * threshold form from [DASH news]).
+ *   scores:  [T] fp32.
+ *   kind:    DASH_SELECT_TOPK (uses keep_ratio) or DASH_SELECT_THRESHOLD
+ *            (uses threshold: keep iff score >= threshold).
+ *   Order among scores: larger first; equal scores (+0 and -0 are equal)
+ *   go to the lower index.
+ *   idx:     [T] int32 out (capacity T): the active indices, ascending,
+ *            unique; forced tokens always included.
+ *   halted:  [T] int32 out or NULL: the complement, ascending.
+ *   count:   [1] int32 device out: number of active tokens, or -3
+ *            (= -DASH_ERR_NONFINITE) if any score is NaN/Inf (then idx is
+ *            not written and the NONFINITE device error is set).
+ * Identical fp32 inputs give bit-identical outputs. */
+dash_status dash_select(const float* scores, int64_t T, int32_t kind, double keep_ratio,
+                        float threshold, int32_t keep_first, int32_t keep_last,
+                        int32_t* idx, int32_t* halted, int32_t* count,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------ compact/scatter --
+ * Gather of the active rows ([DASH blog] §3.1 "复用活跃集合"):
+ * Y[i, :] = X[idx[i], :] for i < K.  X: [T, d], Y: [K, d] bf16, d % 8 == 0.
+ * An idx entry outside [0, T) sets the INDEX device error; its row is not
+ * written. */
+dash_status dash_compact(const dash_bf16* X, int64_t T, const int32_t* idx, int64_t K,
+                         int32_t d, dash_bf16* Y, void* stream);
+
+/* Inverse of dash_compact: X[idx[i], :] = Y[i, :]; other rows of X unchanged.
+ * idx entries must be distinct (ascending lists from dash_select are). */
+dash_status dash_scatter(const dash_bf16* Y, const int32_t* idx, int64_t K, int32_t d,
+                         dash_bf16* X, int64_t T, void* stream);
+
+/* ---------------------------------------------------------------- layer --
+ * Halt-mode context for one compacted layer ([DASH news] "选择性停止机制":
+ * halted tokens keep their state and their K/V stay visible, but issue no
+ * queries).  The active rows are the layer's H argument, in ascending
+ * original-position order.
+ *   active_idx: [M] original positions of the active rows (ascending).
+ *   halted_idx: [T - M] original positions of the halted rows (ascending).
+ *   h_full:     [T, d] hidden states by original position; rows halted_idx
+ *               hold the frozen states (only those rows are read).
+ * The K/V of halted rows are recomputed from their frozen states with this
+ * layer's weights; queries of active rows attend causally, by original
+ * position, over all T rows. */
+typedef struct dash_halt_ctx {
+  const int32_t* active_idx;
+  const int32_t* halted_idx;
+  const dash_bf16* h_full;
+  int64_t T;
+} dash_halt_ctx;
+
+/* Workspace bytes for dash_layer_forward on M query rows with T_kv
+ * key/value rows (T_kv = M unless halt mode) and positions below max_pos. */
+size_t dash_layer_workspace_size(const dash_dims* dims, int64_t M, int64_t T_kv, int64_t max_pos);
+
+/* One pre-norm decoder block in place on H [M, d] ([DASH blog] §2.1).
+ *   pos:   [M] int32 RoPE positions of the rows, ascending, < max_pos; NULL
+ *          means 0..M-1.  Attention is causal over the rows' order (prune /
+ *          dense), or by original position against all T rows (halt).
+ *   halt:  NULL, or the halt-mode context (then pos must be
+ *          halt->active_idx and max_pos >= halt->T).
+ *   delta: [M] fp32 out or NULL: Δ of this layer's attention update U
+ *          (U in fp32 before rounding), absolute or relative to ||H_in||.
+ * Requires 1 <= M and the dims constraints above. */
+dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* w, dash_bf16* H,
+                               int64_t M, const int32_t* pos, int64_t max_pos,
+                               const dash_halt_ctx* halt, float* delta, int32_t relative,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* -------------------------------------------------------------- prefill --
+ * Workspace bytes for dash_prefill of T tokens under cfg. */
+size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_config* cfg);
+
+/* Single-shot DASH prefill ([DASH blog] §2.3 and §3.1; [DASH news]).
+ * Layers 0..halt_layer run on all T tokens; the halting layer's attention
+ * update gives Δ (fused into its o_proj epilogue); the active set is
+ * selected once and reused by every later layer.
+ *   layers:    [dims->n_layers] weights.
+ *   H:         [T, d] bf16 in: input hidden states; out: prune -> rows
+ *              0..K-1 hold the active tokens' final states (rest undefined);
+ *              halt / dense -> all T rows (halted rows frozen at the halting
+ *              layer's output).
+ *   idx_out:   [T] int32 device out or NULL: active indices, ascending.
+ *   K_out:     host out or NULL: number of active tokens (T for dense).
+ *   delta_out: [T] fp32 device out or NULL: Δ at the halting layer.
+ * Synchronises the stream once, after selection, to read K (this is also
+ * where NONFINITE is reported).  Output stays on the device. */
+dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H,
+                         int64_t T, const dash_config* cfg, int32_t* idx_out, int64_t* K_out,
+                         float* delta_out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DASH_H_ */

@@ -1,0 +1,42 @@
+/*
+ * dash_ops.h -- building blocks of dash_layer_forward exported for
+ * per-kernel parity tests and benchmarks.  Conventions are those of dash.h
+ * (device pointers owned by the caller, bf16 bit patterns, row-major,
+ * asynchronous on `stream`, host-side argument checks before any launch).
+ *
+ * Page cited: [DASH blog] "DASH：基于注意力增量的Transformer令牌压缩，实现长序列推理高效加速",
+ * §2.1 (the block H -> norm -> attention -> U, H' = H + U, whose pieces these are).
+ */
+#ifndef DASH_OPS_H_
+#define DASH_OPS_H_
+
+#include "dash.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* RMSNorm: Y[r] = X[r] * rsqrt(mean(X[r]^2) + eps) * g, fp32 math.
+ * X, Y: [M, d] bf16, g: [d].  Requires d % 8 == 0 and d <= 4096. */
+dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf16* g, double eps,
+                         dash_bf16* Y, void* stream);
+
+/* Y[M, N] = A[M, K] * W[N, K]^T on the tensor cores (tcgen05, fp32
+ * accumulation in TMEM, bf16 out).  Requires K % 64 == 0, N % 128 == 0,
+ * 16-byte aligned pointers. */
+dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf16* W, int32_t N,
+                        dash_bf16* Y, void* stream);
+
+/* Causal grouped-query attention (the attention module of §2.1):
+ *   Q: [M, hq*hd], K, V: [T_kv, hkv*hd], O: [M, hq*hd] bf16.
+ *   Query i sees key j iff j <= qpos(i) and j < T_kv, where qpos(i) =
+ *   qpos[i] (ascending int32 positions) or i when qpos is NULL.
+ *   Scale 1/sqrt(hd), fp32 softmax.  hd must be 64 or 128, hq % hkv == 0. */
+dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M,
+                           int64_t T_kv, int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos,
+                           dash_bf16* O, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DASH_OPS_H_ */

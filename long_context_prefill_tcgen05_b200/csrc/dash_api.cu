@@ -1,0 +1,639 @@
+// C ABI of libdash (declared in include/dash.h and include/dash_ops.h):
+// argument checks, workspace carving, tensor-map encoding, kernel launches,
+// and the host-side layer loop of the single-shot DASH prefill.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "dash.h"
+#include "dash_ops.h"
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "rowops.cuh"
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+using dash::attn::attn_kernel;
+using dash::gemm::EpiArgs;
+using dash::gemm::gemm_kernel;
+
+// ------------------------------------------------------------- device info
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+
+dash_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DASH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return DASH_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  if (g_dev[dev].num_sms == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return DASH_ERR_CUDA;
+    g_dev[dev].num_sms = n;
+  }
+  *out = &g_dev[dev];
+  return DASH_OK;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline const bf16* cb(const dash_bf16* p) { return reinterpret_cast<const bf16*>(p); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline dash_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+}
+
+// 2D bf16 tensor map with a 64-element (128-byte) inner box and 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+              uint32_t box_rows) {
+  if (!aligned16(base) || (ld * 2) % 16 != 0 || rows == 0 || cols % 64 != 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------- GEMM
+template <int BN, int EPI>
+dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
+                        const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st) {
+  using C = dash::gemm::Cfg<BN>;
+  if (M == 0) return DASH_OK;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  CUtensorMap ma, mb, mb2;
+  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM)) return DASH_ERR_INVALID_ARG;
+  if (EPI == dash::gemm::kEpiSwiglu) {
+    if (!make_map(&mb, B, N / 2, K, K, BN / 2) || !make_map(&mb2, B2, N / 2, K, K, BN / 2))
+      return DASH_ERR_INVALID_ARG;
+  } else {
+    if (!make_map(&mb, B, N, K, K, BN)) return DASH_ERR_INVALID_ARG;
+    mb2 = mb;
+  }
+  dash::gemm::Shape sh;
+  sh.M = static_cast<int>(M);
+  sh.N = N;
+  sh.K = K;
+  sh.tiles_m = static_cast<int>((M + dash::gemm::BM - 1) / dash::gemm::BM);
+  sh.tiles_n = N / BN;
+  sh.num_tiles = sh.tiles_m * sh.tiles_n;
+  const int grid = sh.num_tiles < di.num_sms ? sh.num_tiles : di.num_sms;
+  gemm_kernel<BN, EPI><<<grid, dash::gemm::kThreads, C::kSmemBytes, st>>>(ma, mb, mb2, sh, ep);
+  return launch_status();
+}
+
+template <int EPI>
+dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
+                 const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int* bn_used = nullptr) {
+  if (K % dash::gemm::BK != 0 || M > INT32_MAX) return DASH_ERR_SHAPE;
+  // SwiGLU tiles hold BN/2 gate + BN/2 up columns, so N = 2F must split into
+  // whole tiles on both halves.
+  const bool can256 = EPI == dash::gemm::kEpiSwiglu ? (N / 2) % 128 == 0 : N % 256 == 0;
+  const bool can128 = EPI == dash::gemm::kEpiSwiglu ? (N / 2) % 64 == 0 : N % 128 == 0;
+  if (can256) {
+    if (bn_used) *bn_used = 256;
+    return launch_gemm<256, EPI>(di, A, lda, M, K, B, B2, N, ep, st);
+  }
+  if (can128) {
+    if (bn_used) *bn_used = 128;
+    return launch_gemm<128, EPI>(di, A, lda, M, K, B, B2, N, ep, st);
+  }
+  return DASH_ERR_SHAPE;
+}
+
+inline int o_proj_tiles(int d) { return d % 256 == 0 ? d / 256 : d / 128; }
+
+// -------------------------------------------------------------- attention
+template <int HD>
+dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
+                           int64_t T_kv, int hq, int hkv, const int32_t* qpos, bf16* O, int64_t ldo,
+                           cudaStream_t st) {
+  using C = dash::attn::Cfg<HD>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, M, static_cast<uint64_t>(hq) * HD, ldq, dash::attn::BQ) ||
+      !make_map(&mk, K, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV) ||
+      !make_map(&mv, V, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV))
+    return DASH_ERR_INVALID_ARG;
+  dash::attn::Params p;
+  p.out = O;
+  p.ldo = ldo;
+  p.qpos = qpos;
+  p.M = static_cast<int>(M);
+  p.T_kv = static_cast<int>(T_kv);
+  p.hq = hq;
+  p.hkv = hkv;
+  p.hd = HD;
+  p.n_qtiles = static_cast<int>((M + dash::attn::BQ - 1) / dash::attn::BQ);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
+  const int64_t grid = static_cast<int64_t>(p.n_qtiles) * hq;
+  attn_kernel<HD><<<static_cast<unsigned>(grid), dash::attn::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+dash_status attention(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
+                      int64_t T_kv, int hq, int hkv, int hd, const int32_t* qpos, bf16* O, int64_t ldo,
+                      cudaStream_t st) {
+  if (M == 0) return DASH_OK;
+  if (T_kv <= 0 || M > INT32_MAX || T_kv > INT32_MAX || hkv <= 0 || hq % hkv != 0) return DASH_ERR_SHAPE;
+  if (hd == 128) return launch_attn_hd<128>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, O, ldo, st);
+  if (hd == 64) return launch_attn_hd<64>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, O, ldo, st);
+  return DASH_ERR_SHAPE;
+}
+
+// ---------------------------------------------------------------- row ops
+dash_status rmsnorm(const bf16* X, int64_t x_rows, const int32_t* rowmap, int64_t rows, int d, const bf16* g,
+                    double eps, bf16* Y, cudaStream_t st) {
+  if (rows == 0) return DASH_OK;
+  const int warps = 8;
+  const int64_t blocks = (rows + warps - 1) / warps;
+  dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
+      X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y);
+  return launch_status();
+}
+
+dash_status move_rows(bool scatter, const bf16* src, bf16* dst, const int32_t* idx, int64_t K, int64_t T, int d,
+                      const DeviceInfo& di, cudaStream_t st) {
+  if (K == 0) return DASH_OK;
+  const int warps = 8;
+  int64_t blocks = (K + warps - 1) / warps;
+  const int64_t cap = static_cast<int64_t>(di.num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  if (scatter)
+    dash::rows::move_rows_kernel<true><<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(src, dst, idx, K, T, d);
+  else
+    dash::rows::move_rows_kernel<false><<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(src, dst, idx, K, T, d);
+  return launch_status();
+}
+
+dash_status rope_table(float2* tab, int64_t max_pos, int hd, double theta, const DeviceInfo& di, cudaStream_t st) {
+  const int64_t n = max_pos * (hd / 2);
+  int64_t blocks = (n + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(di.num_sms) * 32;
+  if (blocks > cap) blocks = cap;
+  if (blocks == 0) return DASH_OK;
+  dash::rows::rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(tab, max_pos, hd / 2, theta);
+  return launch_status();
+}
+
+// -------------------------------------------------------------- workspace
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct LayerWs {
+  float2* rope;  // [max_pos, hd/2]
+  bf16* X;       // [M, max(d, hq*hd)]: norm output, then attention output
+  bf16* Q;       // [M, hq*hd]
+  bf16* Kb;      // [T_kv, hkv*hd]
+  bf16* Vb;      // [T_kv, hkv*hd]
+  bf16* Act;     // [max(M*F, (T_kv-M)*d)]: SwiGLU output; halt-mode frozen-row norms
+  float* ssq_u;  // [o_proj tiles, M]
+  float* ssq_h;
+};
+
+bool dims_ok(const dash_dims* D) {
+  if (!D) return false;
+  const int d = D->d_model, hq = D->n_heads, hkv = D->n_kv_heads, hd = D->head_dim, F = D->ffn_dim;
+  if (D->n_layers <= 0 || d <= 0 || hq <= 0 || hkv <= 0 || F <= 0) return false;
+  if (hd != 64 && hd != 128) return false;
+  if (hq % hkv != 0) return false;
+  if (d % 128 != 0 || d > 4096 || F % 64 != 0 || (hq * hd) % 128 != 0) return false;
+  if (!(D->rms_eps >= 0.0) || !(D->rope_theta > 0.0)) return false;
+  return true;
+}
+
+void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, Carver& c, LayerWs& w) {
+  const int64_t d = D.d_model, qd = static_cast<int64_t>(D.n_heads) * D.head_dim;
+  const int64_t kvd = static_cast<int64_t>(D.n_kv_heads) * D.head_dim, F = D.ffn_dim;
+  w.rope = c.take<float2>(static_cast<size_t>(max_pos) * (D.head_dim / 2));
+  w.X = c.take<bf16>(static_cast<size_t>(M) * (d > qd ? d : qd));
+  w.Q = c.take<bf16>(static_cast<size_t>(M) * qd);
+  w.Kb = c.take<bf16>(static_cast<size_t>(T_kv) * kvd);
+  w.Vb = c.take<bf16>(static_cast<size_t>(T_kv) * kvd);
+  const int64_t act = M * F > (T_kv - M) * d ? M * F : (T_kv - M) * d;
+  w.Act = c.take<bf16>(static_cast<size_t>(act));
+  const int nt = o_proj_tiles(D.d_model);
+  w.ssq_u = c.take<float>(static_cast<size_t>(nt) * M);
+  w.ssq_h = c.take<float>(static_cast<size_t>(nt) * M);
+}
+
+// One pre-norm decoder block on H [M, d] in place (rope table already built).
+dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_layer_weights& w, bf16* H, int64_t M,
+                       const int32_t* pos, const dash_halt_ctx* halt, float* delta, int relative,
+                       const LayerWs& ws, cudaStream_t st) {
+  if (M == 0) return DASH_OK;
+  const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
+  const int qd = hq * hd, kvd = hkv * hd;
+  const int64_t T_kv = halt ? halt->T : M;
+  dash_status s;
+
+  EpiArgs qkv{};
+  qkv.q = ws.Q;
+  qkv.k = ws.Kb;
+  qkv.v = ws.Vb;
+  qkv.ldq = qd;
+  qkv.ldkv = kvd;
+  qkv.rope = reinterpret_cast<const float4*>(ws.rope);
+  qkv.hq = hq;
+  qkv.hkv = hkv;
+  qkv.hd = hd;
+
+  // Keys / values of the halted rows, from their frozen states, at their
+  // original positions ([DASH news] "选择性停止机制").
+  if (halt && T_kv > M) {
+    const int64_t nh = T_kv - M;
+    if ((s = rmsnorm(cb(halt->h_full), T_kv, halt->halted_idx, nh, d, cb(w.attn_norm), D.rms_eps, ws.Act, st)) != DASH_OK)
+      return s;
+    EpiArgs kv = qkv;
+    kv.q = nullptr;
+    kv.pos = halt->halted_idx;
+    kv.kv_rowmap = halt->halted_idx;
+    kv.col_offset = qd;
+    if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.Act, d, nh, d, cb(w.w_qkv) + static_cast<int64_t>(qd) * d, nullptr,
+                                       2 * kvd, kv, st)) != DASH_OK)
+      return s;
+  }
+
+  // a1: input RMSNorm
+  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.attn_norm), D.rms_eps, ws.X, st)) != DASH_OK) return s;
+  // a2: QKV projection + RoPE (k/v of active rows land at their original rows in halt mode)
+  qkv.pos = pos;
+  qkv.kv_rowmap = halt ? halt->active_idx : nullptr;
+  qkv.col_offset = 0;
+  if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st)) != DASH_OK)
+    return s;
+  // a3: causal GQA attention -> O (into X)
+  if ((s = attention(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, ws.X,
+                     qd, st)) != DASH_OK)
+    return s;
+  // a4: o_proj + residual (+ per-row sums of U^2 and H^2 for Δ)
+  EpiArgs o{};
+  o.out = H;
+  o.ldo = d;
+  o.ssq_u = ws.ssq_u;
+  o.ssq_h = ws.ssq_h;
+  int bn = 0;
+  if (delta)
+    s = gemm<dash::gemm::kEpiResidSsq>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, &bn);
+  else
+    s = gemm<dash::gemm::kEpiResid>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, &bn);
+  if (s != DASH_OK) return s;
+  if (delta) {
+    const int64_t blocks = (M + 255) / 256;
+    dash::rows::score_from_ssq_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(ws.ssq_u, ws.ssq_h, d / bn,
+                                                                                     M, relative, delta);
+    if ((s = launch_status()) != DASH_OK) return s;
+  }
+  // a5: post-attention RMSNorm, gate/up GEMM with SwiGLU
+  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.ffn_norm), D.rms_eps, ws.X, st)) != DASH_OK) return s;
+  EpiArgs sw{};
+  sw.out = ws.Act;
+  sw.ldo = F;
+  if ((s = gemm<dash::gemm::kEpiSwiglu>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st)) != DASH_OK) return s;
+  // a6: down projection + residual
+  EpiArgs dn{};
+  dn.out = H;
+  dn.ldo = d;
+  return gemm<dash::gemm::kEpiResid>(di, ws.Act, F, M, F, cb(w.w_down), nullptr, d, dn, st);
+}
+
+bool weights_ok(const dash_layer_weights* w) {
+  return w && w->attn_norm && w->w_qkv && w->w_o && w->ffn_norm && w->w_gate && w->w_up && w->w_down &&
+         aligned16(w->attn_norm) && aligned16(w->w_qkv) && aligned16(w->w_o) && aligned16(w->ffn_norm) &&
+         aligned16(w->w_gate) && aligned16(w->w_up) && aligned16(w->w_down);
+}
+
+struct PrefillWs {
+  LayerWs L;
+  bf16* Hc;       // [T, d] compacted active rows
+  float* delta;   // [T]
+  int32_t* idx;   // [T]
+  int32_t* halted;// [T]
+  int32_t* count; // [1]
+};
+
+void carve_prefill(const dash_dims& D, int64_t T, Carver& c, PrefillWs& w) {
+  carve_layer(D, T, T, T, c, w.L);
+  w.Hc = c.take<bf16>(static_cast<size_t>(T) * D.d_model);
+  w.delta = c.take<float>(static_cast<size_t>(T));
+  w.idx = c.take<int32_t>(static_cast<size_t>(T));
+  w.halted = c.take<int32_t>(static_cast<size_t>(T));
+  w.count = c.take<int32_t>(1);
+}
+
+dash_status select_impl(const float* scores, int64_t T, int kind, double keep, float thr, int keep_first,
+                        int keep_last, int32_t* idx, int32_t* halted, int32_t* count, cudaStream_t st) {
+  const int64_t lo = keep_first < T ? keep_first : T;
+  int64_t hi = keep_last > 0 ? T - keep_last : T;
+  if (hi < lo) hi = lo;
+  const int64_t n_mid = hi - lo;
+  const int64_t k_dyn = static_cast<int64_t>(std::floor(keep * static_cast<double>(n_mid)));
+  if (T == 0) return cudaMemsetAsync(count, 0, sizeof(int32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+  dash::rows::select_kernel<<<1, dash::rows::kSelThreads, 0, st>>>(scores, T, kind, k_dyn, thr, lo, hi, idx, halted,
+                                                                    count);
+  return launch_status();
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* dash_status_string(dash_status s) {
+  switch (s) {
+    case DASH_OK: return "ok";
+    case DASH_ERR_INVALID_ARG: return "invalid argument";
+    case DASH_ERR_SHAPE: return "unsupported shape";
+    case DASH_ERR_NONFINITE: return "non-finite score";
+    case DASH_ERR_NO_MEMORY: return "workspace too small";
+    case DASH_ERR_CUDA: return "CUDA error";
+    case DASH_ERR_TIMEOUT: return "device wait timed out";
+    case DASH_ERR_INDEX: return "index out of range";
+  }
+  return "unknown status";
+}
+
+dash_status dash_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return DASH_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, dash::g_dash_dev_error, sizeof(v)) != cudaSuccess) return DASH_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(dash::g_dash_dev_error, &zero, sizeof(zero)) != cudaSuccess) return DASH_ERR_CUDA;
+  if (v & dash::kDevErrTimeout) return DASH_ERR_TIMEOUT;
+  if (v & dash::kDevErrIndex) return DASH_ERR_INDEX;
+  if (v & dash::kDevErrNonfinite) return DASH_ERR_NONFINITE;
+  return DASH_OK;
+}
+
+dash_status dash_score(const dash_bf16* U, const dash_bf16* H, int64_t T, int32_t d, int32_t relative, float* delta,
+                       void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0) return DASH_ERR_SHAPE;
+  if (T == 0) return DASH_OK;
+  if (!U || !delta || (relative && !H) || !aligned16(U) || (relative && !aligned16(H))) return DASH_ERR_INVALID_ARG;
+  const int warps = 8;
+  const int64_t blocks = (T + warps - 1) / warps;
+  dash::rows::score_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, as_stream(stream)>>>(
+      reinterpret_cast<const bf16*>(U), reinterpret_cast<const bf16*>(H), T, d, relative ? 1 : 0, delta);
+  return launch_status();
+}
+
+int64_t dash_topk_count(int64_t T, double keep_ratio, int32_t keep_first, int32_t keep_last) {
+  if (T <= 0) return 0;
+  const int64_t lo = keep_first > 0 ? (keep_first < T ? keep_first : T) : 0;
+  int64_t hi = keep_last > 0 ? T - keep_last : T;
+  if (hi < lo) hi = lo;
+  return (T - (hi - lo)) + static_cast<int64_t>(std::floor(keep_ratio * static_cast<double>(hi - lo)));
+}
+
+size_t dash_select_workspace_size(int64_t) { return 0; }
+
+dash_status dash_select(const float* scores, int64_t T, int32_t kind, double keep_ratio, float threshold,
+                        int32_t keep_first, int32_t keep_last, int32_t* idx, int32_t* halted, int32_t* count,
+                        void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
+  if (!count || (T > 0 && (!scores || !idx))) return DASH_ERR_INVALID_ARG;
+  if (kind != DASH_SELECT_TOPK && kind != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
+  if (keep_first < 0 || keep_last < 0) return DASH_ERR_INVALID_ARG;
+  if (kind == DASH_SELECT_TOPK && !(keep_ratio >= 0.0 && keep_ratio <= 1.0)) return DASH_ERR_INVALID_ARG;
+  return select_impl(scores, T, kind, keep_ratio, threshold, keep_first, keep_last, idx, halted, count,
+                     as_stream(stream));
+}
+
+dash_status dash_compact(const dash_bf16* X, int64_t T, const int32_t* idx, int64_t K, int32_t d, dash_bf16* Y,
+                         void* stream) {
+  if (K < 0 || T < 0 || d <= 0 || d % 8 != 0) return DASH_ERR_SHAPE;
+  if (K == 0) return DASH_OK;
+  if (!X || !idx || !Y || !aligned16(X) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  return move_rows(false, reinterpret_cast<const bf16*>(X), reinterpret_cast<bf16*>(Y), idx, K, T, d, *di,
+                   as_stream(stream));
+}
+
+dash_status dash_scatter(const dash_bf16* Y, const int32_t* idx, int64_t K, int32_t d, dash_bf16* X, int64_t T,
+                         void* stream) {
+  if (K < 0 || T < 0 || d <= 0 || d % 8 != 0) return DASH_ERR_SHAPE;
+  if (K == 0) return DASH_OK;
+  if (!X || !idx || !Y || !aligned16(X) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  return move_rows(true, reinterpret_cast<const bf16*>(Y), reinterpret_cast<bf16*>(X), idx, K, T, d, *di,
+                   as_stream(stream));
+}
+
+dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf16* g, double eps, dash_bf16* Y,
+                         void* stream) {
+  if (M < 0 || d <= 0 || d % 8 != 0 || d > 8 * 32 * dash::rows::kMaxVec) return DASH_ERR_SHAPE;
+  if (M == 0) return DASH_OK;
+  if (!X || !g || !Y || !aligned16(X) || !aligned16(g) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
+  return rmsnorm(reinterpret_cast<const bf16*>(X), M, nullptr, M, d, reinterpret_cast<const bf16*>(g), eps,
+                 reinterpret_cast<bf16*>(Y), as_stream(stream));
+}
+
+dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf16* W, int32_t N, dash_bf16* Y,
+                        void* stream) {
+  if (M < 0 || K <= 0 || N <= 0 || K % 64 != 0 || N % 128 != 0) return DASH_ERR_SHAPE;
+  if (M == 0) return DASH_OK;
+  if (!A || !W || !Y || !aligned16(A) || !aligned16(W) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  EpiArgs ep{};
+  ep.out = reinterpret_cast<bf16*>(Y);
+  ep.ldo = N;
+  return gemm<dash::gemm::kEpiStore>(*di, reinterpret_cast<const bf16*>(A), K, M, K, reinterpret_cast<const bf16*>(W),
+                                     nullptr, N, ep, as_stream(stream));
+}
+
+dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M, int64_t T_kv,
+                           int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos, dash_bf16* O, void* stream) {
+  if (M < 0 || T_kv < 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || (hd != 64 && hd != 128)) return DASH_ERR_SHAPE;
+  if (M == 0) return DASH_OK;
+  if (T_kv == 0) return DASH_ERR_SHAPE;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return DASH_ERR_INVALID_ARG;
+  if (!qpos && M > T_kv) return DASH_ERR_SHAPE;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  const int64_t qd = static_cast<int64_t>(hq) * hd, kvd = static_cast<int64_t>(hkv) * hd;
+  return attention(reinterpret_cast<const bf16*>(Q), qd, reinterpret_cast<const bf16*>(K),
+                   reinterpret_cast<const bf16*>(V), kvd, M, T_kv, hq, hkv, hd, qpos, reinterpret_cast<bf16*>(O), qd,
+                   as_stream(stream));
+}
+
+size_t dash_layer_workspace_size(const dash_dims* dims, int64_t M, int64_t T_kv, int64_t max_pos) {
+  if (!dims_ok(dims) || M < 0 || T_kv < M || max_pos < 0) return 0;
+  Carver c{nullptr};
+  LayerWs w;
+  carve_layer(*dims, M, T_kv, max_pos, c, w);
+  return c.off + 256;
+}
+
+dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* w, dash_bf16* H, int64_t M,
+                               const int32_t* pos, int64_t max_pos, const dash_halt_ctx* halt, float* delta,
+                               int32_t relative, void* ws, size_t ws_bytes, void* stream) {
+  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
+  if (!weights_ok(w) || !H || !aligned16(H)) return DASH_ERR_INVALID_ARG;
+  if (M < 0 || M > INT32_MAX) return DASH_ERR_SHAPE;
+  if (M == 0) return DASH_OK;
+  int64_t T_kv = M;
+  if (halt) {
+    if (!halt->active_idx || !halt->h_full || halt->T < M || pos != halt->active_idx) return DASH_ERR_INVALID_ARG;
+    if (halt->T > M && !halt->halted_idx) return DASH_ERR_INVALID_ARG;
+    T_kv = halt->T;
+    if (max_pos < halt->T) return DASH_ERR_INVALID_ARG;
+  }
+  if (!pos && max_pos < M) return DASH_ERR_INVALID_ARG;
+  if (max_pos > INT32_MAX) return DASH_ERR_SHAPE;
+  const size_t need = dash_layer_workspace_size(dims, M, T_kv, max_pos);
+  if (!ws || ws_bytes < need) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  LayerWs L;
+  carve_layer(*dims, M, T_kv, max_pos, c, L);
+  cudaStream_t st = as_stream(stream);
+  if ((s = rope_table(L.rope, max_pos, dims->head_dim, dims->rope_theta, *di, st)) != DASH_OK) return s;
+  return layer_impl(*di, *dims, *w, reinterpret_cast<bf16*>(H), M, pos, halt, delta, relative, L, st);
+}
+
+size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_config* cfg) {
+  if (!dims_ok(dims) || T < 0 || !cfg) return 0;
+  Carver c{nullptr};
+  PrefillWs w;
+  carve_prefill(*dims, T, c, w);
+  return c.off + 256;
+}
+
+dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, int64_t T,
+                         const dash_config* cfg, int32_t* idx_out, int64_t* K_out, float* delta_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
+  if (!layers || !H || !cfg || !aligned16(H)) return DASH_ERR_INVALID_ARG;
+  if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
+  if (cfg->mode != DASH_MODE_PRUNE && cfg->mode != DASH_MODE_HALT && cfg->mode != DASH_MODE_DENSE)
+    return DASH_ERR_INVALID_ARG;
+  if (cfg->mode != DASH_MODE_DENSE) {
+    if (cfg->halt_layer < 0 || cfg->halt_layer >= dims->n_layers) return DASH_ERR_INVALID_ARG;
+    if (cfg->select != DASH_SELECT_TOPK && cfg->select != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
+    if (cfg->score != DASH_SCORE_ABS && cfg->score != DASH_SCORE_REL) return DASH_ERR_INVALID_ARG;
+    if (cfg->select == DASH_SELECT_TOPK && !(cfg->keep_ratio >= 0.0 && cfg->keep_ratio <= 1.0))
+      return DASH_ERR_INVALID_ARG;
+    if (cfg->keep_first < 0 || cfg->keep_last < 0) return DASH_ERR_INVALID_ARG;
+  }
+  for (int l = 0; l < dims->n_layers; ++l)
+    if (!weights_ok(&layers[l])) return DASH_ERR_INVALID_ARG;
+  if (T == 0) {
+    if (K_out) *K_out = 0;
+    return DASH_OK;
+  }
+  const size_t need = dash_prefill_workspace_size(dims, T, cfg);
+  if (!ws || ws_bytes < need) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  PrefillWs P;
+  carve_prefill(*dims, T, c, P);
+  cudaStream_t st = as_stream(stream);
+  bf16* h = reinterpret_cast<bf16*>(H);
+  const dash_dims& D = *dims;
+  if ((s = rope_table(P.L.rope, T, D.head_dim, D.rope_theta, *di, st)) != DASH_OK) return s;
+
+  if (cfg->mode == DASH_MODE_DENSE) {
+    for (int l = 0; l < D.n_layers; ++l)
+      if ((s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, nullptr, 0, P.L, st)) != DASH_OK) return s;
+    if (K_out) *K_out = T;
+    return DASH_OK;
+  }
+
+  // Layers 0..L_s on all T tokens; Δ from the halting layer's o_proj epilogue.
+  const int Ls = cfg->halt_layer;
+  float* delta = delta_out ? delta_out : P.delta;
+  for (int l = 0; l <= Ls; ++l) {
+    if ((s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, l == Ls ? delta : nullptr,
+                        cfg->score == DASH_SCORE_REL, P.L, st)) != DASH_OK)
+      return s;
+  }
+  // One-shot selection of the active set S*.
+  int32_t* idx = idx_out ? idx_out : P.idx;
+  if ((s = select_impl(delta, T, cfg->select, cfg->keep_ratio, cfg->threshold, cfg->keep_first, cfg->keep_last,
+                       idx, P.halted, P.count, st)) != DASH_OK)
+    return s;
+  int32_t K32 = 0;
+  if (cudaMemcpyAsync(&K32, P.count, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  if (K32 < 0) return DASH_ERR_NONFINITE;
+  const int64_t K = K32;
+  if (K_out) *K_out = K;
+
+  // Gather the active rows; later layers run on them only.
+  if ((s = move_rows(false, h, P.Hc, idx, K, T, D.d_model, *di, st)) != DASH_OK) return s;
+  if (cfg->mode == DASH_MODE_PRUNE) {
+    for (int l = Ls + 1; l < D.n_layers; ++l)
+      if ((s = layer_impl(*di, D, layers[l], P.Hc, K, idx, nullptr, nullptr, 0, P.L, st)) != DASH_OK) return s;
+    if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16), cudaMemcpyDeviceToDevice,
+                                 st) != cudaSuccess)
+      return DASH_ERR_CUDA;
+    return DASH_OK;
+  }
+  dash_halt_ctx hc;
+  hc.active_idx = idx;
+  hc.halted_idx = P.halted;
+  hc.h_full = H;
+  hc.T = T;
+  for (int l = Ls + 1; l < D.n_layers; ++l)
+    if ((s = layer_impl(*di, D, layers[l], P.Hc, K, idx, &hc, nullptr, 0, P.L, st)) != DASH_OK) return s;
+  return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
+}
+
+}  // extern "C"

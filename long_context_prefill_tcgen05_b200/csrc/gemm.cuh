@@ -1,0 +1,372 @@
+// Persistent tcgen05 GEMM for sm_100a: D[M, N] = A[M, K] * B[N, K]^T with
+// bf16 operands, fp32 accumulation in tensor memory, and epilogues fused for
+// the decoder block of the DASH prefill path:
+//
+//   kEpiStore     out = D (bf16)
+//   kEpiResid     out = out + D             (residual add, in place)
+//   kEpiResidSsq  out = out + D, plus per-row partial sums of D^2 and out_in^2
+//                 over the tile's columns -> the attention-update norm
+//                 ||U_t||_2 (and ||H_t||_2) of the DASH blog post, §2.1,
+//                 with no extra pass over U
+//   kEpiSwiglu    out = silu(D_gate) * D_up  (B tile = BN/2 gate rows + BN/2 up rows)
+//   kEpiQkv       rotate-half RoPE on q/k heads, split into q / k / v buffers,
+//                 k/v rows optionally remapped (halt mode writes them at the
+//                 tokens' original positions)
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A and B tiles (128B swizzle) into a smem ring
+//   warp 1      TMEM allocator and MMA issuer (one thread issues tcgen05.mma)
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator, fused math, stores
+// The accumulator is double-buffered in TMEM so the epilogue of tile i
+// overlaps the main loop of tile i+1.
+#pragma once
+
+#include "common.cuh"
+
+namespace dash {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kGroupM = 16;  // M tiles per raster group (L2 reuse of B)
+
+enum Epi : int { kEpiStore = 0, kEpiResid = 1, kEpiResidSsq = 2, kEpiSwiglu = 3, kEpiQkv = 4 };
+
+struct EpiArgs {
+  __nv_bfloat16* out;  // store / resid / swiglu destination
+  int64_t ldo;
+  float* ssq_u;  // [tiles_n, M] partial sums of D^2 (kEpiResidSsq)
+  float* ssq_h;  // [tiles_n, M] partial sums of out_in^2
+  __nv_bfloat16* q;
+  __nv_bfloat16* k;
+  __nv_bfloat16* v;
+  int64_t ldq, ldkv;
+  const int32_t* pos;        // RoPE position of row m (NULL: m)
+  const int32_t* kv_rowmap;  // k/v destination row of row m (NULL: m)
+  const float4* rope;        // [max_pos, hd/2] float2 (cos, sin), read as float4 pairs
+  int col_offset;            // qkv column of this GEMM's column 0
+  int hq, hkv, hd;
+};
+
+struct Shape {
+  int M, N, K;
+  int tiles_m, tiles_n, num_tiles;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 8;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarBytes;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+  const int per_group = kGroupM * tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gsize = min(tiles_m - first_m, kGroupM);
+  const int r = t - g * per_group;
+  tm = first_m + r % gsize;
+  tn = r / gsize;
+}
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 w;
+    w.x = pack_bf16(v[8 * i + 0], v[8 * i + 1]);
+    w.y = pack_bf16(v[8 * i + 2], v[8 * i + 3]);
+    w.z = pack_bf16(v[8 * i + 4], v[8 * i + 5]);
+    w.w = pack_bf16(v[8 * i + 6], v[8 * i + 7]);
+    d[i] = w;
+  }
+}
+
+// ----------------------------------------------------------------- epilogues
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, const Shape& sh,
+                                              const EpiArgs& ep) {
+  const bool live = m < sh.M;
+  if constexpr (EPI == kEpiStore || EPI == kEpiResid || EPI == kEpiResidSsq) {
+    float su = 0.f, sq = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + c, r);
+      tmem_ld_wait();
+      if (live) {
+        __nv_bfloat16* p = ep.out + static_cast<int64_t>(m) * ep.ldo + tn * BN + c;
+        float o[32];
+        if constexpr (EPI == kEpiStore) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+        } else {
+          const uint4* hp = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 hv = hp[j];
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float h0 = bf16_lo(hw[e]), h1 = bf16_hi(hw[e]);
+              const float a0 = __uint_as_float(r[8 * j + 2 * e]);
+              const float a1 = __uint_as_float(r[8 * j + 2 * e + 1]);
+              o[8 * j + 2 * e] = h0 + a0;
+              o[8 * j + 2 * e + 1] = h1 + a1;
+              if constexpr (EPI == kEpiResidSsq) {
+                su = fmaf(a0, a0, fmaf(a1, a1, su));
+                sq = fmaf(h0, h0, fmaf(h1, h1, sq));
+              }
+            }
+          }
+        }
+        store32_bf16(p, o);
+      }
+    }
+    if constexpr (EPI == kEpiResidSsq) {
+      if (live) {
+        ep.ssq_u[static_cast<int64_t>(tn) * sh.M + m] = su;
+        ep.ssq_h[static_cast<int64_t>(tn) * sh.M + m] = sq;
+      }
+    }
+  } else if constexpr (EPI == kEpiSwiglu) {
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld32(tbase + c, g);
+      tmem_ld32(tbase + BN / 2 + c, u);
+      tmem_ld_wait();
+      if (live) {
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gf = __uint_as_float(g[i]);
+          o[i] = gf / (1.f + __expf(-gf)) * __uint_as_float(u[i]);
+        }
+        store32_bf16(ep.out + static_cast<int64_t>(m) * ep.ldo + tn * (BN / 2) + c, o);
+      }
+    }
+  } else {  // kEpiQkv
+    const int hd = ep.hd, half = hd >> 1;
+    int p = 0, kvrow = 0;
+    if (live) {
+      p = ep.pos ? ep.pos[m] : m;
+      kvrow = ep.kv_rowmap ? ep.kv_rowmap[m] : m;
+    }
+#pragma unroll 1
+    for (int hb = 0; hb < BN / hd; ++hb) {
+      const int head = (ep.col_offset + tn * BN + hb * hd) / hd;  // warp-uniform
+      __nv_bfloat16* dst;
+      bool rope = true;
+      if (head < ep.hq) {
+        dst = ep.q + static_cast<int64_t>(m) * ep.ldq + head * hd;
+      } else if (head < ep.hq + ep.hkv) {
+        dst = ep.k + static_cast<int64_t>(kvrow) * ep.ldkv + (head - ep.hq) * hd;
+      } else {
+        dst = ep.v + static_cast<int64_t>(kvrow) * ep.ldkv + (head - ep.hq - ep.hkv) * hd;
+        rope = false;
+      }
+      const uint32_t tb = tbase + hb * hd;
+      if (rope) {
+#pragma unroll 1
+        for (int c = 0; c < half; c += 32) {
+          uint32_t x1[32], x2[32];
+          tmem_ld32(tb + c, x1);
+          tmem_ld32(tb + half + c, x2);
+          tmem_ld_wait();
+          if (live) {
+            const float4* cs = ep.rope + ((static_cast<int64_t>(p) * half + c) >> 1);
+            float y1[32], y2[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float4 t = cs[i];  // (cos_2i, sin_2i, cos_2i+1, sin_2i+1)
+              const float a0 = __uint_as_float(x1[2 * i]), b0 = __uint_as_float(x2[2 * i]);
+              const float a1 = __uint_as_float(x1[2 * i + 1]), b1 = __uint_as_float(x2[2 * i + 1]);
+              y1[2 * i] = a0 * t.x - b0 * t.y;
+              y2[2 * i] = b0 * t.x + a0 * t.y;
+              y1[2 * i + 1] = a1 * t.z - b1 * t.w;
+              y2[2 * i + 1] = b1 * t.z + a1 * t.w;
+            }
+            store32_bf16(dst + c, y1);
+            store32_bf16(dst + half + c, y2);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < hd; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tb + c, r);
+          tmem_ld_wait();
+          if (live) {
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+            store32_bf16(dst + c, o);
+          }
+        }
+      }
+    }
+  }
+}
+
+// -------------------------------------------------------------------- kernel
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_b2, const Shape sh, const EpiArgs ep) {
+  using C = Cfg<BN>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain[1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t drain = smem_u32(bars + 2 * S + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 128);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    if (EPI == kEpiSwiglu) prefetch_tmap(&tmap_b2);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nk = sh.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < sh.num_tiles && ok; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, C::kStageBytes);
+          const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
+          tma_load_2d(&tmap_a, a_dst, fb, kb * BK, tm * BM);
+          if constexpr (EPI == kEpiSwiglu) {
+            tma_load_2d(&tmap_b, b_dst, fb, kb * BK, tn * (BN / 2));
+            tma_load_2d(&tmap_b2, b_dst + (BN / 2) * BK * 2, fb, kb * BK, tn * (BN / 2));
+          } else {
+            tma_load_2d(&tmap_b, b_dst, fb, kb * BK, tn * BN);
+          }
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Let every load this thread issued land before the CTA can exit.
+      for (int s = 0; s < S; ++s)
+        if ((armed >> s) & 1u) mbar_wait_drain(full0 + 8 * s, (armed_par >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
+    int stage = 0, local = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < sh.num_tiles && ok; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait(tempty0 + 8 * acc, acc_par ^ 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = umma_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(empty0 + 8 * stage);
+        }
+        __syncwarp();
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(tfull0 + 8 * acc);
+      __syncwarp();
+    }
+    // Every MMA this warp issued must finish before TMEM is released.
+    if (lane == 0) umma_commit(drain);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+  } else {
+    const int wq = warp & 3;  // TMEM lane quarter this warp may access
+    int local = 0;
+    for (int t = blockIdx.x; t < sh.num_tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_par)) break;
+      tc_fence_after();
+      int tm, tn;
+      tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn);
+      const int m = tm * BM + wq * 32 + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + acc * BN;
+      epilogue_tile<BN, EPI>(tbase, m, tn, sh, ep);
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace gemm
+}  // namespace dash

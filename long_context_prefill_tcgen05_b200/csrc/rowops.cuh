@@ -1,0 +1,362 @@
+// Row-wise kernels of the DASH prefill path (SIMT, HBM- or latency-bound):
+// RMSNorm, the Δattn score, its reduction from GEMM-epilogue partial sums,
+// the active-set selection (radix top-k / threshold + ordered compaction),
+// row gather / scatter, and the RoPE cos/sin table.
+#pragma once
+
+#include "common.cuh"
+
+namespace dash {
+namespace rows {
+
+constexpr int kMaxVec = 16;  // 16-byte vectors per lane: rows of up to 4096 bf16
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float sumsq8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a = bf16_lo(w[e]), b = bf16_hi(w[e]);
+    s = fmaf(a, a, fmaf(b, b, s));
+  }
+  return s;
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// y[r] = x[src(r)] * rsqrt(mean(x^2) + eps) * g, one warp per row, fp32 math.
+// src(r) = rowmap[r] when a row map is given (halt mode normalises the frozen
+// rows straight from the full hidden-state buffer).
+__global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_rows,
+                               const int32_t* __restrict__ rowmap, int64_t rows, int d,
+                               const __nv_bfloat16* __restrict__ g, float eps,
+                               __nv_bfloat16* __restrict__ y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  if (r >= rows) return;
+  int64_t src = r;
+  if (rowmap) {
+    src = rowmap[r];
+    if (src < 0 || src >= x_rows) {
+      if (lane == 0) flag_error(kDevErrIndex);
+      return;
+    }
+  }
+  const int nv = d >> 3;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + src * d);
+  uint4 v[kMaxVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nv) {
+      v[i] = xr[c];
+      ss += sumsq8(v[i]);
+    }
+  }
+  ss = warp_sum(ss);
+  const float rs = rsqrtf(ss / static_cast<float>(d) + eps);
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  uint4* yr = reinterpret_cast<uint4*>(y + r * d);
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nv) {
+      const uint4 gv = gr[c];
+      const uint32_t xw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = pack_bf16(bf16_lo(xw[e]) * rs * bf16_lo(gw[e]), bf16_hi(xw[e]) * rs * bf16_hi(gw[e]));
+      yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// -------------------------------------------------------------------- score
+// Δ_t = ||U_t||_2, or ||U_t||_2 / ||H_t||_2 (one warp per row).
+__global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ h,
+                             int64_t T, int d, int relative, float* __restrict__ delta) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  if (r >= T) return;
+  const int nv = d >> 3;
+  const uint4* ur = reinterpret_cast<const uint4*>(u + r * d);
+  float su = 0.f, sh = 0.f;
+#pragma unroll 4
+  for (int c = lane; c < nv; c += 32) su += sumsq8(__ldcs(ur + c));
+  if (relative) {
+    const uint4* hr = reinterpret_cast<const uint4*>(h + r * d);
+#pragma unroll 4
+    for (int c = lane; c < nv; c += 32) sh += sumsq8(__ldcs(hr + c));
+  }
+  su = warp_sum(su);
+  if (relative) sh = warp_sum(sh);
+  if (lane == 0) {
+    const float dl = relative ? sqrtf(su) / sqrtf(sh) : sqrtf(su);
+    if (!isfinite(dl)) flag_error(kDevErrNonfinite);
+    delta[r] = dl;
+  }
+}
+
+// Δ from the o_proj epilogue's per-tile partial sums [ntiles, M], reduced in
+// a fixed order so the result is deterministic.
+__global__ void score_from_ssq_kernel(const float* __restrict__ ssq_u, const float* __restrict__ ssq_h,
+                                      int ntiles, int64_t M, int relative, float* __restrict__ delta) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= M) return;
+  float su = 0.f, sh = 0.f;
+  for (int j = 0; j < ntiles; ++j) su += ssq_u[j * M + t];
+  if (relative)
+    for (int j = 0; j < ntiles; ++j) sh += ssq_h[j * M + t];
+  const float dl = relative ? sqrtf(su) / sqrtf(sh) : sqrtf(su);
+  if (!isfinite(dl)) flag_error(kDevErrNonfinite);
+  delta[t] = dl;
+}
+
+// ------------------------------------------------------------------- select
+// Monotone 32-bit key of an fp32 score: larger score -> larger key; -0 and +0
+// share a key (they compare equal).
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelPerThread = 4;  // consecutive elements per thread in a chunk
+constexpr int kSelChunk = kSelThreads * kSelPerThread;
+
+// Exclusive block-wide prefix sum of one value per thread; also returns the total.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t wv = warp_tot[lane];
+    uint32_t wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_tot[32 + lane] = wi - wv;  // exclusive
+    if (lane == 31) warp_tot[64] = wi;
+  }
+  __syncthreads();
+  const uint32_t res = warp_tot[32 + warp] + incl - v;
+  total = warp_tot[64];
+  __syncthreads();
+  return res;
+}
+
+// Single-CTA selection over T scores.
+//   kind 0 (top-k): among tokens in [lo, hi) choose the k_dyn best by
+//     (score desc, index asc); kind 1 (threshold): score >= thr.
+//   Tokens outside [lo, hi) (the forced first / last tokens) are always kept.
+// Writes the kept indices ascending to idx, the others to halted (optional),
+// and the count to count[0]; a NaN/Inf score writes count = -3 instead.
+// Top-k finds the k-th key by an 8-bit MSB-first radix select over
+// shared-memory histograms, then compacts in index order with block-wide
+// ballot prefix sums; among keys equal to the k-th, the lowest indices win.
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const float* __restrict__ scores, int64_t T, int kind, int64_t k_dyn, float thr,
+                  int64_t lo, int64_t hi, int32_t* __restrict__ idx, int32_t* __restrict__ halted,
+                  int32_t* __restrict__ count) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t warp_tot[65];
+  __shared__ uint32_t s_prefix, s_k;
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  int bad = 0;
+  for (int64_t t = tid; t < T; t += kSelThreads) bad |= !isfinite(scores[t]);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) s_bad = 1;
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      count[0] = -3;
+      flag_error(kDevErrNonfinite);
+    }
+    return;
+  }
+
+  const int64_t n_mid = hi - lo;
+  // mode: 0 none of the middle, 1 all of the middle, 2 radix cut, 3 threshold
+  int mode;
+  if (kind == 1) mode = 3;
+  else if (k_dyn <= 0) mode = 0;
+  else if (k_dyn >= n_mid) mode = 1;
+  else mode = 2;
+
+  uint32_t kth = 0, k_rem = 0;
+  if (mode == 2) {
+    uint32_t prefix = 0, mask = 0, k = static_cast<uint32_t>(k_dyn);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
+      __syncthreads();
+      for (int64_t base = lo; base < hi; base += kSelThreads) {
+        const int64_t t = base + tid;
+        const bool in = t < hi;
+        uint32_t key = in ? score_key(scores[t]) : 0u;
+        const bool match = in && ((key & mask) == prefix);
+        const uint32_t bin = (key >> shift) & 255u;
+        const uint32_t active = __ballot_sync(0xffffffffu, match);
+        if (match) {
+          const uint32_t peers = __match_any_sync(active, bin);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins [8l, 8l + 8); find the bin holding the k-th largest
+        uint32_t cnt[8], own = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          cnt[i] = hist[8 * lane + i];
+          own += cnt[i];
+        }
+        uint32_t above = 0;  // keys in bins of higher lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_down_sync(0xffffffffu, above + own, o);
+          // accumulate suffix sums of `own` over lanes > lane
+          (void)n;
+        }
+        // plain suffix sum: incl[l] = sum_{l' >= l} own[l']
+        uint32_t incl = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += n;
+        }
+        above = incl - own;
+        if (above < k && k <= incl) {
+          uint32_t acc = above;
+          int b = 7;
+          for (; b > 0; --b) {
+            if (acc + cnt[b] >= k) break;
+            acc += cnt[b];
+          }
+          s_prefix = prefix | (static_cast<uint32_t>(8 * lane + b) << shift);
+          s_k = k - acc;
+        }
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      k = s_k;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    kth = prefix;
+    k_rem = k;  // how many keys equal to kth (lowest indices first) are taken
+  }
+
+  // Ordered compaction, kSelChunk consecutive tokens per round.
+  uint32_t sel_base = 0, hal_base = 0, eq_base = 0;
+  for (int64_t c0 = 0; c0 < T; c0 += kSelChunk) {
+    const int64_t t0 = c0 + static_cast<int64_t>(tid) * kSelPerThread;
+    bool gt[kSelPerThread], eq[kSelPerThread], valid[kSelPerThread], forced[kSelPerThread];
+    uint32_t n_eq = 0;
+#pragma unroll
+    for (int i = 0; i < kSelPerThread; ++i) {
+      const int64_t t = t0 + i;
+      valid[i] = t < T;
+      forced[i] = valid[i] && (t < lo || t >= hi);
+      gt[i] = eq[i] = false;
+      if (valid[i] && !forced[i]) {
+        const float s = scores[t];
+        if (mode == 1) gt[i] = true;
+        else if (mode == 3) gt[i] = s >= thr;
+        else if (mode == 2) {
+          const uint32_t key = score_key(s);
+          gt[i] = key > kth;
+          eq[i] = key == kth;
+        }
+      }
+      n_eq += eq[i];
+    }
+    uint32_t tot_eq;
+    uint32_t eq_rank = eq_base + block_excl_scan(n_eq, warp_tot, tot_eq);
+    bool sel[kSelPerThread];
+    uint32_t n_sel = 0, n_hal = 0;
+#pragma unroll
+    for (int i = 0; i < kSelPerThread; ++i) {
+      bool take_eq = false;
+      if (eq[i]) {
+        take_eq = eq_rank < k_rem;
+        ++eq_rank;
+      }
+      sel[i] = valid[i] && (forced[i] || gt[i] || take_eq);
+      n_sel += sel[i];
+      n_hal += valid[i] && !sel[i];
+    }
+    uint32_t tot_pk;
+    const uint32_t pk = block_excl_scan((n_sel << 16) | n_hal, warp_tot, tot_pk);
+    uint32_t ps = sel_base + (pk >> 16), ph = hal_base + (pk & 0xffffu);
+#pragma unroll
+    for (int i = 0; i < kSelPerThread; ++i) {
+      if (!valid[i]) continue;
+      if (sel[i]) idx[ps++] = static_cast<int32_t>(t0 + i);
+      else if (halted) halted[ph++] = static_cast<int32_t>(t0 + i);
+    }
+    sel_base += tot_pk >> 16;
+    hal_base += tot_pk & 0xffffu;
+    eq_base += tot_eq;
+  }
+  if (tid == 0) count[0] = static_cast<int32_t>(sel_base);
+}
+
+// -------------------------------------------------------- gather / scatter
+// Y[i] = X[idx[i]] (gather) or X[idx[i]] = Y[i] (scatter); one warp per row.
+template <bool kScatter>
+__global__ void move_rows_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                 const int32_t* __restrict__ idx, int64_t K, int64_t T, int d) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int nv = d >> 3;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * wpb + warp; i < K; i += gridDim.x * wpb) {
+    const int64_t t = idx[i];
+    if (t < 0 || t >= T) {
+      if (lane == 0) flag_error(kDevErrIndex);
+      continue;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(src + (kScatter ? i : t) * d);
+    uint4* o = reinterpret_cast<uint4*>(dst + (kScatter ? t : i) * d);
+#pragma unroll 4
+    for (int c = lane; c < nv; c += 32) o[c] = __ldcs(s + c);
+  }
+}
+
+// ------------------------------------------------------------- RoPE table
+// tab[p * half + i] = (cos, sin) of p * theta^(-2i / (2 half)), evaluated in
+// fp64 and rounded to fp32.
+__global__ void rope_table_kernel(float2* __restrict__ tab, int64_t max_pos, int half, double theta) {
+  const int64_t n = max_pos * half;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = e / half;
+    const int i = static_cast<int>(e - p * half);
+    const double inv = pow(theta, -2.0 * i / (2.0 * half));
+    double s, c;
+    sincos(static_cast<double>(p) * inv, &s, &c);
+    tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  }
+}
+
+}  // namespace rows
+}  // namespace dash

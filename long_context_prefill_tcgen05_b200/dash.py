@@ -1,0 +1,258 @@
+"""ctypes binding of libdash.so (include/dash.h, include/dash_ops.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers
+plus sizes, torch supplies memory and the current stream, and every step of
+the path runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing, ``lib()`` raises.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+from .build import LIB, INCLUDE
+
+c_i32, c_i64, c_f32, c_f64, c_vp, c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                          ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t)
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "non-finite score",
+          4: "workspace too small", 5: "CUDA error", 6: "device wait timed out",
+          7: "index out of range"}
+MODES = {"prune": 0, "halt": 1, "dense": 2}
+SELECTS = {"topk": 0, "threshold": 1}
+
+
+class DashError(RuntimeError):
+    def __init__(self, status, what=""):
+        super().__init__(f"{what}: dash status {status} ({STATUS.get(status, '?')})")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("n_layers", c_i32), ("d_model", c_i32), ("n_heads", c_i32), ("n_kv_heads", c_i32),
+                ("head_dim", c_i32), ("ffn_dim", c_i32), ("rms_eps", c_f64), ("rope_theta", c_f64)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, c_vp) for n in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_gate", "w_up", "w_down")]
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("halt_layer", c_i32), ("mode", c_i32), ("select", c_i32), ("score", c_i32),
+                ("keep_ratio", c_f64), ("threshold", c_f32), ("keep_first", c_i32), ("keep_last", c_i32)]
+
+
+class HaltCtx(ctypes.Structure):
+    _fields_ = [("active_idx", c_vp), ("halted_idx", c_vp), ("h_full", c_vp), ("T", c_i64)]
+
+
+_SIGS = {
+    "dash_status_string": (ctypes.c_char_p, [c_i32]),
+    "dash_device_error": (c_i32, []),
+    "dash_score": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp]),
+    "dash_topk_count": (c_i64, [c_i64, c_f64, c_i32, c_i32]),
+    "dash_select_workspace_size": (c_sz, [c_i64]),
+    "dash_select": (c_i32, [c_vp, c_i64, c_i32, c_f64, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "dash_compact": (c_i32, [c_vp, c_i64, c_vp, c_i64, c_i32, c_vp, c_vp]),
+    "dash_scatter": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp, c_i64, c_vp]),
+    "dash_layer_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i64, c_i64, c_i64]),
+    "dash_layer_forward": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, c_vp, c_i64,
+                                   ctypes.POINTER(HaltCtx), c_vp, c_i32, c_vp, c_sz, c_vp]),
+    "dash_prefill_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i64, ctypes.POINTER(Config)]),
+    "dash_prefill": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, ctypes.POINTER(Config),
+                             c_vp, ctypes.POINTER(c_i64), c_vp, c_vp, c_sz, c_vp]),
+    "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
+    "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
+    "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+}
+
+_LIB = None
+
+
+def lib():
+    """Loads libdash.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"{LIB} is missing; build it with "
+                               "`python -m long_context_prefill_tcgen05_b200.build`")
+        L = ctypes.CDLL(LIB)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def declared_symbols():
+    """Every dash_* function declared in include/*.h."""
+    names = set()
+    for fn in os.listdir(INCLUDE):
+        if fn.endswith(".h"):
+            with open(os.path.join(INCLUDE, fn)) as f:
+                names |= set(re.findall(r"\b(dash_[a-z_0-9]+)\s*\(", f.read()))
+    return sorted(names)
+
+
+def _check(status, what):
+    if status != 0:
+        raise DashError(status, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def device_error():
+    """Reads and clears the library's sticky device error (synchronises)."""
+    return lib().dash_device_error()
+
+
+def check_device():
+    _check(device_error(), "device")
+
+
+# ----------------------------------------------------------- workspaces
+_WS = {}
+
+
+def workspace(nbytes, device):
+    """A cached uint8 device buffer of at least nbytes (reused across calls)."""
+    key = str(device)
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < nbytes:
+        _WS[key] = buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    return buf
+
+
+def release_workspaces():
+    _WS.clear()
+
+
+# ------------------------------------------------------------- row ops
+def score(U, H=None, relative=False, out=None, stream=None):
+    T, d = U.shape
+    out = torch.empty(T, dtype=torch.float32, device=U.device) if out is None else out
+    _check(lib().dash_score(_p(U), _p(H), T, d, int(relative), _p(out), _stream(stream)), "dash_score")
+    return out
+
+
+def topk_count(T, keep, keep_first=0, keep_last=0):
+    return lib().dash_topk_count(T, keep, keep_first, keep_last)
+
+
+def select(scores, kind="topk", keep=0.5, threshold=0.0, keep_first=0, keep_last=0, want_halted=False,
+           stream=None):
+    """Returns (idx [count] int32, halted [T-count] or None, count) after a sync."""
+    T = scores.numel()
+    dev = scores.device
+    idx = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
+    halted = torch.empty(max(T, 1), dtype=torch.int32, device=dev) if want_halted else None
+    count = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(lib().dash_select(_p(scores), T, SELECTS[kind], keep, threshold, keep_first, keep_last, _p(idx),
+                             _p(halted), _p(count), None, 0, _stream(stream)), "dash_select")
+    n = int(count.item())
+    if n < 0:
+        raise DashError(-n, "dash_select")
+    return idx[:n], (halted[:T - n] if want_halted else None), n
+
+
+def compact(X, idx, stream=None):
+    K = idx.numel()
+    Y = torch.empty(K, X.shape[1], dtype=X.dtype, device=X.device)
+    _check(lib().dash_compact(_p(X), X.shape[0], _p(idx), K, X.shape[1], _p(Y), _stream(stream)), "dash_compact")
+    return Y
+
+
+def scatter(Y, idx, X, stream=None):
+    _check(lib().dash_scatter(_p(Y), _p(idx), idx.numel(), X.shape[1], _p(X), X.shape[0], _stream(stream)),
+           "dash_scatter")
+    return X
+
+
+def rmsnorm(X, g, eps, stream=None):
+    Y = torch.empty_like(X)
+    _check(lib().dash_rmsnorm(_p(X), X.shape[0], X.shape[1], _p(g), eps, _p(Y), _stream(stream)), "dash_rmsnorm")
+    return Y
+
+
+def linear(A, W, out=None, stream=None):
+    M, K = A.shape
+    N = W.shape[0]
+    out = torch.empty(M, N, dtype=A.dtype, device=A.device) if out is None else out
+    _check(lib().dash_linear(_p(A), M, K, _p(W), N, _p(out), _stream(stream)), "dash_linear")
+    return out
+
+
+def attention(Q, K, V, hq, hkv, hd, qpos=None, out=None, stream=None):
+    M = Q.shape[0]
+    out = torch.empty(M, hq * hd, dtype=Q.dtype, device=Q.device) if out is None else out
+    _check(lib().dash_attention(_p(Q), _p(K), _p(V), M, K.shape[0], hq, hkv, hd, _p(qpos), _p(out),
+                                _stream(stream)), "dash_attention")
+    return out
+
+
+# --------------------------------------------------------------- stack
+class Stack:
+    """A decoder stack's dims plus its weights laid out for the library
+    (w_qkv = [wq; wk; wv] concatenated once, at load time)."""
+
+    def __init__(self, dims, layers):
+        self.model = dims
+        self.dims = Dims(dims.n_layers if len(layers) == dims.n_layers else len(layers), dims.d_model,
+                         dims.n_heads, dims.n_kv_heads, dims.head_dim, dims.ffn_dim, dims.rms_eps,
+                         dims.rope_theta)
+        self.tensors = []
+        arr = (LayerWeights * len(layers))()
+        for i, w in enumerate(layers):
+            qkv = torch.cat([w["wq"], w["wk"], w["wv"]], 0).contiguous()
+            keep = [w["attn_norm"].contiguous(), qkv, w["wo"].contiguous(), w["ffn_norm"].contiguous(),
+                    w["wg"].contiguous(), w["wu"].contiguous(), w["wd"].contiguous()]
+            self.tensors.append(keep)
+            arr[i] = LayerWeights(*[t.data_ptr() for t in keep])
+        self.layers = arr
+        self.n_layers = len(layers)
+
+
+def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, relative=False, stream=None):
+    """One block in place on H [M, d].  halt = (active_idx, halted_idx, h_full) or None."""
+    M = H.shape[0]
+    T_kv = M
+    hctx = None
+    if halt is not None:
+        active, halted, h_full = halt
+        T_kv = h_full.shape[0]
+        hctx = HaltCtx(active.data_ptr(), halted.data_ptr() if halted.numel() else None, h_full.data_ptr(), T_kv)
+        pos = active
+    if max_pos is None:
+        max_pos = T_kv
+    need = lib().dash_layer_workspace_size(ctypes.byref(stack.dims), M, T_kv, max_pos)
+    ws = workspace(need, H.device)
+    w = ctypes.pointer(stack.layers[l])
+    _check(lib().dash_layer_forward(ctypes.byref(stack.dims), w, _p(H), M, _p(pos), max_pos,
+                                    ctypes.byref(hctx) if hctx is not None else None, _p(delta), int(relative),
+                                    _p(ws), ws.numel(), _stream(stream)), "dash_layer_forward")
+    return H
+
+
+def make_config(halt_layer=0, mode="prune", select="topk", keep=0.5, threshold=0.0, relative=False,
+                keep_first=0, keep_last=0):
+    return Config(halt_layer, MODES[mode], SELECTS[select], int(relative), keep, threshold, keep_first, keep_last)
+
+
+def prefill(stack, H, cfg, idx_out=None, delta_out=None, stream=None):
+    """Runs dash_prefill in place on H [T, d]; returns K (the active count)."""
+    T = H.shape[0]
+    need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
+    ws = workspace(need, H.device)
+    K = c_i64(0)
+    _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _p(H), T, ctypes.byref(cfg), _p(idx_out),
+                              ctypes.byref(K), _p(delta_out), _p(ws), ws.numel(), _stream(stream)), "dash_prefill")
+    return K.value

@@ -1,0 +1,105 @@
+"""C-ABI boundary checks that need no GPU: the library builds and loads,
+exports every symbol the headers declare, and its host-side arithmetic and
+argument checks behave (no kernel is launched by any call here)."""
+import ctypes
+import math
+
+import pytest
+
+import oracle as O
+from long_context_prefill_tcgen05_b200 import build, dash, inputs
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return dash.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = dash.declared_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, text in dash.STATUS.items():
+        assert L.dash_status_string(code).decode() == text
+
+
+@pytest.mark.parametrize("T", [0, 1, 7, 100, 512, 32768, 131072])
+@pytest.mark.parametrize("keep", [0.0, 0.1, 0.333, 0.4, 0.5, 0.7, 1.0])
+@pytest.mark.parametrize("nf,nl", [(0, 0), (64, 32), (3, 0), (0, 5), (200, 200)])
+def test_topk_count_matches_oracle(L, T, keep, nf, nl):
+    assert dash.topk_count(T, keep, nf, nl) == (O.topk_count(T, keep, nf, nl) if T > 0 else 0)
+
+
+FAKE = 1 << 20  # an aligned non-null address; the calls below fail before using it
+
+
+def _dims(**kw):
+    d = inputs.TINY
+    base = dict(n_layers=d.n_layers, d_model=d.d_model, n_heads=d.n_heads, n_kv_heads=d.n_kv_heads,
+                head_dim=d.head_dim, ffn_dim=d.ffn_dim, rms_eps=d.rms_eps, rope_theta=d.rope_theta)
+    base.update(kw)
+    return dash.Dims(**base)
+
+
+def _fake_layers(n):
+    arr = (dash.LayerWeights * n)()
+    for i in range(n):
+        arr[i] = dash.LayerWeights(*([FAKE] * 7))
+    return arr
+
+
+def test_argument_errors_are_caught_on_the_host(L):
+    dims = _dims()
+    cfg = dash.make_config(halt_layer=2, mode="prune", keep=0.5)
+    layers = _fake_layers(4)
+    K = ctypes.c_int64(0)
+    call = lambda d, lay, H, T, c, ws=None, wsb=0: L.dash_prefill(
+        ctypes.byref(d), lay, H, T, ctypes.byref(c), None, ctypes.byref(K), None, ws, wsb, None)
+    assert call(dims, layers, None, 512, cfg) == 1                       # null H
+    assert call(_dims(head_dim=96), layers, FAKE, 512, cfg) == 2         # unsupported head_dim
+    assert call(_dims(n_heads=3), layers, FAKE, 512, cfg) == 2           # hq % hkv != 0
+    assert call(_dims(d_model=200), layers, FAKE, 512, cfg) == 2         # d % 128 != 0
+    assert call(dims, layers, FAKE + 2, 512, cfg) == 1                   # misaligned H
+    bad = dash.make_config(halt_layer=4, mode="prune")
+    assert call(dims, layers, FAKE, 512, bad) == 1                       # halt layer out of range
+    bad = dash.make_config(halt_layer=1, keep=1.5)
+    assert call(dims, layers, FAKE, 512, bad) == 1                       # keep > 1
+    bad = dash.make_config(halt_layer=1); bad.mode = 9
+    assert call(dims, layers, FAKE, 512, bad) == 1                       # unknown mode
+    holes = _fake_layers(4); holes[3] = dash.LayerWeights(*([FAKE] * 6 + [0]))
+    assert call(dims, holes, FAKE, 512, cfg) == 1                        # a null weight
+    assert call(dims, layers, FAKE, 512, cfg, None, 0) == 4              # no workspace
+    need = L.dash_prefill_workspace_size(ctypes.byref(dims), 512, ctypes.byref(cfg))
+    assert call(dims, layers, FAKE, 512, cfg, FAKE, need - 1) == 4       # workspace one byte short
+    assert call(dims, layers, FAKE, 0, cfg) == 0 and K.value == 0        # empty input: nothing to do
+
+    # select / score / compact shape and argument checks
+    cnt = FAKE
+    assert L.dash_select(FAKE, 10, 7, 0.5, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 1
+    assert L.dash_select(FAKE, 10, 0, -0.1, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 1
+    assert L.dash_select(FAKE, 10, 0, 0.5, 0.0, -1, 0, FAKE, None, cnt, None, 0, None) == 1
+    assert L.dash_select(None, 10, 0, 0.5, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 1
+    assert L.dash_score(FAKE, None, 10, 7, 0, FAKE, None) == 2
+    assert L.dash_score(FAKE, None, 10, 64, 1, FAKE, None) == 1          # relative needs H
+    assert L.dash_compact(FAKE, 10, FAKE, 5, 12, FAKE, None) == 2
+    assert L.dash_linear(FAKE, 10, 100, FAKE, 128, FAKE, None) == 2      # K % 64
+    assert L.dash_attention(FAKE, FAKE, FAKE, 10, 10, 4, 2, 96, None, FAKE, None) == 2
+    assert L.dash_attention(FAKE, FAKE, FAKE, 20, 10, 4, 2, 64, None, FAKE, None) == 2  # M > T_kv causal
+
+
+def test_workspace_sizes_grow_with_tokens(L):
+    dims = _dims()
+    cfg = dash.make_config(halt_layer=2)
+    sizes = [L.dash_prefill_workspace_size(ctypes.byref(dims), T, ctypes.byref(cfg)) for T in (1, 512, 4096)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    q = inputs.QWEN7B
+    qd = dash.Dims(q.n_layers, q.d_model, q.n_heads, q.n_kv_heads, q.head_dim, q.ffn_dim, q.rms_eps, q.rope_theta)
+    big = L.dash_prefill_workspace_size(ctypes.byref(qd), 32768, ctypes.byref(cfg))
+    # activations for T = 32768 fit well inside one GPU's memory
+    assert 1 << 30 < big < 8 << 30
+    assert L.dash_layer_workspace_size(ctypes.byref(dims), 100, 50, 100) == 0  # T_kv < M rejected

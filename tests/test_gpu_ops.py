@@ -1,0 +1,166 @@
+"""GPU parity of the building-block kernels against the CPU oracle, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from long_context_prefill_tcgen05_b200 import dash, inputs
+from conftest import to_np, row_rel_err, elem_rel_err, DELTA_TOL
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _no_device_error():
+    assert dash.device_error() == 0
+
+
+# ------------------------------------------------------------------ score
+@pytest.mark.parametrize("relative", [False, True])
+@pytest.mark.parametrize("T,d", [(1, 256), (777, 3584), (4096, 4096)])
+def test_score_matches_oracle(gpu_lib, T, d, relative):
+    U, H, _ = inputs.make_score_bench_inputs(T=T, d=d, seed=3)
+    got = dash.score(U.to(DEV), H.to(DEV), relative=relative).cpu().numpy()
+    ref = O.delta_scores(to_np(U), to_np(H), relative)
+    assert np.max(np.abs(got - ref) / ref) < 1e-5  # fp32 sums of bf16 values
+    assert np.max(np.abs(got - ref) / ref) < DELTA_TOL
+    _no_device_error()
+
+
+# ----------------------------------------------------------------- select
+KINDS = ["random", "all_equal", "few_values", "signed_zero", "denormal", "negative", "spiky"]
+
+
+def _check_select(s, kind, keep=0.5, thr=0.0, nf=0, nl=0):
+    sd = s.to(DEV)
+    idx, halted, n = dash.select(sd, kind, keep, thr, nf, nl, want_halted=True)
+    ref = (O.select_topk(s.double().numpy(), keep, nf, nl) if kind == "topk"
+           else O.select_threshold(s.double().numpy(), float(np.float32(thr)), nf, nl))
+    got = idx.cpu().numpy()
+    assert n == len(ref)
+    assert np.array_equal(got, ref)
+    comp = np.setdiff1d(np.arange(len(s)), ref)
+    assert np.array_equal(halted.cpu().numpy(), comp)
+
+
+@pytest.mark.parametrize("pattern", KINDS)
+@pytest.mark.parametrize("T", [1, 33, 1000, 4097, 32768, 100003])
+def test_select_topk_bit_exact(gpu_lib, pattern, T):
+    s = inputs.adversarial_scores(pattern, T, seed=T)
+    for keep in (0.0, 1.0 / T, 0.5, 0.9, (T - 1) / T, 1.0):
+        _check_select(s, "topk", keep)
+    _check_select(s, "topk", 0.5, nf=64, nl=32)
+    _check_select(s, "topk", 0.3, nf=T, nl=5)
+    _no_device_error()
+
+
+@pytest.mark.parametrize("pattern", KINDS)
+@pytest.mark.parametrize("T", [1, 1000, 32768])
+def test_select_threshold_bit_exact(gpu_lib, pattern, T):
+    s = inputs.adversarial_scores(pattern, T, seed=T + 1)
+    vals = s.numpy()
+    for thr in (float(np.median(vals)), float(vals.max()), 0.0, float(vals[T // 2])):
+        _check_select(s, "threshold", thr=thr)
+    _check_select(s, "threshold", thr=float(np.median(vals)), nf=10, nl=10)
+    _no_device_error()
+
+
+def test_select_nonfinite_is_an_error(gpu_lib):
+    for bad in (float("nan"), float("inf"), -float("inf")):
+        s = torch.rand(5000)
+        s[1234] = bad
+        with pytest.raises(dash.DashError) as e:
+            dash.select(s.to(DEV), "topk", 0.5)
+        assert e.value.status == 3
+        assert dash.device_error() == 3  # reported and cleared
+    _no_device_error()
+
+
+def test_select_empty(gpu_lib):
+    idx, _, n = dash.select(torch.empty(0, device=DEV), "topk", 0.5)
+    assert n == 0
+
+
+# ------------------------------------------------------- compact / scatter
+@pytest.mark.parametrize("T,d,K", [(1, 256, 1), (5000, 3584, 2500), (33000, 4096, 7)])
+def test_compact_scatter_bit_exact(gpu_lib, T, d, K):
+    g = torch.Generator().manual_seed(T)
+    X = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    idx = torch.sort(torch.randperm(T, generator=g)[:K]).values.to(torch.int32)
+    Y = dash.compact(X.to(DEV), idx.to(DEV))
+    assert torch.equal(Y.cpu(), X[idx.long()])
+    Z = X.clone().to(DEV)
+    dash.scatter((Y * 2).contiguous(), idx.to(DEV), Z)
+    ref = X.clone()
+    ref[idx.long()] = X[idx.long()] * 2
+    assert torch.equal(Z.cpu(), ref)
+    _no_device_error()
+
+
+def test_compact_bad_index_sets_device_error(gpu_lib):
+    X = torch.randn(100, 256, device=DEV).to(torch.bfloat16)
+    idx = torch.tensor([3, 100], dtype=torch.int32, device=DEV)   # 100 is out of range
+    dash.compact(X, idx)
+    assert dash.device_error() == 7
+    _no_device_error()
+
+
+# ----------------------------------------------------------------- RMSNorm
+@pytest.mark.parametrize("M,d", [(1, 256), (1000, 3584), (300, 4096)])
+def test_rmsnorm_matches_oracle(gpu_lib, M, d):
+    g = torch.Generator().manual_seed(M)
+    X = (torch.randn(M, d, generator=g) * 3).to(torch.bfloat16)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16)
+    got = dash.rmsnorm(X.to(DEV), w.to(DEV), 1e-6).cpu()
+    ref = O.rms_norm(to_np(X), to_np(w), 1e-6)
+    assert row_rel_err(to_np(got), ref) < 8e-3   # bf16 output rounding
+    _no_device_error()
+
+
+# ----------------------------------------------------------- tcgen05 GEMM
+@pytest.mark.parametrize("M,K,N", [(128, 64, 128), (1, 256, 512), (300, 3584, 4608), (1000, 704, 256),
+                                   (129, 18944, 256), (2048, 3584, 3584)])
+def test_linear_matches_fp64(gpu_lib, M, K, N):
+    g = torch.Generator().manual_seed(M * 7 + N)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    got = dash.linear(A.to(DEV), W.to(DEV)).cpu()
+    ref = to_np(A) @ to_np(W).T
+    assert elem_rel_err(to_np(got), ref) < 1e-2
+    assert row_rel_err(to_np(got), ref) < 5e-3
+    _no_device_error()
+
+
+# -------------------------------------------------------------- attention
+def _attn_case(M, T_kv, hq, hkv, hd, qpos, seed):
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(M, hq * hd, generator=g).to(torch.bfloat16)
+    K = torch.randn(T_kv, hkv * hd, generator=g).to(torch.bfloat16)
+    V = torch.randn(T_kv, hkv * hd, generator=g).to(torch.bfloat16)
+    qp = None if qpos is None else torch.tensor(qpos, dtype=torch.int32)
+    got = dash.attention(Q.to(DEV), K.to(DEV), V.to(DEV), hq, hkv, hd,
+                         None if qp is None else qp.to(DEV)).cpu()
+    q_pos = np.arange(M) if qpos is None else np.asarray(qpos)
+    ref = O.causal_gqa_attention(to_np(Q).reshape(M, hq, hd), to_np(K).reshape(T_kv, hkv, hd),
+                                 to_np(V).reshape(T_kv, hkv, hd), q_pos, np.arange(T_kv)).reshape(M, -1)
+    return to_np(got), ref
+
+
+@pytest.mark.parametrize("M,hq,hkv,hd", [(1, 4, 2, 64), (300, 4, 2, 64), (128, 7, 1, 128), (700, 28, 4, 128),
+                                         (1030, 8, 2, 128)])
+def test_attention_causal_matches_oracle(gpu_lib, M, hq, hkv, hd):
+    got, ref = _attn_case(M, M, hq, hkv, hd, None, seed=M + hq)
+    assert row_rel_err(got.reshape(M * hq, hd), ref.reshape(M * hq, hd)) < 2e-2
+    assert elem_rel_err(got, ref) < 2e-2
+    _no_device_error()
+
+
+@pytest.mark.parametrize("M,T_kv,hq,hkv,hd", [(150, 500, 4, 2, 64), (260, 2000, 7, 1, 128), (1, 300, 4, 2, 64)])
+def test_attention_indexed_queries_match_oracle(gpu_lib, M, T_kv, hq, hkv, hd):
+    rng = np.random.default_rng(M)
+    qpos = np.sort(rng.choice(T_kv, M, replace=False))
+    got, ref = _attn_case(M, T_kv, hq, hkv, hd, qpos, seed=T_kv)
+    assert row_rel_err(got.reshape(M * hq, hd), ref.reshape(M * hq, hd)) < 2e-2
+    _no_device_error()
