@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""DASH long-context prefill benchmark on B200: prefill tokens/s, halted vs dense.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen7b-32k]
+                    [--mode prune|halt] [--impl ours|reference]
+
+One step = one full prefill (all layers, selection, compaction) of one
+synthetic sequence through libdash's C ABI, inputs resident in HBM.  The
+headline `value` is the halted (DASH) prefill; the same kernels without
+halting give the dense figure.  With N > 1 (torchrun), every rank runs an
+independent replica (the path has no data-parallel exchange) and the time is
+the max over ranks.  Prints ONE JSON line on rank 0.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_prefill_tcgen05_b200 import costs, inputs  # noqa: E402
+
+WORKLOADS = {
+    "qwen7b-32k": dict(dims=inputs.QWEN7B, T=32768, halt_layer=11, keep=0.5, select="topk", relative=False,
+                       span_rows=0, span_len=64,
+                       name="Qwen2.5-7B-shaped stack (28 layers, d=3584, 28q/4kv, hd=128, FFN 18944), "
+                            "T=32768, halt at layer 11, keep 0.5"),
+    "qwen7b-128k": dict(dims=inputs.QWEN7B, T=131072, halt_layer=11, keep=0.3, select="topk", relative=True,
+                        span_rows=6528, span_len=128,
+                        name="Qwen2.5-7B-shaped stack, T=131072, halt at layer 11, relative delta, keep 0.3"),
+    "tiny": dict(dims=inputs.TINY, T=512, halt_layer=2, keep=0.5, select="topk", relative=False, span_rows=0,
+                 span_len=64, name="tiny decoder stack (4 layers, d=256, 4q/2kv, hd=64, FFN 704), T=512"),
+}
+METRIC = "prefill tokens/s @T=32K/128K, halted vs dense, and % of B200 roofline"
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# -------------------------------------------------------------- CPU side
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        if blas:
+            return int(max(blas))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample_time(dims, layer_np, T_s, seed=0):
+    """Seconds for the oracle to run one Qwen-shaped decoder block on T_s tokens."""
+    import numpy as np
+    import oracle as O
+    h = inputs.make_hidden(T_s, dims.d_model, seed=seed)[0].double().numpy()
+    pos = np.arange(T_s)
+    t0 = time.perf_counter()
+    O.decoder_block(h, pos, h, pos, layer_np, dims.as_dict())
+    return time.perf_counter() - t0
+
+
+def cpu_layer_np(dims):
+    layer = inputs.make_layers(dims, seed=0, device="cpu", n_layers=1)[0]
+    return {k: v.double().numpy() for k, v in layer.items()}
+
+
+def cpu_baseline(dims, T, target_flops, budget_s=15.0):
+    """The oracle timed on host cores on a bounded sample (one decoder block
+    on T_s tokens), extrapolated by algorithmic FLOPs to the whole workload."""
+    layer_np = cpu_layer_np(dims)
+    lin = costs.linear_flops_per_token(dims)
+    T_s, t = 32, oracle_sample_time(dims, layer_np, 32)
+    while t < budget_s / 4 and T_s < 2048:
+        T_s = min(2048, int(T_s * max(2.0, budget_s / 2 / max(t, 1e-3))))
+        t = oracle_sample_time(dims, layer_np, T_s)
+    f_s = T_s * lin + costs.attn_flops(dims, costs.causal_pairs(T_s))
+    est_s = t * target_flops / f_s
+    return {"value": T / est_s, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"one decoder block of the same stack on {T_s} tokens ({f_s / 1e9:.0f} GFLOP fp64, "
+                      f"{t:.1f} s), extrapolated by algorithmic FLOPs to the full prefill",
+            "sample_seconds": t}
+
+
+# ------------------------------------------------------------ reference
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    dims, T = wl["dims"], wl["T"]
+    K = math.floor(wl["keep"] * T)
+    target = costs.prefill_flops(dims, T, wl["halt_layer"], K, "prune")
+    layer_np = cpu_layer_np(dims)
+    T_s = 64 if dims.d_model > 1024 else T
+    lin = costs.linear_flops_per_token(dims)
+    f_s = T_s * lin + costs.attn_flops(dims, costs.causal_pairs(T_s))
+    for _ in range(args.warmup):
+        oracle_sample_time(dims, layer_np, T_s)
+    ts = [oracle_sample_time(dims, layer_np, T_s) for _ in range(args.steps)]
+    t = sum(ts) / len(ts)
+    value = T / (t * target / f_s)
+    cb = {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+          "sample": f"each step: one decoder block on {T_s} tokens ({f_s / 1e9:.1f} GFLOP fp64), "
+                    f"extrapolated by algorithmic FLOPs to the full halted prefill"}
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+                      "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": t * target / f_s * 1e3, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                      "config": {"workload": wl["name"], "seq_len": T, "halt_layer": wl["halt_layer"],
+                                 "keep": wl["keep"], "mode": "prune"},
+                      "cpu_baseline": cb,
+                      "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+
+
+# ------------------------------------------------------------------ ours
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="qwen7b-32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--mode", default="prune", choices=["prune", "halt"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the dense / other-mode / e2e legs")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    from long_context_prefill_tcgen05_b200 import build, dash
+    if rank == 0:
+        build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    dims, T = wl["dims"], wl["T"]
+    peaks = load_peaks()
+
+    stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev))
+    h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=dev, span_rows=wl["span_rows"],
+                               span_len=wl["span_len"])
+    H = torch.empty_like(h0)
+    idx = torch.empty(T, dtype=torch.int32, device=dev)
+    delta = torch.empty(T, dtype=torch.float32, device=dev)
+    cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select=wl["select"], keep=wl["keep"],
+                           relative=wl["relative"])
+    cfg_dense = dash.make_config(mode="dense")
+
+    def step(c):
+        H.copy_(h0)
+        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
+
+    def timed(c, k, record=False):
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if record:
+            dash.timing_start()
+        e0.record()
+        K = None
+        for _ in range(k):
+            K = step(c)
+        e1.record()
+        torch.cuda.synchronize()
+        recs = dash.timing_stop() if record else None
+        barrier(world)
+        return max_over_ranks(e0.elapsed_time(e1) / k, world), K, recs
+
+    for _ in range(args.warmup):
+        step(cfg)
+    dash.check_device()
+    clock = ClockSampler(local)
+    clock.start()
+    ms, K, recs = timed(cfg, args.steps, record=True)
+    clocks = clock.stop()
+    dash.check_device()
+    active = idx[:K].cpu().numpy()
+    halted_flops = costs.prefill_flops(dims, T, wl["halt_layer"], K, args.mode, active)
+    value = world * T / (ms / 1e3)
+
+    # per-kernel breakdown of the timed steps (CUDA events around every launch)
+    halt_pairs = int(sum(int(i) + 1 for i in active))
+    per = {}
+    for r in recs:
+        unit, amount = costs.launch_work(r, dims, halt_pairs)
+        p = per.setdefault(r["kind"], {"launches": 0, "ms": 0.0, "unit": unit, "work": 0})
+        p["launches"] += 1
+        p["ms"] += r["ms"]
+        p["work"] += amount
+    total_ms = sum(p["ms"] for p in per.values())
+    kernels = {}
+    for kind, p in sorted(per.items(), key=lambda kv: -kv[1]["ms"]):
+        rate = p["work"] / (p["ms"] / 1e3) if p["ms"] > 0 else 0.0
+        kernels[kind] = {"launches_per_step": p["launches"] // args.steps, "ms_per_step": p["ms"] / args.steps,
+                         "share": p["ms"] / total_ms if total_ms else 0.0,
+                         ("tflops" if p["unit"] == "flop" else "gbs"): rate / 1e12 if p["unit"] == "flop"
+                         else rate / 1e9}
+    dom_kind = max(per, key=lambda k: per[k]["ms"])
+    dom = per[dom_kind]
+    if dom["unit"] == "flop":
+        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+    else:
+        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof.update({"kernel": dom_kind, "traffic": None,
+                 "peak_source": f"{peaks['source']} ({'sustained bf16' if dom['unit'] == 'flop' else 'HBM copy'})",
+                 "step_tflops": halted_flops / (ms / 1e3) / 1e12})
+
+    extra = {}
+    if not args.no_extra:
+        step(cfg_dense)
+        ms_d, _, _ = timed(cfg_dense, max(2, args.steps // 2))
+        dense_flops = costs.prefill_flops(dims, T)
+        other = "halt" if args.mode == "prune" else "prune"
+        cfg_o = dash.make_config(halt_layer=wl["halt_layer"], mode=other, select=wl["select"], keep=wl["keep"],
+                                 relative=wl["relative"])
+        step(cfg_o)
+        ms_o, K_o, _ = timed(cfg_o, max(2, args.steps // 2))
+        act_o = idx[:K_o].cpu().numpy()
+        extra = {
+            "dense": {"tokens_per_s": world * T / (ms_d / 1e3), "ms_per_step": ms_d,
+                      "tflops": dense_flops / (ms_d / 1e3) / 1e12},
+            other + "_mode": {"tokens_per_s": world * T / (ms_o / 1e3), "ms_per_step": ms_o, "K": K_o,
+                              "speedup_vs_dense": ms_d / ms_o,
+                              "flop_bound": dense_flops / costs.prefill_flops(dims, T, wl["halt_layer"], K_o,
+                                                                              other, act_o)},
+            "speedup_vs_dense": ms_d / ms,
+            "flop_bound": dense_flops / halted_flops,
+        }
+        # end to end through the C ABI from pinned host memory: H2D of the
+        # input, the prefill, D2H of the K active rows' final states
+        h_host = h0.cpu().pin_memory()
+        out_host = torch.empty(T, dims.d_model, dtype=torch.bfloat16).pin_memory()
+        def e2e_step():
+            H.copy_(h_host, non_blocking=True)
+            k = dash.prefill(stack, H, cfg, idx_out=idx, delta_out=delta)
+            rows = k if args.mode == "prune" else T
+            out_host[:rows].copy_(H[:rows], non_blocking=True)
+            return rows
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        n_e2e = max(2, args.steps // 2)
+        for _ in range(n_e2e):
+            rows = e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms_e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        extra["e2e"] = {"value": world * T / (ms_e / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": T * dims.d_model * 2, "d2h_bytes_per_step": rows * dims.d_model * 2}
+    dash.check_device()
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, N(0,1) inputs)",
+        "config": {"workload": wl["name"], "model": "qwen2.5-7b-shaped random init" if dims is inputs.QWEN7B
+                   else "tiny", "global_batch": world, "seq_len": T, "halt_layer": wl["halt_layer"],
+                   "keep": wl["keep"], "mode": args.mode, "select": wl["select"],
+                   "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (13 GB of weights per step)"},
+        "K": K, "halted_tflop_per_step": halted_flops / 1e12,
+        "gpu_launches": len(recs), "roofline": roof, "kernels": kernels, "clocks": clocks,
+    }
+    out.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(dims, T, halted_flops)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -36,6 +36,34 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
                            int64_t T_kv, int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos,
                            dash_bf16* O, void* stream);
 
+/* ------------------------------------------------------ launch timing --
+ * Optional CUDA-event timing of every kernel the library launches (off by
+ * default; no page counterpart: this is measurement plumbing).  While
+ * recording, each launch is bracketed by two events on its own stream. */
+typedef enum dash_kernel_kind {
+  DASH_K_ROPE_TABLE = 0, DASH_K_RMSNORM = 1, DASH_K_GEMM_QKV = 2, DASH_K_GEMM_KV_HALTED = 3,
+  DASH_K_ATTENTION = 4, DASH_K_GEMM_O = 5, DASH_K_SCORE = 6, DASH_K_GEMM_GATE_UP = 7,
+  DASH_K_GEMM_DOWN = 8, DASH_K_SELECT = 9, DASH_K_GATHER = 10, DASH_K_SCATTER = 11,
+  DASH_K_GEMM = 12, DASH_K_COUNT = 13
+} dash_kernel_kind;
+
+typedef struct dash_launch_record {
+  int32_t kind;   /* dash_kernel_kind */
+  int32_t layer;  /* decoder layer, -1 outside the layer loop */
+  int64_t m;      /* rows (GEMM M, attention query rows, selection T) */
+  int64_t n;      /* GEMM N, attention key rows */
+  int64_t k;      /* GEMM K, attention causal (query, key) pairs */
+  float ms;       /* device time between the two events */
+} dash_launch_record;
+
+/* Starts recording (clears earlier records).  capacity = max launches kept. */
+dash_status dash_timing_start(int32_t capacity);
+/* Stops recording, synchronises on the recorded events and copies up to
+ * cap records to out (host memory).  Returns the number recorded, or -1. */
+int32_t dash_timing_stop(dash_launch_record* out, int32_t cap);
+/* Static name of a kernel kind. */
+const char* dash_kernel_name(int32_t kind);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,65 @@
+"""Algorithmic work of the DASH prefill path (FLOPs and HBM bytes).
+
+Counting rules: a linear layer costs 2 FLOPs per weight per token; causal
+attention costs 4*hq*hd FLOPs per visible (query, key) pair (QK^T and PV);
+HBM-bound kernels count the bytes they must read and write once.
+"""
+
+
+def linear_flops_per_token(dims):
+    d, hd, F = dims.d_model, dims.head_dim, dims.ffn_dim
+    qd, kvd = dims.n_heads * hd, dims.n_kv_heads * hd
+    return 2 * d * (qd + 2 * kvd) + 2 * qd * d + 2 * d * 2 * F + 2 * F * d
+
+
+def attn_flops(dims, pairs):
+    return 4 * dims.n_heads * dims.head_dim * pairs
+
+
+def causal_pairs(n):
+    return n * (n + 1) // 2
+
+
+def prefill_flops(dims, T, halt_layer=None, K=None, mode="dense", active_idx=None):
+    """Total algorithmic FLOPs of one prefill.
+
+    dense: every layer on T tokens.  prune: layers 0..halt_layer on T, later
+    layers on K tokens with causal attention among them.  halt: later layers
+    run K queries against all visible keys (sum of active positions + 1) and
+    recompute the K/V projections of the T-K halted rows.
+    """
+    lin = linear_flops_per_token(dims)
+    full = T * lin + attn_flops(dims, causal_pairs(T))
+    L = dims.n_layers
+    if mode == "dense" or halt_layer is None:
+        return L * full
+    n_full = halt_layer + 1
+    n_late = L - n_full
+    if mode == "prune":
+        late = K * lin + attn_flops(dims, causal_pairs(K))
+    else:
+        pairs = int(sum(int(i) + 1 for i in active_idx)) if active_idx is not None else causal_pairs(T) // 2
+        kvd = dims.n_kv_heads * dims.head_dim
+        late = K * lin + attn_flops(dims, pairs) + (T - K) * 2 * dims.d_model * 2 * kvd
+    return n_full * full + n_late * late
+
+
+def launch_work(rec, dims, halt_pairs=None):
+    """(unit, amount) of algorithmic work for one timed launch record."""
+    kind, m, n, k = rec["kind"], rec["m"], rec["n"], rec["k"]
+    if kind.startswith("gemm"):
+        return "flop", 2 * m * n * k
+    if kind == "attention":
+        pairs = k if k >= 0 else halt_pairs
+        return "flop", attn_flops(dims, pairs or 0)
+    if kind == "rmsnorm":
+        return "byte", 2 * m * n * 2
+    if kind in ("gather", "scatter"):
+        return "byte", 2 * m * n * 2
+    if kind == "score":
+        return "byte", m * 4 * (2 * n + 1) if n < 1024 else m * n * 2 * (1 + k) + 4 * m
+    if kind == "select":
+        return "byte", m * 4 + m * 4
+    if kind == "rope_table":
+        return "byte", m * n * 8
+    return "byte", 0

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "dash.h"
 #include "dash_ops.h"
@@ -63,6 +64,59 @@ inline dash_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ launch timing
+// While recording, each kernel launch is bracketed by two CUDA events on its
+// stream (host-side bookkeeping; meant for a single host thread).
+struct TimingRec {
+  dash_launch_record r;
+  cudaEvent_t e0, e1;
+};
+struct Timing {
+  bool on = false;
+  int cap = 0;
+  int layer = -1;
+  std::vector<TimingRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+} g_timing;
+
+cudaEvent_t next_event() {
+  if (g_timing.used == g_timing.pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_timing.pool.push_back(e);
+  }
+  return g_timing.pool[g_timing.used++];
+}
+
+class TimedLaunch {
+ public:
+  TimedLaunch(int kind, int64_t m, int64_t n, int64_t k, cudaStream_t st) : st_(st) {
+    if (!g_timing.on || static_cast<int>(g_timing.recs.size()) >= g_timing.cap) return;
+    cudaEvent_t e0 = next_event(), e1 = next_event();
+    if (!e0 || !e1) return;
+    TimingRec t;
+    t.r.kind = kind;
+    t.r.layer = g_timing.layer;
+    t.r.m = m;
+    t.r.n = n;
+    t.r.k = k;
+    t.r.ms = 0.f;
+    t.e0 = e0;
+    t.e1 = e1;
+    g_timing.recs.push_back(t);
+    idx_ = static_cast<int>(g_timing.recs.size()) - 1;
+    cudaEventRecord(e0, st_);
+  }
+  ~TimedLaunch() {
+    if (idx_ >= 0) cudaEventRecord(g_timing.recs[idx_].e1, st_);
+  }
+
+ private:
+  cudaStream_t st_;
+  int idx_ = -1;
+};
+
 // 2D bf16 tensor map with a 64-element (128-byte) inner box and 128B swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
               uint32_t box_rows) {
@@ -79,7 +133,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // ------------------------------------------------------------------- GEMM
 template <int BN, int EPI>
 dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
-                        const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st) {
+                        const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
   using C = dash::gemm::Cfg<BN>;
   if (M == 0) return DASH_OK;
   static std::once_flag attr_once;
@@ -106,13 +160,14 @@ dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_
   sh.tiles_n = N / BN;
   sh.num_tiles = sh.tiles_m * sh.tiles_n;
   const int grid = sh.num_tiles < di.num_sms ? sh.num_tiles : di.num_sms;
+  TimedLaunch tl(kind, M, N, K, st);
   gemm_kernel<BN, EPI><<<grid, dash::gemm::kThreads, C::kSmemBytes, st>>>(ma, mb, mb2, sh, ep);
   return launch_status();
 }
 
 template <int EPI>
 dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
-                 const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int* bn_used = nullptr) {
+                 const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind, int* bn_used = nullptr) {
   if (K % dash::gemm::BK != 0 || M > INT32_MAX) return DASH_ERR_SHAPE;
   // SwiGLU tiles hold BN/2 gate + BN/2 up columns, so N = 2F must split into
   // whole tiles on both halves.
@@ -120,11 +175,11 @@ dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, in
   const bool can128 = EPI == dash::gemm::kEpiSwiglu ? (N / 2) % 64 == 0 : N % 128 == 0;
   if (can256) {
     if (bn_used) *bn_used = 256;
-    return launch_gemm<256, EPI>(di, A, lda, M, K, B, B2, N, ep, st);
+    return launch_gemm<256, EPI>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
   if (can128) {
     if (bn_used) *bn_used = 128;
-    return launch_gemm<128, EPI>(di, A, lda, M, K, B, B2, N, ep, st);
+    return launch_gemm<128, EPI>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
   return DASH_ERR_SHAPE;
 }
@@ -161,6 +216,7 @@ dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16
   p.n_qtiles = static_cast<int>((M + dash::attn::BQ - 1) / dash::attn::BQ);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * hq;
+  TimedLaunch tl(DASH_K_ATTENTION, M, T_kv, qpos ? -1 : M * (M + 1) / 2, st);
   attn_kernel<HD><<<static_cast<unsigned>(grid), dash::attn::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
   return launch_status();
 }
@@ -181,6 +237,7 @@ dash_status rmsnorm(const bf16* X, int64_t x_rows, const int32_t* rowmap, int64_
   if (rows == 0) return DASH_OK;
   const int warps = 8;
   const int64_t blocks = (rows + warps - 1) / warps;
+  TimedLaunch tl(DASH_K_RMSNORM, rows, d, 0, st);
   dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
       X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y);
   return launch_status();
@@ -193,6 +250,7 @@ dash_status move_rows(bool scatter, const bf16* src, bf16* dst, const int32_t* i
   int64_t blocks = (K + warps - 1) / warps;
   const int64_t cap = static_cast<int64_t>(di.num_sms) * 16;
   if (blocks > cap) blocks = cap;
+  TimedLaunch tl(scatter ? DASH_K_SCATTER : DASH_K_GATHER, K, d, 0, st);
   if (scatter)
     dash::rows::move_rows_kernel<true><<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(src, dst, idx, K, T, d);
   else
@@ -206,6 +264,7 @@ dash_status rope_table(float2* tab, int64_t max_pos, int hd, double theta, const
   const int64_t cap = static_cast<int64_t>(di.num_sms) * 32;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return DASH_OK;
+  TimedLaunch tl(DASH_K_ROPE_TABLE, max_pos, hd / 2, 0, st);
   dash::rows::rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(tab, max_pos, hd / 2, theta);
   return launch_status();
 }
@@ -293,7 +352,7 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
     kv.kv_rowmap = halt->halted_idx;
     kv.col_offset = qd;
     if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.Act, d, nh, d, cb(w.w_qkv) + static_cast<int64_t>(qd) * d, nullptr,
-                                       2 * kvd, kv, st)) != DASH_OK)
+                                       2 * kvd, kv, st, DASH_K_GEMM_KV_HALTED)) != DASH_OK)
       return s;
   }
 
@@ -303,7 +362,7 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   qkv.pos = pos;
   qkv.kv_rowmap = halt ? halt->active_idx : nullptr;
   qkv.col_offset = 0;
-  if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st)) != DASH_OK)
+  if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st, DASH_K_GEMM_QKV)) != DASH_OK)
     return s;
   // a3: causal GQA attention -> O (into X)
   if ((s = attention(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, ws.X,
@@ -317,12 +376,13 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   o.ssq_h = ws.ssq_h;
   int bn = 0;
   if (delta)
-    s = gemm<dash::gemm::kEpiResidSsq>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, &bn);
+    s = gemm<dash::gemm::kEpiResidSsq>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
   else
-    s = gemm<dash::gemm::kEpiResid>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, &bn);
+    s = gemm<dash::gemm::kEpiResid>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
   if (s != DASH_OK) return s;
   if (delta) {
     const int64_t blocks = (M + 255) / 256;
+    TimedLaunch tl(DASH_K_SCORE, M, d / bn, 0, st);
     dash::rows::score_from_ssq_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(ws.ssq_u, ws.ssq_h, d / bn,
                                                                                      M, relative, delta);
     if ((s = launch_status()) != DASH_OK) return s;
@@ -332,12 +392,12 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   EpiArgs sw{};
   sw.out = ws.Act;
   sw.ldo = F;
-  if ((s = gemm<dash::gemm::kEpiSwiglu>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st)) != DASH_OK) return s;
+  if ((s = gemm<dash::gemm::kEpiSwiglu>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st, DASH_K_GEMM_GATE_UP)) != DASH_OK) return s;
   // a6: down projection + residual
   EpiArgs dn{};
   dn.out = H;
   dn.ldo = d;
-  return gemm<dash::gemm::kEpiResid>(di, ws.Act, F, M, F, cb(w.w_down), nullptr, d, dn, st);
+  return gemm<dash::gemm::kEpiResid>(di, ws.Act, F, M, F, cb(w.w_down), nullptr, d, dn, st, DASH_K_GEMM_DOWN);
 }
 
 bool weights_ok(const dash_layer_weights* w) {
@@ -372,6 +432,7 @@ dash_status select_impl(const float* scores, int64_t T, int kind, double keep, f
   const int64_t n_mid = hi - lo;
   const int64_t k_dyn = static_cast<int64_t>(std::floor(keep * static_cast<double>(n_mid)));
   if (T == 0) return cudaMemsetAsync(count, 0, sizeof(int32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+  TimedLaunch tl(DASH_K_SELECT, T, k_dyn, 0, st);
   dash::rows::select_kernel<<<1, dash::rows::kSelThreads, 0, st>>>(scores, T, kind, k_dyn, thr, lo, hi, idx, halted,
                                                                     count);
   return launch_status();
@@ -414,6 +475,7 @@ dash_status dash_score(const dash_bf16* U, const dash_bf16* H, int64_t T, int32_
   if (!U || !delta || (relative && !H) || !aligned16(U) || (relative && !aligned16(H))) return DASH_ERR_INVALID_ARG;
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
+  TimedLaunch tl(DASH_K_SCORE, T, d, relative ? 1 : 0, as_stream(stream));
   dash::rows::score_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, as_stream(stream)>>>(
       reinterpret_cast<const bf16*>(U), reinterpret_cast<const bf16*>(H), T, d, relative ? 1 : 0, delta);
   return launch_status();
@@ -488,7 +550,7 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
   ep.out = reinterpret_cast<bf16*>(Y);
   ep.ldo = N;
   return gemm<dash::gemm::kEpiStore>(*di, reinterpret_cast<const bf16*>(A), K, M, K, reinterpret_cast<const bf16*>(W),
-                                     nullptr, N, ep, as_stream(stream));
+                                     nullptr, N, ep, as_stream(stream), DASH_K_GEMM);
 }
 
 dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M, int64_t T_kv,
@@ -589,8 +651,12 @@ dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers
   if ((s = rope_table(P.L.rope, T, D.head_dim, D.rope_theta, *di, st)) != DASH_OK) return s;
 
   if (cfg->mode == DASH_MODE_DENSE) {
-    for (int l = 0; l < D.n_layers; ++l)
-      if ((s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, nullptr, 0, P.L, st)) != DASH_OK) return s;
+    for (int l = 0; l < D.n_layers; ++l) {
+      g_timing.layer = l;
+      s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, nullptr, 0, P.L, st);
+      g_timing.layer = -1;
+      if (s != DASH_OK) return s;
+    }
     if (K_out) *K_out = T;
     return DASH_OK;
   }
@@ -599,9 +665,11 @@ dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers
   const int Ls = cfg->halt_layer;
   float* delta = delta_out ? delta_out : P.delta;
   for (int l = 0; l <= Ls; ++l) {
-    if ((s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, l == Ls ? delta : nullptr,
-                        cfg->score == DASH_SCORE_REL, P.L, st)) != DASH_OK)
-      return s;
+    g_timing.layer = l;
+    s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, l == Ls ? delta : nullptr,
+                   cfg->score == DASH_SCORE_REL, P.L, st);
+    g_timing.layer = -1;
+    if (s != DASH_OK) return s;
   }
   // One-shot selection of the active set S*.
   int32_t* idx = idx_out ? idx_out : P.idx;
@@ -619,8 +687,12 @@ dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers
   // Gather the active rows; later layers run on them only.
   if ((s = move_rows(false, h, P.Hc, idx, K, T, D.d_model, *di, st)) != DASH_OK) return s;
   if (cfg->mode == DASH_MODE_PRUNE) {
-    for (int l = Ls + 1; l < D.n_layers; ++l)
-      if ((s = layer_impl(*di, D, layers[l], P.Hc, K, idx, nullptr, nullptr, 0, P.L, st)) != DASH_OK) return s;
+    for (int l = Ls + 1; l < D.n_layers; ++l) {
+      g_timing.layer = l;
+      s = layer_impl(*di, D, layers[l], P.Hc, K, idx, nullptr, nullptr, 0, P.L, st);
+      g_timing.layer = -1;
+      if (s != DASH_OK) return s;
+    }
     if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16), cudaMemcpyDeviceToDevice,
                                  st) != cudaSuccess)
       return DASH_ERR_CUDA;
@@ -631,9 +703,47 @@ dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers
   hc.halted_idx = P.halted;
   hc.h_full = H;
   hc.T = T;
-  for (int l = Ls + 1; l < D.n_layers; ++l)
-    if ((s = layer_impl(*di, D, layers[l], P.Hc, K, idx, &hc, nullptr, 0, P.L, st)) != DASH_OK) return s;
+  for (int l = Ls + 1; l < D.n_layers; ++l) {
+    g_timing.layer = l;
+    s = layer_impl(*di, D, layers[l], P.Hc, K, idx, &hc, nullptr, 0, P.L, st);
+    g_timing.layer = -1;
+    if (s != DASH_OK) return s;
+  }
   return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
+}
+
+dash_status dash_timing_start(int32_t capacity) {
+  if (capacity <= 0) return DASH_ERR_INVALID_ARG;
+  g_timing.recs.clear();
+  g_timing.recs.reserve(static_cast<size_t>(capacity));
+  g_timing.cap = capacity;
+  g_timing.used = 0;
+  g_timing.layer = -1;
+  g_timing.on = true;
+  return DASH_OK;
+}
+
+int32_t dash_timing_stop(dash_launch_record* out, int32_t cap) {
+  g_timing.on = false;
+  int32_t n = 0;
+  for (TimingRec& t : g_timing.recs) {
+    if (cudaEventSynchronize(t.e1) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t.e0, t.e1) != cudaSuccess) return -1;
+    t.r.ms = ms;
+    if (out && n < cap) out[n] = t.r;
+    ++n;
+  }
+  g_timing.recs.clear();
+  g_timing.used = 0;
+  return n < cap || !out ? n : cap;
+}
+
+const char* dash_kernel_name(int32_t kind) {
+  static const char* names[DASH_K_COUNT] = {"rope_table", "rmsnorm", "gemm_qkv_rope", "gemm_kv_halted",
+                                            "attention", "gemm_o_resid_delta", "score", "gemm_gate_up_swiglu",
+                                            "gemm_down_resid", "select", "gather", "scatter", "gemm"};
+  return kind >= 0 && kind < DASH_K_COUNT ? names[kind] : "unknown";
 }
 
 }  // extern "C"

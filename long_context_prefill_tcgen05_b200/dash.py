@@ -43,6 +43,10 @@ class Config(ctypes.Structure):
                 ("keep_ratio", c_f64), ("threshold", c_f32), ("keep_first", c_i32), ("keep_last", c_i32)]
 
 
+class LaunchRecord(ctypes.Structure):
+    _fields_ = [("kind", c_i32), ("layer", c_i32), ("m", c_i64), ("n", c_i64), ("k", c_i64), ("ms", c_f32)]
+
+
 class HaltCtx(ctypes.Structure):
     _fields_ = [("active_idx", c_vp), ("halted_idx", c_vp), ("h_full", c_vp), ("T", c_i64)]
 
@@ -65,6 +69,9 @@ _SIGS = {
     "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
     "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
     "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "dash_timing_start": (c_i32, [c_i32]),
+    "dash_timing_stop": (c_i32, [ctypes.POINTER(LaunchRecord), c_i32]),
+    "dash_kernel_name": (ctypes.c_char_p, [c_i32]),
 }
 
 _LIB = None
@@ -117,6 +124,21 @@ def device_error():
 
 def check_device():
     _check(device_error(), "device")
+
+
+# --------------------------------------------------------- launch timing
+def timing_start(capacity=1 << 16):
+    _check(lib().dash_timing_start(capacity), "dash_timing_start")
+
+
+def timing_stop(capacity=1 << 16):
+    """Stops recording; returns a list of dicts (kind name, layer, m, n, k, ms)."""
+    buf = (LaunchRecord * capacity)()
+    n = lib().dash_timing_stop(buf, capacity)
+    if n < 0:
+        raise DashError(5, "dash_timing_stop")
+    return [{"kind": lib().dash_kernel_name(r.kind).decode(), "layer": r.layer, "m": r.m, "n": r.n,
+             "k": r.k, "ms": r.ms} for r in buf[:n]]
 
 
 # ----------------------------------------------------------- workspaces

@@ -1,0 +1,262 @@
+"""GPU parity of dash_layer_forward and dash_prefill against the CPU oracle.
+
+Tiny stack (4 layers, d=256, T=512): full end-to-end comparison.  Qwen2.5-7B-
+shaped stack: one layer at a time, teacher-forced (the oracle gets the GPU's
+bf16 layer input) on sampled query rows, at the full T=32768 launch shapes
+the benchmark times, plus properties that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from long_context_prefill_tcgen05_b200 import dash, inputs
+from conftest import to_np, layers_np, row_rel_err, HIDDEN_TOL, DELTA_TOL, CUT_BAND
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _dev_layers(layers):
+    return [{k: v.to(DEV) for k, v in w.items()} for w in layers]
+
+
+@pytest.fixture(scope="module")
+def tiny(gpu_lib, tiny_stack):
+    dims, layers, h0 = tiny_stack
+    return dims, h0, dash.Stack(dims, _dev_layers(layers)), layers_np(layers)
+
+
+def _prefill(stack, h0, **kw):
+    H = h0.to(DEV).clone()
+    T = H.shape[0]
+    idx = torch.full((T,), -1, dtype=torch.int32, device=DEV)
+    delta = torch.empty(T, dtype=torch.float32, device=DEV)
+    K = dash.prefill(stack, H, dash.make_config(**kw), idx_out=idx, delta_out=delta)
+    assert dash.device_error() == 0
+    return H.cpu(), idx[:K].cpu().numpy(), delta.cpu().numpy(), K
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(np.asarray(a, np.float64) - b) / np.abs(b)))
+
+
+def _check_sets(idx, ref_idx, ref_delta, cut):
+    diff = np.setxor1d(idx, ref_idx)
+    for t in diff:
+        assert abs(ref_delta[t] - cut) <= CUT_BAND * abs(cut), (t, ref_delta[t], cut)
+
+
+def _topk_cut(delta, keep, nf=0, nl=0):
+    T = len(delta)
+    mid = np.flatnonzero(~O.forced_mask(T, nf, nl))
+    k = math.floor(keep * len(mid))
+    return np.sort(delta[mid])[::-1][k - 1] if k > 0 else np.inf
+
+
+# ------------------------------------------------------------- tiny layer
+def test_layer_dense_matches_oracle(tiny):
+    dims, h0, stack, L = tiny
+    T = h0.shape[0]
+    H = h0.to(DEV).clone()
+    delta = torch.empty(T, device=DEV)
+    dash.layer_forward(stack, 0, H, delta=delta)
+    pos = np.arange(T)
+    ref, u = O.decoder_block(to_np(h0), pos, to_np(h0), pos, L[0], dims.as_dict())
+    assert row_rel_err(to_np(H), ref) < HIDDEN_TOL
+    assert _rel(delta.cpu().numpy(), O.delta_scores(u)) < DELTA_TOL
+    delta_r = torch.empty(T, device=DEV)
+    dash.layer_forward(stack, 0, h0.to(DEV).clone(), delta=delta_r, relative=True)
+    assert _rel(delta_r.cpu().numpy(), O.delta_scores(u, to_np(h0), True)) < DELTA_TOL
+
+
+def test_layer_compacted_rows_at_original_positions(tiny):
+    dims, h0, stack, L = tiny
+    rng = np.random.default_rng(5)
+    idx = np.sort(rng.choice(512, 200, replace=False))
+    H = h0[idx].to(DEV).contiguous()
+    dash.layer_forward(stack, 1, H, pos=torch.tensor(idx, dtype=torch.int32, device=DEV), max_pos=512)
+    hn = to_np(h0)[idx]
+    ref, _ = O.decoder_block(hn, idx, hn, idx, L[1], dims.as_dict())
+    assert row_rel_err(to_np(H), ref) < HIDDEN_TOL
+
+
+def test_layer_halt_context(tiny):
+    dims, h0, stack, L = tiny
+    rng = np.random.default_rng(6)
+    idx = np.sort(rng.choice(512, 130, replace=False))
+    halted = np.setdiff1d(np.arange(512), idx)
+    H = h0[idx].to(DEV).contiguous()
+    hf = h0.to(DEV)
+    ti = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    th = torch.tensor(halted, dtype=torch.int32, device=DEV)
+    delta = torch.empty(len(idx), device=DEV)
+    dash.layer_forward(stack, 3, H, halt=(ti, th, hf), delta=delta)
+    ref, u = O.decoder_block(to_np(h0)[idx], idx, to_np(h0), np.arange(512), L[3], dims.as_dict())
+    assert row_rel_err(to_np(H), ref) < HIDDEN_TOL
+    assert _rel(delta.cpu().numpy(), O.delta_scores(u)) < DELTA_TOL
+
+
+# ----------------------------------------------------------- tiny prefill
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+@pytest.mark.parametrize("keep,nf,nl", [(0.5, 0, 0), (0.3, 64, 32)])
+def test_prefill_tiny_matches_oracle(tiny, mode, keep, nf, nl):
+    dims, h0, stack, L = tiny
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=2, mode=mode, keep=keep, keep_first=nf, keep_last=nl)
+    free = O.dash_prefill(to_np(h0), L, dims.as_dict(), 2, mode, keep=keep, keep_first=nf, keep_last=nl)
+    assert K == O.topk_count(512, keep, nf, nl) == len(free["idx"])
+    assert _rel(delta, free["delta"]) < DELTA_TOL
+    assert np.all(np.diff(idx) > 0)
+    # the GPU's selection on its own fp32 scores is exactly the oracle's rule
+    assert np.array_equal(idx, O.select_topk(delta.astype(np.float64), keep, nf, nl))
+    _check_sets(idx, free["idx"], free["delta"], _topk_cut(free["delta"], keep, nf, nl))
+    forced = O.dash_prefill(to_np(h0), L, dims.as_dict(), 2, mode, forced_idx=idx)
+    got = to_np(Hg[:K]) if mode == "prune" else to_np(Hg)
+    assert row_rel_err(got, forced["hidden"]) < HIDDEN_TOL
+
+
+def test_prefill_tiny_threshold_relative(tiny):
+    dims, h0, stack, L = tiny
+    free0 = O.dash_prefill(to_np(h0), L, dims.as_dict(), 1, "halt", keep=1.0, relative=True)
+    thr = float(np.float32(np.quantile(free0["delta"], 0.7)))
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=1, mode="halt", select="threshold", threshold=thr,
+                                 relative=True)
+    free = O.dash_prefill(to_np(h0), L, dims.as_dict(), 1, "halt", select="threshold", threshold=thr,
+                          relative=True)
+    assert _rel(delta, free["delta"]) < DELTA_TOL
+    assert np.array_equal(idx, O.select_threshold(delta.astype(np.float64), np.float32(thr)))
+    _check_sets(idx, free["idx"], free["delta"], thr)
+    forced = O.dash_prefill(to_np(h0), L, dims.as_dict(), 1, "halt", forced_idx=idx)
+    assert row_rel_err(to_np(Hg), forced["hidden"]) < HIDDEN_TOL
+
+
+def test_prefill_tiny_dense_matches_oracle(tiny):
+    dims, h0, stack, L = tiny
+    Hg, _, _, K = _prefill(stack, h0, mode="dense")
+    assert K == 512
+    assert row_rel_err(to_np(Hg), O.dense_forward(to_np(h0), L, dims.as_dict())) < HIDDEN_TOL
+
+
+def test_keep_one_prune_is_bitwise_dense(tiny):
+    dims, h0, stack, L = tiny
+    Hd, _, _, _ = _prefill(stack, h0, mode="dense")
+    Hp, idx, _, K = _prefill(stack, h0, halt_layer=1, mode="prune", keep=1.0)
+    Hh, _, _, _ = _prefill(stack, h0, halt_layer=2, mode="halt", keep=1.0)
+    assert K == 512 and np.array_equal(idx, np.arange(512))
+    assert torch.equal(Hp, Hd) and torch.equal(Hh, Hd)
+
+
+def test_halted_rows_frozen_at_halting_layer_output(tiny):
+    dims, h0, stack, L = tiny
+    Hh, idx, _, K = _prefill(stack, h0, halt_layer=1, mode="halt", keep=0.25)
+    first2 = dash.Stack(dims, _tiny_layers(dims)[:2])
+    Hs, _, _, _ = _prefill(first2, h0, mode="dense")
+    halted = np.setdiff1d(np.arange(512), idx)
+    assert torch.equal(Hh[halted], Hs[halted])
+
+
+def _tiny_layers(dims):
+    return _dev_layers(inputs.make_layers(dims, seed=0))
+
+
+def test_prefill_zero_keep(tiny):
+    dims, h0, stack, L = tiny
+    Hp, idx, _, K = _prefill(stack, h0, halt_layer=2, mode="prune", keep=0.0)
+    assert K == 0
+    Hh, idx, _, K = _prefill(stack, h0, halt_layer=2, mode="halt", keep=0.0)
+    first3 = dash.Stack(dims, _tiny_layers(dims)[:3])
+    Hs, _, _, _ = _prefill(first3, h0, mode="dense")
+    assert torch.equal(Hh, Hs)
+
+
+def test_prefill_reports_nonfinite(tiny):
+    dims, h0, stack, L = tiny
+    bad = h0.clone()
+    bad[7, :] = 0  # ||H_7|| = 0 at layer 0 in relative mode -> Δ is not finite
+    with pytest.raises(dash.DashError) as e:
+        _prefill(stack, bad, halt_layer=0, mode="prune", keep=0.5, relative=True)
+    assert e.value.status == 3
+    assert dash.device_error() == 3
+
+
+# ------------------------------------------------- Qwen2.5-7B-shaped layers
+@pytest.fixture(scope="module")
+def qwen_layer(gpu_lib):
+    dims = inputs.QWEN7B
+    layers = inputs.make_layers(dims, seed=11, device=DEV, n_layers=1)
+    return dims, dash.Stack(dims, layers), {k: to_np(v) for k, v in layers[0].items()}
+
+
+def _sampled_check(dims, W, h_in, h_out, rows, q_pos, kv_rows, kv_pos, delta=None):
+    """Oracle block for the sampled query rows (keys/values from every kv row)."""
+    hin = to_np(h_in)
+    ref, u = O.decoder_block(hin[rows], q_pos, to_np(kv_rows), kv_pos, W, dims.as_dict())
+    assert row_rel_err(to_np(h_out)[rows], ref) < HIDDEN_TOL
+    if delta is not None:
+        assert _rel(delta[rows], O.delta_scores(u)) < DELTA_TOL
+
+
+@pytest.mark.slow
+def test_qwen_layer_full_T_sampled_rows(qwen_layer):
+    dims, stack, W = qwen_layer
+    T = 32768
+    h0, _ = inputs.make_hidden(T, dims.d_model, seed=21, device=DEV)
+    H = h0.clone()
+    delta = torch.empty(T, device=DEV)
+    dash.layer_forward(stack, 0, H, delta=delta)
+    assert dash.device_error() == 0
+    rows = np.sort(np.concatenate([[0, 1, 127, 128, 4095, T - 1],
+                                   np.random.default_rng(0).choice(T, 58, replace=False)]))
+    _sampled_check(dims, W, h0.cpu(), H.cpu(), rows, rows, h0.cpu(), np.arange(T), delta.cpu().numpy())
+
+
+@pytest.mark.slow
+def test_qwen_layer_compacted_prune_shape(qwen_layer):
+    dims, stack, W = qwen_layer
+    T, K = 32768, 16384
+    rng = np.random.default_rng(1)
+    idx = np.sort(rng.choice(T, K, replace=False))
+    h0, _ = inputs.make_hidden(K, dims.d_model, seed=22, device=DEV)
+    H = h0.clone()
+    dash.layer_forward(stack, 0, H, pos=torch.tensor(idx, dtype=torch.int32, device=DEV), max_pos=T)
+    assert dash.device_error() == 0
+    rows = np.sort(rng.choice(K, 48, replace=False))
+    _sampled_check(dims, W, h0.cpu(), H.cpu(), rows, idx[rows], h0.cpu(), idx)
+
+
+@pytest.mark.slow
+def test_qwen_layer_halt_shape(qwen_layer):
+    dims, stack, W = qwen_layer
+    T, K = 32768, 16384
+    rng = np.random.default_rng(2)
+    idx = np.sort(rng.choice(T, K, replace=False))
+    halted = np.setdiff1d(np.arange(T), idx)
+    hfull, _ = inputs.make_hidden(T, dims.d_model, seed=23, device=DEV)
+    H = hfull[torch.tensor(idx, device=DEV)].contiguous()
+    h_in = H.clone()
+    ti = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    dash.layer_forward(stack, 0, H, halt=(ti, torch.tensor(halted, dtype=torch.int32, device=DEV), hfull))
+    assert dash.device_error() == 0
+    rows = np.sort(rng.choice(K, 48, replace=False))
+    _sampled_check(dims, W, h_in.cpu(), H.cpu(), rows, idx[rows], hfull.cpu(), np.arange(T))
+
+
+# ----------------------------------------- full-size prefill properties
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+def test_qwen_prefill_32k_properties(gpu_lib, mode):
+    """The benchmark's workload (28 layers, T=32768, halt at 11, keep 0.5):
+    count, order, selection = the oracle rule on the GPU's own Δ, finite output."""
+    dims = inputs.QWEN7B
+    stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=DEV))
+    h0, _ = inputs.make_hidden(32768, dims.d_model, seed=0, device=DEV)
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=11, mode=mode, keep=0.5)
+    assert K == 16384
+    assert np.all(np.diff(idx) > 0)
+    assert np.array_equal(idx, O.select_topk(delta.astype(np.float64), 0.5))
+    out = Hg[:K] if mode == "prune" else Hg
+    assert torch.isfinite(out.float()).all()
+    del stack
+    torch.cuda.empty_cache()
