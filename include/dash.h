@@ -205,6 +205,31 @@ dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* 
                                const dash_halt_ctx* halt, float* delta, int32_t relative,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* The same block as dash_layer_forward, for callers that cannot allocate
+ * device memory: code with no allocator of its own (for example a plugin
+ * whose host owns every device buffer), or a latency-bound loop that must
+ * not call cudaMalloc / cudaFree because they can synchronise the device.
+ * The caller still passes every input and output; the scratch that
+ * dash_layer_forward takes from a workspace lives instead in one fixed
+ * 32 MiB device array inside the library, which each GPU that loads the
+ * library holds until the process exits.  No counterpart on the pages: this
+ * is a deployment convenience.
+ *   - Shapes whose workspace (dash_layer_workspace_size) exceeds 32 MiB are
+ *     rejected with DASH_ERR_NO_MEMORY before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; no
+ *     part of it needs to start at zero (each call writes every byte it
+ *     reads).  Calls whose executions overlap on the GPU (other streams,
+ *     other host threads) race on it and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library
+ *     routine.  Arguments and errors otherwise as dash_layer_forward. */
+dash_status dash_layer_forward_noalloc(const dash_dims* dims, const dash_layer_weights* w, dash_bf16* H,
+                                       int64_t M, const int32_t* pos, int64_t max_pos,
+                                       const dash_halt_ctx* halt, float* delta, int32_t relative,
+                                       void* stream);
+
 /* -------------------------------------------------------------- prefill --
  * Workspace bytes for dash_prefill of T tokens under cfg. */
 size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_config* cfg);

@@ -438,6 +438,29 @@ dash_status select_impl(const float* scores, int64_t T, int kind, double keep, f
   return launch_status();
 }
 
+// Scratch of dash_layer_forward_noalloc: a file-scope device array, so that
+// entry point never allocates.  Every GPU that loads the library holds it
+// until the process exits.  In host code the array's name is only a
+// host-side stand-in; its device address comes from cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device (with that device current) and cached.
+dash_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DASH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DASH_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DASH_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -605,6 +628,23 @@ dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* 
   cudaStream_t st = as_stream(stream);
   if ((s = rope_table(L.rope, max_pos, dims->head_dim, dims->rope_theta, *di, st)) != DASH_OK) return s;
   return layer_impl(*di, *dims, *w, reinterpret_cast<bf16*>(H), M, pos, halt, delta, relative, L, st);
+}
+
+dash_status dash_layer_forward_noalloc(const dash_dims* dims, const dash_layer_weights* w, dash_bf16* H,
+                                       int64_t M, const int32_t* pos, int64_t max_pos, const dash_halt_ctx* halt,
+                                       float* delta, int32_t relative, void* stream) {
+  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
+  if (M < 0 || max_pos < 0) return DASH_ERR_SHAPE;
+  if (M == 0) return DASH_OK;
+  const int64_t T_kv = halt ? halt->T : M;
+  const size_t need = dash_layer_workspace_size(dims, M, T_kv, max_pos);
+  if (need == 0) return DASH_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return DASH_ERR_NO_MEMORY;
+  void* scratch = nullptr;
+  const dash_status s = noalloc_scratch(&scratch);
+  if (s != DASH_OK) return s;
+  return dash_layer_forward(dims, w, H, M, pos, max_pos, halt, delta, relative, scratch, kNoAllocScratchBytes,
+                            stream);
 }
 
 size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_config* cfg) {

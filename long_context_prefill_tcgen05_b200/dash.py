@@ -69,6 +69,8 @@ _SIGS = {
     "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
     "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
     "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "dash_layer_forward_noalloc": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, c_vp,
+                                           c_i64, ctypes.POINTER(HaltCtx), c_vp, c_i32, c_vp]),
     "dash_timing_start": (c_i32, [c_i32]),
     "dash_timing_stop": (c_i32, [ctypes.POINTER(LaunchRecord), c_i32]),
     "dash_kernel_name": (ctypes.c_char_p, [c_i32]),
