@@ -1,0 +1,92 @@
+"""Runs one kernel of the DASH prefill path at a chosen shape (for timing and
+for ncu captures of a single kernel on a small case).
+
+    python -m long_context_prefill_tcgen05_b200.kernel_cases attention --T 8192
+    python -m long_context_prefill_tcgen05_b200.kernel_cases linear --M 4096 --N 37888 --K 3584
+    python -m long_context_prefill_tcgen05_b200.kernel_cases layer --T 4096
+    python -m long_context_prefill_tcgen05_b200.kernel_cases select --T 32768
+
+Shapes default to the Qwen2.5-7B-shaped stack (28 q / 4 kv heads, hd 128,
+d 3584, FFN 18944).  Prints one JSON line with the mean CUDA-event time.
+"""
+import argparse
+import json
+
+import torch
+
+from . import build, costs, dash, inputs
+
+
+def _time(fn, iters, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["attention", "linear", "layer", "select", "score", "gather"])
+    ap.add_argument("--T", type=int, default=8192)
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=37888)
+    ap.add_argument("--K", type=int, default=3584)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=2)
+    args = ap.parse_args()
+    build.build()
+    dims = inputs.QWEN7B
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    rnd = lambda *s: torch.randn(*s, generator=g, device=dev).to(torch.bfloat16)
+    out = {"case": args.case}
+    if args.case == "attention":
+        T, hq, hkv, hd = args.T, dims.n_heads, dims.n_kv_heads, dims.head_dim
+        Q, K, V = rnd(T, hq * hd), rnd(T, hkv * hd), rnd(T, hkv * hd)
+        O = torch.empty_like(Q)
+        ms = _time(lambda: dash.attention(Q, K, V, hq, hkv, hd, out=O), args.iters, args.warmup)
+        fl = costs.attn_flops(dims, costs.causal_pairs(T))
+        out.update(T=T, ms=ms, tflops=fl / ms / 1e9)
+    elif args.case == "linear":
+        A, W = rnd(args.M, args.K), rnd(args.N, args.K) * 0.02
+        Y = torch.empty(args.M, args.N, dtype=torch.bfloat16, device=dev)
+        ms = _time(lambda: dash.linear(A, W, out=Y), args.iters, args.warmup)
+        out.update(M=args.M, N=args.N, K=args.K, ms=ms, tflops=2 * args.M * args.N * args.K / ms / 1e9)
+    elif args.case == "layer":
+        stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev, n_layers=1))
+        h0 = rnd(args.T, dims.d_model)
+        H = torch.empty_like(h0)
+        delta = torch.empty(args.T, device=dev)
+
+        def run():
+            H.copy_(h0)
+            dash.layer_forward(stack, 0, H, delta=delta)
+        ms = _time(run, args.iters, args.warmup)
+        fl = args.T * costs.linear_flops_per_token(dims) + costs.attn_flops(dims, costs.causal_pairs(args.T))
+        out.update(T=args.T, ms=ms, tflops=fl / ms / 1e9)
+    elif args.case == "select":
+        s = torch.rand(args.T, generator=g, device=dev)
+        ms = _time(lambda: dash.select(s, "topk", 0.5), args.iters, args.warmup)
+        out.update(T=args.T, ms=ms)
+    elif args.case == "score":
+        U = rnd(args.T, dims.d_model)
+        d = torch.empty(args.T, device=dev)
+        ms = _time(lambda: dash.score(U, out=d), args.iters, args.warmup)
+        out.update(T=args.T, ms=ms, gbs=args.T * dims.d_model * 2 / ms / 1e6)
+    elif args.case == "gather":
+        X = rnd(args.T, dims.d_model)
+        idx = torch.sort(torch.randperm(args.T, generator=g, device=dev)[:args.T // 2]).values.int()
+        ms = _time(lambda: dash.compact(X, idx), args.iters, args.warmup)
+        out.update(T=args.T, ms=ms, gbs=2 * (args.T // 2) * dims.d_model * 2 / ms / 1e6)
+    dash.check_device()
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
