@@ -6,18 +6,26 @@
 // queries at their original positions attend over all T keys), else i
 // (dense and prune mode: causal over the rows' own order).  This is the
 // attention module whose output, after o_proj, is the update U that the DASH
-// blog post (§2.1) scores; it never materialises the T x T matrix.
+// blog post (§2.1) scores; the T x T matrix is never materialised.
 //
-// One CTA = one 128-row query tile of one query head.  Warp roles:
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 2-stage ring
-//   warp 1      TMEM allocator and MMA issuer:
-//                 S_j = Q K_j^T   into S[j % 2] (TMEM, fp32)
-//                 O  += P_j V_j   into O        (TMEM, fp32), V as an MN-major operand
-//   warps 2..5  softmax: one query row per thread; reads S_j from TMEM, keeps
-//               the running max / sum, rescales O in TMEM when the max grows by
-//               more than 2^8 (lazy rescaling keeps the result exact), writes
-//               P_j (bf16) into swizzled shared memory, and finally writes
-//               O / l to global memory.
+// One CTA = two 128-row query tiles (Q0, Q1) of one query head, sharing every
+// K/V tile.  Warp roles (320 threads):
+//   warp 0      TMA producer: Q0/Q1 once, then K_j (3-stage ring) and V_j
+//               (2-stage ring)
+//   warp 1      TMEM allocator and MMA issuer, in the order
+//                 S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 ...
+//               so each softmax warpgroup overlaps two MMAs of the other tile.
+//   warps 2..5  softmax of Q0, warps 6..9 softmax of Q1: one query row per
+//               thread (TMEM lane = row); S_j is read from TMEM, the running
+//               max / sum kept in registers, O rescaled in TMEM only when the
+//               max grows by more than 2^8 (exact: l and O share the stale
+//               reference), and P_j written back to TMEM as packed bf16 pairs
+//               over the upper half of S_j, where the P*V MMA reads it as its
+//               A operand.
+// TMEM columns: S0/P0 [0,128) S1/P1 [128,256) O0 [256,384) O1 [384,512).
+// MMAs issued by one thread complete in order, so the commit that signals
+// S_i(j+1) also proves that P_i(j) V_j is finished: the softmax may then
+// overwrite P_i and rescale O_i without another barrier.
 #pragma once
 
 #include "common.cuh"
@@ -25,35 +33,50 @@
 namespace dash {
 namespace attn {
 
-constexpr int BQ = 128;  // query rows per CTA
-constexpr int BKV = 128; // keys per tile
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int BQ = 128;   // query rows per tile (two tiles per CTA)
+constexpr int BKV = 128;  // keys per tile
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Params {
   __nv_bfloat16* out;  // [M, hq*hd]
   int64_t ldo;
-  const int32_t* qpos; // [M] or NULL
-  int M, T_kv, hq, hkv, hd, n_qtiles;
-  float scale_log2;    // log2(e) / sqrt(hd)
+  const int32_t* qpos;  // [M] or NULL
+  int M, T_kv, hq, hkv, hd, n_qblocks;
+  float scale_log2;  // log2(e) / sqrt(hd)
 };
 
 template <int HD>
 struct Cfg {
-  static constexpr int kPanels = HD / 64;            // 128-byte swizzle panels per row
-  static constexpr int kQBytes = BQ * HD * 2;
-  static constexpr int kKBytes = BKV * HD * 2;
-  static constexpr int kPBytes = BQ * BKV * 2;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKBytes;
-  static constexpr int kOffP = kOffV + kStages * kKBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 1 + 1 + 1;
+  static constexpr int kPanels = HD / 64;  // 128-byte swizzle panels per row
+  static constexpr int kTileBytes = 128 * HD * 2;
+  static constexpr int kOffQ = 0;  // Q0, Q1
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
-  static constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256, 256+HD)
+  static constexpr uint32_t kTmemCols = 512;
 };
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -64,39 +87,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  // barrier slots
-  const uint32_t bar_q = smem_u32(bars + 0);
-  const uint32_t bar_kfull0 = smem_u32(bars + 1);
-  const uint32_t bar_vfull0 = smem_u32(bars + 1 + kStages);
-  const uint32_t bar_kvempty0 = smem_u32(bars + 1 + 2 * kStages);
-  const uint32_t bar_sfull0 = smem_u32(bars + 1 + 3 * kStages);
-  const uint32_t bar_pfull = smem_u32(bars + 3 + 3 * kStages);
-  const uint32_t bar_odone = smem_u32(bars + 4 + 3 * kStages);
-  const uint32_t bar_drain = smem_u32(bars + 5 + 3 * kStages);
+  const uint32_t bar_q = smem_u32(bars);
+  const uint32_t bar_kfull = smem_u32(bars + 1);
+  const uint32_t bar_kempty = smem_u32(bars + 1 + kKStages);
+  const uint32_t bar_vfull = smem_u32(bars + 1 + 2 * kKStages);
+  const uint32_t bar_vempty = smem_u32(bars + 1 + 2 * kKStages + kVStages);
+  const uint32_t bar_sfull = smem_u32(bars + 1 + 2 * kKStages + 2 * kVStages);
+  const uint32_t bar_pfull = bar_sfull + 16;
+  const uint32_t bar_odone = bar_sfull + 32;
+  const uint32_t bar_drain = bar_sfull + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x % p.hq;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / p.hq);  // heavy tiles first
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / p.hq);  // heavy blocks first
   const int kvh = head / (p.hq / p.hkv);
-  const int q0 = qt * BQ;
-  const int q_last = min(p.M - 1, q0 + BQ - 1);
-  const int pos_first = p.qpos ? p.qpos[q0] : q0;
-  const int pos_last = p.qpos ? p.qpos[q_last] : q_last;
-  const int kv_limit = min(pos_last + 1, p.T_kv);
-  const int n_tiles = (kv_limit + BKV - 1) / BKV;
+  const int q0 = qb * 2 * BQ;
+  const bool has1 = q0 + BQ < p.M;
+  // Key tiles each query tile needs (positions ascend within the block).
+  int n_t[2], pos_first[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first = min(q0 + t * BQ, p.M - 1);
+    const int last = min(q0 + t * BQ + BQ - 1, p.M - 1);
+    pos_first[t] = p.qpos ? p.qpos[first] : first;
+    const int pos_last = p.qpos ? p.qpos[last] : last;
+    const int lim = min(pos_last + 1, p.T_kv);
+    n_t[t] = (lim + BKV - 1) / BKV;
+  }
+  if (!has1) n_t[1] = 0;
+  const int n_kv = max(n_t[0], n_t[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_kfull0 + 8 * s, 1);
-      mbar_init(bar_vfull0 + 8 * s, 1);
-      mbar_init(bar_kvempty0 + 8 * s, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar_kfull + 8 * s, 1);
+      mbar_init(bar_kempty + 8 * s, 1);
     }
-    mbar_init(bar_sfull0, 1);
-    mbar_init(bar_sfull0 + 8, 1);
-    mbar_init(bar_pfull, 128);
-    mbar_init(bar_odone, 1);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar_vfull + 8 * s, 1);
+      mbar_init(bar_vempty + 8 * s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_sfull + 8 * t, 1);
+      mbar_init(bar_pfull + 8 * t, 128);
+      mbar_init(bar_odone + 8 * t, 1);
+    }
     mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
@@ -113,209 +149,199 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_o = tmem_base + 256;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------- producer
+      // ------------------------------------------------------------ producer
       const uint32_t sq = smem_u32(smem + C::kOffQ);
-      mbar_arrive_expect_tx(bar_q, C::kQBytes);
-      for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_2d(&tmap_q, sq + pn * (BQ * 128), bar_q, head * HD + pn * 64, q0);
-      uint32_t armed = 0, armed_par = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!mbar_wait(bar_kvempty0 + 8 * st, ph ^ 1u)) break;
-        const uint32_t sk = smem_u32(smem + C::kOffK + st * C::kKBytes);
-        const uint32_t sv = smem_u32(smem + C::kOffV + st * C::kKBytes);
-        mbar_arrive_expect_tx(bar_kfull0 + 8 * st, C::kKBytes);
+      mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * C::kTileBytes);
+      for (int t = 0; t < (has1 ? 2 : 1); ++t)
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(&tmap_k, sk + pn * (BKV * 128), bar_kfull0 + 8 * st, kvh * HD + pn * 64,
-                      j * BKV);
-        mbar_arrive_expect_tx(bar_vfull0 + 8 * st, C::kKBytes);
+          tma_load_2d(&tmap_q, sq + t * C::kTileBytes + pn * (BQ * 128), bar_q, head * HD + pn * 64, q0 + t * BQ);
+      uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int ks = j % kKStages, vs = j % kVStages;
+        const uint32_t kph = (j / kKStages) & 1, vph = (j / kVStages) & 1;
+        if (!mbar_wait(bar_kempty + 8 * ks, kph ^ 1u)) break;
+        const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
+        mbar_arrive_expect_tx(bar_kfull + 8 * ks, C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(&tmap_v, sv + pn * (BKV * 128), bar_vfull0 + 8 * st, kvh * HD + pn * 64,
-                      j * BKV);
-        armed |= 1u << st;
-        armed_par = (armed_par & ~(1u << st)) | (ph << st);
+          tma_load_2d(&tmap_k, sk + pn * (BKV * 128), bar_kfull + 8 * ks, kvh * HD + pn * 64, j * BKV);
+        karmed |= 1u << ks;
+        kpar = (kpar & ~(1u << ks)) | (kph << ks);
+        if (!mbar_wait(bar_vempty + 8 * vs, vph ^ 1u)) break;
+        const uint32_t sv = smem_u32(smem + C::kOffV + vs * C::kTileBytes);
+        mbar_arrive_expect_tx(bar_vfull + 8 * vs, C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d(&tmap_v, sv + pn * (BKV * 128), bar_vfull + 8 * vs, kvh * HD + pn * 64, j * BKV);
+        varmed |= 1u << vs;
+        vpar = (vpar & ~(1u << vs)) | (vph << vs);
       }
       mbar_wait_drain(bar_q, 0);
-      for (int s = 0; s < kStages; ++s) {
-        if ((armed >> s) & 1u) {
-          mbar_wait_drain(bar_kfull0 + 8 * s, (armed_par >> s) & 1u);
-          mbar_wait_drain(bar_vfull0 + 8 * s, (armed_par >> s) & 1u);
-        }
-      }
+      for (int s = 0; s < kKStages; ++s)
+        if ((karmed >> s) & 1u) mbar_wait_drain(bar_kfull + 8 * s, (kpar >> s) & 1u);
+      for (int s = 0; s < kVStages; ++s)
+        if ((varmed >> s) & 1u) mbar_wait_drain(bar_vfull + 8 * s, (vpar >> s) & 1u);
     }
   } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA
+    // ---------------------------------------------------------------- MMA
     const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
     const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
     const uint32_t sq = smem_u32(smem + C::kOffQ);
-    const uint32_t sp = smem_u32(smem + C::kOffP);
+    auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+      const int ks = j % kKStages;
+      if (!mbar_wait(bar_kfull + 8 * ks, (j / kKStages) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
+        const uint32_t qa = sq + t * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          umma_bf16_ss(tmem_base + t * BKV, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(sk + off, 16, 1024),
+                       idesc_s, kk != 0 ? 1u : 0u);
+        }
+        umma_commit(bar_sfull + 8 * t);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j  (P from TMEM)
+      const int vs = j % kVStages;
+      if (!mbar_wait(bar_pfull + 8 * t, j & 1)) return false;
+      if (!mbar_wait(bar_vfull + 8 * vs, (j / kVStages) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sv = smem_u32(smem + C::kOffV + vs * C::kTileBytes);
+        const uint32_t pa = tmem_base + t * BKV + BKV / 2;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, umma_desc_sw128(sv + kk * 16 * 128, BKV * 128, 1024),
+                       idesc_o, (j | kk) != 0 ? 1u : 0u);
+        umma_commit(bar_odone + 8 * t);
+      }
+      __syncwarp();
+      return true;
+    };
     bool ok = mbar_wait(bar_q, 0);
-    for (int j = 0; ok && j <= n_tiles; ++j) {
-      if (j < n_tiles) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!mbar_wait(bar_kfull0 + 8 * st, ph)) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sk = smem_u32(smem + C::kOffK + st * C::kKBytes);
-          const uint32_t d = tmem_base + (j & 1) * BKV;
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-            umma_bf16_ss(d, umma_desc_sw128(sq + off, 16, 1024), umma_desc_sw128(sk + off, 16, 1024),
-                         idesc_s, kk != 0 ? 1u : 0u);
-          }
-          umma_commit(bar_sfull0 + 8 * (j & 1));
-        }
-        __syncwarp();
+    if (ok && n_t[0] > 0) ok = issue_s(0, 0);
+    if (ok && n_t[1] > 0) ok = issue_s(1, 0);
+    for (int j = 0; ok && j < n_kv; ++j) {
+      if (j < n_t[0]) {
+        ok = issue_pv(0, j);
+        if (ok && j + 1 < n_t[0]) ok = issue_s(0, j + 1);
       }
-      if (j >= 1) {
-        const int jp = j - 1;
-        const int st = jp % kStages;
-        const uint32_t ph = (jp / kStages) & 1;
-        if (!mbar_wait(bar_pfull, jp & 1)) break;
-        if (!mbar_wait(bar_vfull0 + 8 * st, ph)) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sv = smem_u32(smem + C::kOffV + st * C::kKBytes);
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint32_t aoff = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-            umma_bf16_ss(tmem_o, umma_desc_sw128(sp + aoff, 16, 1024),
-                         umma_desc_sw128(sv + kk * 16 * 128, BKV * 128, 1024), idesc_o,
-                         (jp | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(bar_odone);
-          umma_commit(bar_kvempty0 + 8 * st);
-        }
-        __syncwarp();
+      if (ok && j < n_t[1]) {
+        ok = issue_pv(1, j);
+        if (ok && j + 1 < n_t[1]) ok = issue_s(1, j + 1);
       }
+      if (ok && lane == 0) {
+        umma_commit(bar_kempty + 8 * (j % kKStages));
+        umma_commit(bar_vempty + 8 * (j % kVStages));
+      }
+      __syncwarp();
     }
     if (lane == 0) umma_commit(bar_drain);
     __syncwarp();
     mbar_wait_drain(bar_drain, 0);
   } else {
-    // ---------------------------------------------------------- softmax
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // row within the tile == TMEM lane
-    const int m = q0 + r;
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;   // query tile of this warpgroup
+    const int wq = warp & 3;         // TMEM lane quarter
+    const int r = wq * 32 + lane;    // row within the tile == TMEM lane
+    const int m = q0 + t * BQ + r;
     const int mrow = min(m, p.M - 1);
     const int row_pos = p.qpos ? p.qpos[mrow] : m;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    uint8_t* sp_row = smem + C::kOffP + r * 128;
+    const uint32_t s_addr = tmem_base + lane_off + t * BKV;
+    const uint32_t o_addr = tmem_base + lane_off + 256 + t * 128;
+    const int n = n_t[t];
+    const float sc = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!mbar_wait(bar_sfull0 + 8 * (j & 1), (j >> 1) & 1)) {
+    for (int j = 0; j < n; ++j) {
+      if (!mbar_wait(bar_sfull + 8 * t, j & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // Four loads in flight, one wait; the registers are read only after it.
-      uint32_t u0[32], u1[32], u2[32], u3[32];
-      const uint32_t srow = tmem_base + lane_off + (j & 1) * BKV;
-      tmem_ld32(srow + 0, u0);
-      tmem_ld32(srow + 32, u1);
-      tmem_ld32(srow + 64, u2);
-      tmem_ld32(srow + 96, u3);
+      uint32_t u[BKV];
+      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(u + 0));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(u + 64));
+      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(u + 96));
       tmem_ld_wait();
-      float s[BKV];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        s[i] = __uint_as_float(u0[i]);
-        s[32 + i] = __uint_as_float(u1[i]);
-        s[64 + i] = __uint_as_float(u2[i]);
-        s[96 + i] = __uint_as_float(u3[i]);
-      }
+      float* s = reinterpret_cast<float*>(u);
       const int kv0 = j * BKV;
-      const bool need_mask = (kv0 + BKV - 1 > pos_first) || (kv0 + BKV > p.T_kv);
-      float rmax = -INFINITY;
-      if (need_mask) {
+      if (kv0 + BKV - 1 > pos_first[t] || kv0 + BKV > p.T_kv) {
         const int lim = min(row_pos, p.T_kv - 1) - kv0;  // last visible column of this row
 #pragma unroll
-        for (int c = 0; c < BKV; ++c) {
-          s[c] = (c <= lim) ? s[c] * p.scale_log2 : -INFINITY;
-          rmax = fmaxf(rmax, s[c]);
-        }
-      } else {
+        for (int c = 0; c < BKV; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
+      }
+      float mx[8];
 #pragma unroll
-        for (int c = 0; c < BKV; ++c) {
-          s[c] *= p.scale_log2;
-          rmax = fmaxf(rmax, s[c]);
-        }
-      }
-      // P_j may be written and O rescaled only once O += P_{j-1} V_{j-1} is done.
-      if (j >= 1 && !mbar_wait(bar_odone, (j - 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+      for (int c = 8; c < BKV; c += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
+      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
       if (j == 0) {
         m_run = rmax;  // every row sees key 0, so rmax is finite here
       } else if (__any_sync(0xffffffffu, rmax > m_run + kRescaleThreshold)) {
+        // P_t(j-1) V_(j-1) is complete (in-order MMAs, see above): O_t may be rescaled.
         const float m_new = fmaxf(m_run, rmax);
-        const float alpha = exp2f(m_run - m_new);
+        const float alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
         l_run *= alpha;
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + c, o);
+          tmem_ld32(o_addr + c, o);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem_o + lane_off + c, o);
+          tmem_st32(o_addr + c, o);
         }
-        tmem_st_wait();
       }
-      float lsum = 0.f;
+      const float neg = -m_run;
+      float ls[8];
 #pragma unroll
-      for (int ch = 0; ch < BKV / 8; ++ch) {
-        float e[8];
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+      uint32_t pk[BKV / 2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          e[i] = exp2f(s[8 * ch + i] - m_run);
-          lsum += e[i];
-        }
-        uint4 w;
-        w.x = pack_bf16(e[0], e[1]);
-        w.y = pack_bf16(e[2], e[3]);
-        w.z = pack_bf16(e[4], e[5]);
-        w.w = pack_bf16(e[6], e[7]);
-        const int pn = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(sp_row + pn * (BQ * 128) + ((cc ^ (r & 7)) << 4)) = w;
+      for (int c = 0; c < BKV; c += 2) {
+        const float e0 = ex2_approx(fmaf(s[c], sc, neg));
+        const float e1 = ex2_approx(fmaf(s[c + 1], sc, neg));
+        ls[(c >> 1) & 7] += e0 + e1;
+        pk[c >> 1] = pack_bf16(e0, e1);
       }
-      l_run += lsum;
-      fence_proxy_async_smem();
+      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      tmem_st32(s_addr + BKV / 2, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
+      tmem_st32(s_addr + BKV / 2 + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_pfull);
+      mbar_arrive(bar_pfull + 8 * t);
     }
-    if (ok && n_tiles > 0 && mbar_wait(bar_odone, (n_tiles - 1) & 1)) {
+    if (ok && n > 0 && mbar_wait(bar_odone + 8 * t, (n - 1) & 1)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       __nv_bfloat16* dst = p.out + static_cast<int64_t>(mrow) * p.ldo + head * HD;
 #pragma unroll 1
       for (int c = 0; c < HD; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tmem_o + lane_off + c, o);
+        tmem_ld32(o_addr + c, o);
         tmem_ld_wait();
         if (m < p.M) {
-          float f[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(o[i]) * inv_l;
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
-            w.x = pack_bf16(f[8 * i + 0], f[8 * i + 1]);
-            w.y = pack_bf16(f[8 * i + 2], f[8 * i + 3]);
-            w.z = pack_bf16(f[8 * i + 4], f[8 * i + 5]);
-            w.w = pack_bf16(f[8 * i + 6], f[8 * i + 7]);
+            w.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            w.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            w.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            w.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
             d4[i] = w;
           }
         }
