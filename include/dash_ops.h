@@ -36,6 +36,13 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
                            int64_t T_kv, int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos,
                            dash_bf16* O, void* stream);
 
+/* The FMA-pipe exponential the attention softmax uses for half of its
+ * elements (no page counterpart; exported so tests can hold it to its error
+ * bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
+ * (max relative error 7.5e-5) and an exponent-field add; inputs below -125
+ * are clamped (result ~2e-38).  x, y: [n] fp32 device arrays. */
+dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream);
+
 /* ------------------------------------------------------ launch timing --
  * Optional CUDA-event timing of every kernel the library launches (off by
  * default; no page counterpart: this is measurement plumbing).  While

@@ -39,6 +39,12 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// One exponential in every 2 * kEmuPeriod columns is computed on the FMA pipe
+// (ex2_fma); the rest use MUFU.  0 disables the FMA path.
+#ifndef DASH_ATTN_EMU_PERIOD
+#define DASH_ATTN_EMU_PERIOD 0
+#endif
+constexpr int kEmuPeriod = DASH_ATTN_EMU_PERIOD;
 
 struct Params {
   __nv_bfloat16* out;  // [M, hq*hd]
@@ -66,6 +72,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA / integer pipes, relieving the MUFU unit that the other half
+// of the softmax exponentials use.  Range split: x = j + f with j = round(x)
+// (the 1.5 * 2^23 addition rounds to an integer held in the low mantissa
+// bits) and f in [-0.5, 0.5]; 2^f by a cubic whose coefficients were fitted
+// here to minimise the relative error on [-0.5, 0.5] (iteratively reweighted
+// least squares on Chebyshev nodes; max relative error 7.5e-5 in fp32, far
+// below bf16's 3.9e-3); 2^j is added to the exponent field.  Inputs are
+// clamped at -125 so the exponent add stays within normal numbers (j <= -127
+// would wrap into the sign bit); fully masked scores give ~2e-38 instead of 0,
+// negligible next to any bf16 weight.
+__device__ __forceinline__ float ex2_fma(float x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.0f);
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  const float q = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -287,14 +312,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
       const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
+      bool rescale = false;
+      float alpha = 1.f;
       if (j == 0) {
         m_run = rmax;  // every row sees key 0, so rmax is finite here
       } else if (__any_sync(0xffffffffu, rmax > m_run + kRescaleThreshold)) {
-        // P_t(j-1) V_(j-1) is complete (in-order MMAs, see above): O_t may be rescaled.
         const float m_new = fmaxf(m_run, rmax);
-        const float alpha = ex2_approx(m_run - m_new);
+        alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
-        l_run *= alpha;
+        rescale = true;
+      }
+      const float neg = -m_run;
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+      float lsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // 64 columns at a time keeps pk small
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = half * 64 + 2 * i;
+          const float e0 = ex2_approx(fmaf(s[c], sc, neg));  // MUFU
+          const float x1 = fmaf(s[c + 1], sc, neg);
+          const float e1 = (kEmuPeriod > 0 && (i % (kEmuPeriod > 0 ? kEmuPeriod : 1)) == kEmuPeriod - 1)
+                               ? ex2_fma(x1)  // FMA pipe
+                               : ex2_approx(x1);
+          ls[i & 7] += e0 + e1;
+          pk[i] = pack_bf16(e0, e1);
+        }
+        tmem_st32(s_addr + BKV / 2 + 32 * half, pk);
+      }
+      lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      l_run = fmaf(l_run, alpha, lsum);
+      if (rescale) {
+        // P_t(j-1) V_(j-1) is complete (in-order MMAs): O_t may be rescaled.
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           uint32_t o[32];
@@ -305,21 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(o_addr + c, o);
         }
       }
-      const float neg = -m_run;
-      float ls[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-      uint32_t pk[BKV / 2];
-#pragma unroll
-      for (int c = 0; c < BKV; c += 2) {
-        const float e0 = ex2_approx(fmaf(s[c], sc, neg));
-        const float e1 = ex2_approx(fmaf(s[c + 1], sc, neg));
-        ls[(c >> 1) & 7] += e0 + e1;
-        pk[c >> 1] = pack_bf16(e0, e1);
-      }
-      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      tmem_st32(s_addr + BKV / 2, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
-      tmem_st32(s_addr + BKV / 2 + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_pfull + 8 * t);

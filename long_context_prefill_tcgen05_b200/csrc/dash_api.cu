@@ -461,6 +461,12 @@ dash_status noalloc_scratch(void** out) {
   return DASH_OK;
 }
 
+__global__ void exp2_fma_kernel(const float* __restrict__ x, int64_t n, float* __restrict__ y) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = dash::attn::ex2_fma(x[i]);
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -574,6 +580,15 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
   ep.ldo = N;
   return gemm<dash::gemm::kEpiStore>(*di, reinterpret_cast<const bf16*>(A), K, M, K, reinterpret_cast<const bf16*>(W),
                                      nullptr, N, ep, as_stream(stream), DASH_K_GEMM);
+}
+
+dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream) {
+  if (n < 0) return DASH_ERR_SHAPE;
+  if (n == 0) return DASH_OK;
+  if (!x || !y) return DASH_ERR_INVALID_ARG;
+  const int64_t blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+  exp2_fma_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(x, n, y);
+  return launch_status();
 }
 
 dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M, int64_t T_kv,

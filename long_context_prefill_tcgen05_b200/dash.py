@@ -71,6 +71,7 @@ _SIGS = {
     "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
     "dash_layer_forward_noalloc": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, c_vp,
                                            c_i64, ctypes.POINTER(HaltCtx), c_vp, c_i32, c_vp]),
+    "dash_exp2_fma": (c_i32, [c_vp, c_i64, c_vp, c_vp]),
     "dash_timing_start": (c_i32, [c_i32]),
     "dash_timing_stop": (c_i32, [ctypes.POINTER(LaunchRecord), c_i32]),
     "dash_kernel_name": (ctypes.c_char_p, [c_i32]),
@@ -213,6 +214,12 @@ def linear(A, W, out=None, stream=None):
     out = torch.empty(M, N, dtype=A.dtype, device=A.device) if out is None else out
     _check(lib().dash_linear(_p(A), M, K, _p(W), N, _p(out), _stream(stream)), "dash_linear")
     return out
+
+
+def exp2_fma(x, stream=None):
+    y = torch.empty_like(x)
+    _check(lib().dash_exp2_fma(_p(x), x.numel(), _p(y), _stream(stream)), "dash_exp2_fma")
+    return y
 
 
 def attention(Q, K, V, hq, hkv, hd, qpos=None, out=None, stream=None):

@@ -164,3 +164,13 @@ def test_attention_indexed_queries_match_oracle(gpu_lib, M, T_kv, hq, hkv, hd):
     got, ref = _attn_case(M, T_kv, hq, hkv, hd, qpos, seed=T_kv)
     assert row_rel_err(got.reshape(M * hq, hd), ref.reshape(M * hq, hd)) < 2e-2
     _no_device_error()
+
+
+def test_exp2_fma_within_its_error_bound(gpu_lib):
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.999])])
+    y = dash.exp2_fma(x.to(DEV)).cpu().double().numpy()
+    ref = np.exp2(x.double().numpy())
+    assert np.max(np.abs(y - ref) / ref) < 1e-4          # fitted cubic: 7.5e-5
+    low = dash.exp2_fma(torch.tensor([-125.5, -127.0, -200.0, -float("inf")], device=DEV)).cpu().numpy()
+    assert np.all(np.isfinite(low) & (low > 0) & (low < 1e-37))  # clamped far below any bf16 weight
+    _no_device_error()
