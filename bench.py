@@ -30,16 +30,36 @@ from long_context_prefill_tcgen05_b200 import costs, inputs  # noqa: E402
 
 WORKLOADS = {
     "qwen7b-32k": dict(dims=inputs.QWEN7B, T=32768, halt_layer=11, keep=0.5, select="topk", relative=False,
-                       span_rows=0, span_len=64,
+                       span_rows=0, span_len=64, mode="prune",
                        name="Qwen2.5-7B-shaped stack (28 layers, d=3584, 28q/4kv, hd=128, FFN 18944), "
                             "T=32768, halt at layer 11, keep 0.5"),
-    "qwen7b-128k": dict(dims=inputs.QWEN7B, T=131072, halt_layer=11, keep=0.3, select="topk", relative=True,
-                        span_rows=6528, span_len=128,
-                        name="Qwen2.5-7B-shaped stack, T=131072, halt at layer 11, relative delta, keep 0.3"),
+    # threshold = the relative delta at rank floor(0.3 T) of a calibration prefill on the
+    # same input, then frozen (the timed run is a pure threshold run)
+    "qwen7b-128k": dict(dims=inputs.QWEN7B, T=131072, halt_layer=11, keep=0.3, select="threshold", relative=True,
+                        span_rows=6528, span_len=128, mode="halt", calibrate=True,
+                        name="Qwen2.5-7B-shaped stack, T=131072, halt at layer 11, relative-delta threshold "
+                             "calibrated to keep 30%, halt mode"),
     "tiny": dict(dims=inputs.TINY, T=512, halt_layer=2, keep=0.5, select="topk", relative=False, span_rows=0,
-                 span_len=64, name="tiny decoder stack (4 layers, d=256, 4q/2kv, hd=64, FFN 704), T=512"),
+                 span_len=64, mode="prune", name="tiny decoder stack (4 layers, d=256, 4q/2kv, hd=64, FFN 704), T=512"),
 }
 METRIC = "prefill tokens/s @T=32K/128K, halted vs dense, and % of B200 roofline"
+
+
+def recorded_traffic(kind, recs):
+    """DRAM bytes per launch of `kind` from the committed ncu record, scaled by rows to
+    the launches of this run; None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kind)
+        src = os.path.join(ROOT, "long_context_prefill_tcgen05_b200", "csrc", f"{kind}.cuh")
+        with open(src, "rb") as f:
+            if rec is None or hashlib.sha256(f.read()).hexdigest() != rec["src_sha256"]:
+                return None
+    except (OSError, ValueError, KeyError):
+        return None
+    launches = [r for r in recs if r["kind"] == kind]
+    return sum(rec["bytes_per_launch"] * r["m"] / rec["rows"] for r in launches) / max(1, len(launches))
 
 
 def load_peaks():
@@ -215,7 +235,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="qwen7b-32k", choices=sorted(WORKLOADS))
-    ap.add_argument("--mode", default="prune", choices=["prune", "halt"])
+    ap.add_argument("--mode", default=None, choices=["prune", "halt"], help="default: the workload's mode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the dense / other-mode / e2e legs")
@@ -235,6 +255,7 @@ def main():
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
     dims, T = wl["dims"], wl["T"]
+    args.mode = args.mode or wl["mode"]
     peaks = load_peaks()
 
     stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev))
@@ -243,8 +264,16 @@ def main():
     H = torch.empty_like(h0)
     idx = torch.empty(T, dtype=torch.int32, device=dev)
     delta = torch.empty(T, dtype=torch.float32, device=dev)
+    threshold = 0.0
+    if wl.get("calibrate"):
+        cal = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select="topk", keep=wl["keep"],
+                               relative=wl["relative"])
+        H.copy_(h0)
+        dash.prefill(stack, H, cal, idx_out=idx, delta_out=delta)
+        kcal = math.floor(wl["keep"] * T)
+        threshold = float(torch.sort(delta.cpu(), descending=True).values[kcal - 1])
     cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select=wl["select"], keep=wl["keep"],
-                           relative=wl["relative"])
+                           threshold=threshold, relative=wl["relative"])
     cfg_dense = dash.make_config(mode="dense")
 
     def step(c):
@@ -306,7 +335,7 @@ def main():
         achieved = dom["work"] / (dom["ms"] / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
-    roof.update({"kernel": dom_kind, "traffic": None,
+    roof.update({"kernel": dom_kind, "traffic": recorded_traffic(dom_kind, recs),
                  "peak_source": f"{peaks['source']} ({'sustained bf16' if dom['unit'] == 'flop' else 'HBM copy'})",
                  "step_tflops": halted_flops / (ms / 1e3) / 1e12})
 
@@ -317,7 +346,7 @@ def main():
         dense_flops = costs.prefill_flops(dims, T)
         other = "halt" if args.mode == "prune" else "prune"
         cfg_o = dash.make_config(halt_layer=wl["halt_layer"], mode=other, select=wl["select"], keep=wl["keep"],
-                                 relative=wl["relative"])
+                                 threshold=threshold, relative=wl["relative"])
         step(cfg_o)
         ms_o, K_o, _ = timed(cfg_o, max(2, args.steps // 2))
         act_o = idx[:K_o].cpu().numpy()
@@ -363,6 +392,7 @@ def main():
         "config": {"workload": wl["name"], "model": "qwen2.5-7b-shaped random init" if dims is inputs.QWEN7B
                    else "tiny", "global_batch": world, "seq_len": T, "halt_layer": wl["halt_layer"],
                    "keep": wl["keep"], "mode": args.mode, "select": wl["select"],
+                   **({"threshold": threshold} if wl["select"] == "threshold" else {}),
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (13 GB of weights per step)"},
         "K": K, "halted_tflop_per_step": halted_flops / 1e12,
         "gpu_launches": len(recs), "roofline": roof, "kernels": kernels, "clocks": clocks,
