@@ -252,6 +252,29 @@ dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers
                          int64_t T, const dash_config* cfg, int32_t* idx_out, int64_t* K_out,
                          float* delta_out, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------- varlen prefill --
+ * dash_prefill over a batch of independent sequences concatenated along the
+ * rows of H ([DASH blog] §5.1: in a batch every sample takes its own halting
+ * decision, and gather/scatter must not mix samples).
+ *   cu_seqlens: [nseq + 1] HOST int32, cu_seqlens[0] = 0, non-decreasing;
+ *               sequence s is rows [cu_seqlens[s], cu_seqlens[s+1]) of H.
+ *   Attention is causal within each sequence only (block-diagonal); RoPE
+ *   positions count from each sequence's first row; selection (top-k with
+ *   K_s = forced + floor(keep * (len_s - forced)), or threshold), forced
+ *   first / last tokens and Δ are per sequence.
+ *   idx_out:    [T] device out or NULL: active indices (absolute rows),
+ *               ascending, grouped by sequence.
+ *   seq_counts: [nseq] HOST out or NULL: active tokens per sequence.
+ *   Other arguments, output layout and the single synchronisation as in
+ *   dash_prefill (prune: the first K rows of H hold the active rows of
+ *   sequence 0, then sequence 1, ...). */
+size_t dash_prefill_varlen_workspace_size(const dash_dims* dims, int64_t T, int32_t nseq,
+                                          const dash_config* cfg);
+dash_status dash_prefill_varlen(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H,
+                                const int32_t* cu_seqlens, int32_t nseq, const dash_config* cfg,
+                                int32_t* idx_out, int64_t* K_out, int32_t* seq_counts, float* delta_out,
+                                void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,12 +29,15 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
 
 /* Causal grouped-query attention (the attention module of §2.1):
  *   Q: [M, hq*hd], K, V: [T_kv, hkv*hd], O: [M, hq*hd] bf16.
- *   Query i sees key j iff j <= qpos(i) and j < T_kv, where qpos(i) =
- *   qpos[i] (ascending int32 positions) or i when qpos is NULL.
+ *   Query i sees key j iff kstart(i) <= j <= qpos(i) and j < T_kv, where
+ *   qpos(i) = qpos[i] (ascending int32 positions) or i when qpos is NULL,
+ *   and kstart(i) = kstart[i] (non-decreasing; the start of row i's own
+ *   sequence in a varlen batch, making attention block-diagonal) or 0 when
+ *   kstart is NULL.
  *   Scale 1/sqrt(hd), fp32 softmax.  hd must be 64 or 128, hq % hkv == 0. */
 dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M,
                            int64_t T_kv, int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos,
-                           dash_bf16* O, void* stream);
+                           const int32_t* kstart, dash_bf16* O, void* stream);
 
 /* The FMA-pipe exponential the attention softmax uses for half of its
  * elements (no page counterpart; exported so tests can hold it to its error
@@ -42,6 +45,13 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
  * (max relative error 7.5e-5) and an exponent-field add; inputs below -125
  * are clamped (result ~2e-38).  x, y: [n] fp32 device arrays. */
 dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream);
+
+/* Failure-path self test (no page counterpart): launches one kernel whose
+ * bounded mbarrier wait can never complete, waits for it and returns what
+ * dash_device_error() then reports -- DASH_ERR_TIMEOUT when the bounded wait
+ * gave up after its ~2 s limit as designed.  done: [1] int32 device out,
+ * 2 when the wait gave up, 1 if it (wrongly) completed.  Synchronises. */
+dash_status dash_selftest_wait_timeout(int32_t* done);
 
 /* ------------------------------------------------------ launch timing --
  * Optional CUDA-event timing of every kernel the library launches (off by

@@ -1,7 +1,10 @@
 // Causal grouped-query flash attention on tcgen05 (sm_100a).
 //
 // O[i, h, :] = softmax_j( Q[i, h, :] . K[j, g, :] / sqrt(hd) ) V[j, g, :],
-// g = h / (hq / hkv), over keys j visible to query i:  j <= qpos(i), j < T_kv.
+// g = h / (hq / hkv), over keys j visible to query i:
+//   kstart(i) <= j <= qpos(i),  j < T_kv,
+// kstart(i) = kstart[i] when given (varlen batches: the first key of row i's
+// own sequence, so attention is block-diagonal causal), else 0.
 // qpos(i) = qpos[i] when a position list is given (halt mode: compacted
 // queries at their original positions attend over all T keys), else i
 // (dense and prune mode: causal over the rows' own order).  This is the
@@ -49,7 +52,8 @@ constexpr int kEmuPeriod = DASH_ATTN_EMU_PERIOD;
 struct Params {
   __nv_bfloat16* out;  // [M, hq*hd]
   int64_t ldo;
-  const int32_t* qpos;  // [M] or NULL
+  const int32_t* qpos;    // [M] or NULL
+  const int32_t* kstart;  // [M] or NULL (non-decreasing)
   int M, T_kv, hq, hkv, hd, n_qblocks;
   float scale_log2;  // log2(e) / sqrt(hd)
 };
@@ -129,8 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = head / (p.hq / p.hkv);
   const int q0 = qb * 2 * BQ;
   const bool has1 = q0 + BQ < p.M;
-  // Key tiles each query tile needs (positions ascend within the block).
-  int n_t[2], pos_first[2];
+  // Key tiles [jb_t, n_t) each query tile needs (positions and key starts ascend
+  // within the block).
+  int n_t[2], jb_t[2], pos_first[2], ks_last[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int first = min(q0 + t * BQ, p.M - 1);
@@ -139,8 +144,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pos_last = p.qpos ? p.qpos[last] : last;
     const int lim = min(pos_last + 1, p.T_kv);
     n_t[t] = (lim + BKV - 1) / BKV;
+    jb_t[t] = p.kstart ? p.kstart[first] / BKV : 0;
+    ks_last[t] = p.kstart ? p.kstart[last] : 0;
   }
-  if (!has1) n_t[1] = 0;
+  if (!has1) {
+    n_t[1] = 0;
+    jb_t[1] = jb_t[0];
+  }
+  const int j0 = jb_t[0];  // first key tile of the block
   const int n_kv = max(n_t[0], n_t[1]);
 
   if (threadIdx.x == 0) {
@@ -184,9 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_2d(&tmap_q, sq + t * C::kTileBytes + pn * (BQ * 128), bar_q, head * HD + pn * 64, q0 + t * BQ);
       uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j % kKStages, vs = j % kVStages;
-        const uint32_t kph = (j / kKStages) & 1, vph = (j / kVStages) & 1;
+      for (int j = j0; j < n_kv; ++j) {
+        const int jl = j - j0;  // ring index
+        const int ks = jl % kKStages, vs = jl % kVStages;
+        const uint32_t kph = (jl / kKStages) & 1, vph = (jl / kVStages) & 1;
         if (!mbar_wait(bar_kempty + 8 * ks, kph ^ 1u)) break;
         const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
         mbar_arrive_expect_tx(bar_kfull + 8 * ks, C::kTileBytes);
@@ -214,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
     const uint32_t sq = smem_u32(smem + C::kOffQ);
     auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
-      const int ks = j % kKStages;
-      if (!mbar_wait(bar_kfull + 8 * ks, (j / kKStages) & 1)) return false;
+      const int ks = (j - j0) % kKStages;
+      if (!mbar_wait(bar_kfull + 8 * ks, ((j - j0) / kKStages) & 1)) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
@@ -232,9 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j  (P from TMEM)
-      const int vs = j % kVStages;
-      if (!mbar_wait(bar_pfull + 8 * t, j & 1)) return false;
-      if (!mbar_wait(bar_vfull + 8 * vs, (j / kVStages) & 1)) return false;
+      const int vs = (j - j0) % kVStages;
+      if (!mbar_wait(bar_pfull + 8 * t, (j - jb_t[t]) & 1)) return false;
+      if (!mbar_wait(bar_vfull + 8 * vs, ((j - j0) / kVStages) & 1)) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t sv = smem_u32(smem + C::kOffV + vs * C::kTileBytes);
@@ -242,27 +254,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
           umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, umma_desc_sw128(sv + kk * 16 * 128, BKV * 128, 1024),
-                       idesc_o, (j | kk) != 0 ? 1u : 0u);
+                       idesc_o, (j != jb_t[t] || kk != 0) ? 1u : 0u);
         umma_commit(bar_odone + 8 * t);
       }
       __syncwarp();
       return true;
     };
     bool ok = mbar_wait(bar_q, 0);
-    if (ok && n_t[0] > 0) ok = issue_s(0, 0);
-    if (ok && n_t[1] > 0) ok = issue_s(1, 0);
-    for (int j = 0; ok && j < n_kv; ++j) {
-      if (j < n_t[0]) {
-        ok = issue_pv(0, j);
-        if (ok && j + 1 < n_t[0]) ok = issue_s(0, j + 1);
-      }
-      if (ok && j < n_t[1]) {
-        ok = issue_pv(1, j);
-        if (ok && j + 1 < n_t[1]) ok = issue_s(1, j + 1);
+    for (int t = 0; t < 2; ++t)
+      if (ok && jb_t[t] == j0 && j0 < n_t[t]) ok = issue_s(t, j0);
+    for (int j = j0; ok && j < n_kv; ++j) {
+      for (int t = 0; ok && t < 2; ++t) {
+        if (jb_t[t] <= j && j < n_t[t]) ok = issue_pv(t, j);
+        if (ok && jb_t[t] <= j + 1 && j + 1 < n_t[t]) ok = issue_s(t, j + 1);
       }
       if (ok && lane == 0) {
-        umma_commit(bar_kempty + 8 * (j % kKStages));
-        umma_commit(bar_vempty + 8 * (j % kVStages));
+        umma_commit(bar_kempty + 8 * ((j - j0) % kKStages));
+        umma_commit(bar_vempty + 8 * ((j - j0) % kVStages));
       }
       __syncwarp();
     }
@@ -277,15 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = q0 + t * BQ + r;
     const int mrow = min(m, p.M - 1);
     const int row_pos = p.qpos ? p.qpos[mrow] : m;
+    const int row_ks = p.kstart ? p.kstart[mrow] : 0;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_addr = tmem_base + lane_off + t * BKV;
     const uint32_t o_addr = tmem_base + lane_off + 256 + t * 128;
-    const int n = n_t[t];
+    const int n = n_t[t], jb = jb_t[t];
     const float sc = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      if (!mbar_wait(bar_sfull + 8 * t, j & 1)) {
+    for (int j = jb; j < n; ++j) {
+      if (!mbar_wait(bar_sfull + 8 * t, (j - jb) & 1)) {
         ok = false;
         break;
       }
@@ -298,10 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       float* s = reinterpret_cast<float*>(u);
       const int kv0 = j * BKV;
-      if (kv0 + BKV - 1 > pos_first[t] || kv0 + BKV > p.T_kv) {
-        const int lim = min(row_pos, p.T_kv - 1) - kv0;  // last visible column of this row
+      if (kv0 + BKV - 1 > pos_first[t] || kv0 + BKV > p.T_kv || kv0 < ks_last[t]) {
+        const int hi = min(row_pos, p.T_kv - 1) - kv0;  // visible columns of this row: [lo, hi]
+        const int lo = row_ks - kv0;
 #pragma unroll
-        for (int c = 0; c < BKV; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
+        for (int c = 0; c < BKV; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
       }
       float mx[8];
 #pragma unroll
@@ -314,15 +324,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
       bool rescale = false;
       float alpha = 1.f;
-      if (j == 0) {
-        m_run = rmax;  // every row sees key 0, so rmax is finite here
+      if (j == jb) {
+        m_run = rmax;  // -inf if this row's keys start in a later tile
       } else if (__any_sync(0xffffffffu, rmax > m_run + kRescaleThreshold)) {
         const float m_new = fmaxf(m_run, rmax);
-        alpha = ex2_approx(m_run - m_new);
+        // a row still fully masked (-inf - -inf) or unchanged keeps alpha = 1
+        alpha = m_new == m_run ? 1.f : ex2_approx(m_run - m_new);
         m_run = m_new;
         rescale = true;
       }
-      const float neg = -m_run;
+      const float neg = m_run == -INFINITY ? 0.f : -m_run;  // fully masked so far: p = 0
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
@@ -361,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar_pfull + 8 * t);
     }
-    if (ok && n > 0 && mbar_wait(bar_odone + 8 * t, (n - 1) & 1)) {
+    if (ok && n > jb && mbar_wait(bar_odone + 8 * t, (n - 1 - jb) & 1)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       __nv_bfloat16* dst = p.out + static_cast<int64_t>(mrow) * p.ldo + head * HD;

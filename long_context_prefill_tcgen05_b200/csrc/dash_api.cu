@@ -189,8 +189,8 @@ inline int o_proj_tiles(int d) { return d % 256 == 0 ? d / 256 : d / 128; }
 // -------------------------------------------------------------- attention
 template <int HD>
 dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
-                           int64_t T_kv, int hq, int hkv, const int32_t* qpos, bf16* O, int64_t ldo,
-                           cudaStream_t st) {
+                           int64_t T_kv, int hq, int hkv, const int32_t* qpos, const int32_t* kstart, bf16* O,
+                           int64_t ldo, cudaStream_t st) {
   using C = dash::attn::Cfg<HD>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -208,6 +208,7 @@ dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16
   p.out = O;
   p.ldo = ldo;
   p.qpos = qpos;
+  p.kstart = kstart;
   p.M = static_cast<int>(M);
   p.T_kv = static_cast<int>(T_kv);
   p.hq = hq;
@@ -222,24 +223,24 @@ dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16
 }
 
 dash_status attention(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
-                      int64_t T_kv, int hq, int hkv, int hd, const int32_t* qpos, bf16* O, int64_t ldo,
-                      cudaStream_t st) {
+                      int64_t T_kv, int hq, int hkv, int hd, const int32_t* qpos, const int32_t* kstart, bf16* O,
+                      int64_t ldo, cudaStream_t st) {
   if (M == 0) return DASH_OK;
   if (T_kv <= 0 || M > INT32_MAX || T_kv > INT32_MAX || hkv <= 0 || hq % hkv != 0) return DASH_ERR_SHAPE;
-  if (hd == 128) return launch_attn_hd<128>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, O, ldo, st);
-  if (hd == 64) return launch_attn_hd<64>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, O, ldo, st);
+  if (hd == 128) return launch_attn_hd<128>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
+  if (hd == 64) return launch_attn_hd<64>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
   return DASH_ERR_SHAPE;
 }
 
 // ---------------------------------------------------------------- row ops
 dash_status rmsnorm(const bf16* X, int64_t x_rows, const int32_t* rowmap, int64_t rows, int d, const bf16* g,
-                    double eps, bf16* Y, cudaStream_t st) {
+                    double eps, bf16* Y, cudaStream_t st, float* row_scale = nullptr) {
   if (rows == 0) return DASH_OK;
   const int warps = 8;
   const int64_t blocks = (rows + warps - 1) / warps;
   TimedLaunch tl(DASH_K_RMSNORM, rows, d, 0, st);
   dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
-      X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y);
+      X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y, row_scale);
   return launch_status();
 }
 
@@ -291,6 +292,7 @@ struct LayerWs {
   bf16* Act;     // [max(M*F, (T_kv-M)*d)]: SwiGLU output; halt-mode frozen-row norms
   float* ssq_u;  // [o_proj tiles, M]
   float* ssq_h;
+  float* rs;     // [max(M, T_kv - M)] RMSNorm 1/rms per row, applied in the GEMM epilogues
 };
 
 bool dims_ok(const dash_dims* D) {
@@ -317,12 +319,17 @@ void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, C
   const int nt = o_proj_tiles(D.d_model);
   w.ssq_u = c.take<float>(static_cast<size_t>(nt) * M);
   w.ssq_h = c.take<float>(static_cast<size_t>(nt) * M);
+  w.rs = c.take<float>(static_cast<size_t>(M > T_kv - M ? M : T_kv - M));
 }
 
 // One pre-norm decoder block on H [M, d] in place (rope table already built).
+// pos: RoPE position of each row (NULL: row index); kstart: first key each
+// row may attend to (NULL: 0; varlen batches); halted_pos: RoPE positions of
+// the halted rows (NULL: their original index).
 dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_layer_weights& w, bf16* H, int64_t M,
                        const int32_t* pos, const dash_halt_ctx* halt, float* delta, int relative,
-                       const LayerWs& ws, cudaStream_t st) {
+                       const LayerWs& ws, cudaStream_t st, const int32_t* kstart = nullptr,
+                       const int32_t* halted_pos = nullptr) {
   if (M == 0) return DASH_OK;
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd, kvd = hkv * hd;
@@ -344,11 +351,13 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   // original positions ([DASH news] "选择性停止机制").
   if (halt && T_kv > M) {
     const int64_t nh = T_kv - M;
-    if ((s = rmsnorm(cb(halt->h_full), T_kv, halt->halted_idx, nh, d, cb(w.attn_norm), D.rms_eps, ws.Act, st)) != DASH_OK)
+    if ((s = rmsnorm(cb(halt->h_full), T_kv, halt->halted_idx, nh, d, cb(w.attn_norm), D.rms_eps, ws.Act, st,
+                     ws.rs)) != DASH_OK)
       return s;
     EpiArgs kv = qkv;
+    kv.row_scale = ws.rs;
     kv.q = nullptr;
-    kv.pos = halt->halted_idx;
+    kv.pos = halted_pos ? halted_pos : halt->halted_idx;
     kv.kv_rowmap = halt->halted_idx;
     kv.col_offset = qd;
     if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.Act, d, nh, d, cb(w.w_qkv) + static_cast<int64_t>(qd) * d, nullptr,
@@ -356,17 +365,18 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
       return s;
   }
 
-  // a1: input RMSNorm
-  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.attn_norm), D.rms_eps, ws.X, st)) != DASH_OK) return s;
+  // a1: input RMSNorm (its 1/rms is applied to the QKV accumulator)
+  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.attn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
   // a2: QKV projection + RoPE (k/v of active rows land at their original rows in halt mode)
+  qkv.row_scale = ws.rs;
   qkv.pos = pos;
   qkv.kv_rowmap = halt ? halt->active_idx : nullptr;
   qkv.col_offset = 0;
   if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st, DASH_K_GEMM_QKV)) != DASH_OK)
     return s;
   // a3: causal GQA attention -> O (into X)
-  if ((s = attention(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, ws.X,
-                     qd, st)) != DASH_OK)
+  if ((s = attention(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, kstart,
+                     ws.X, qd, st)) != DASH_OK)
     return s;
   // a4: o_proj + residual (+ per-row sums of U^2 and H^2 for Δ)
   EpiArgs o{};
@@ -388,10 +398,11 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
     if ((s = launch_status()) != DASH_OK) return s;
   }
   // a5: post-attention RMSNorm, gate/up GEMM with SwiGLU
-  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.ffn_norm), D.rms_eps, ws.X, st)) != DASH_OK) return s;
+  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.ffn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
   EpiArgs sw{};
   sw.out = ws.Act;
   sw.ldo = F;
+  sw.row_scale = ws.rs;
   if ((s = gemm<dash::gemm::kEpiSwiglu>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st, DASH_K_GEMM_GATE_UP)) != DASH_OK) return s;
   // a6: down projection + residual
   EpiArgs dn{};
@@ -408,33 +419,57 @@ bool weights_ok(const dash_layer_weights* w) {
 
 struct PrefillWs {
   LayerWs L;
-  bf16* Hc;       // [T, d] compacted active rows
-  float* delta;   // [T]
-  int32_t* idx;   // [T]
-  int32_t* halted;// [T]
-  int32_t* count; // [1]
+  bf16* Hc;         // [T, d] compacted active rows
+  float* delta;     // [T]
+  int32_t* idx;     // [T]
+  int32_t* halted;  // [T]
+  int32_t* count;   // [nseq]
+  // varlen batches only (nseq > 1 or a sequence layout given)
+  int32_t* cu;      // [nseq + 1] sequence starts
+  int32_t* cuc;     // [nseq + 1] sequence starts among the active rows
+  int32_t* sel;     // [T] per-sequence selection regions before packing
+  int32_t* selh;    // [T]
+  int32_t* pos;     // [T] RoPE positions of the current rows
+  int32_t* kst;     // [T] first visible key of the current rows
+  int32_t* hpos;    // [T] RoPE positions of halted rows
 };
 
-void carve_prefill(const dash_dims& D, int64_t T, Carver& c, PrefillWs& w) {
+void carve_prefill(const dash_dims& D, int64_t T, int nseq, Carver& c, PrefillWs& w) {
   carve_layer(D, T, T, T, c, w.L);
   w.Hc = c.take<bf16>(static_cast<size_t>(T) * D.d_model);
   w.delta = c.take<float>(static_cast<size_t>(T));
   w.idx = c.take<int32_t>(static_cast<size_t>(T));
   w.halted = c.take<int32_t>(static_cast<size_t>(T));
-  w.count = c.take<int32_t>(1);
+  w.count = c.take<int32_t>(static_cast<size_t>(nseq > 0 ? nseq : 1));
+  const bool varlen = nseq > 1;
+  w.cu = varlen ? c.take<int32_t>(static_cast<size_t>(nseq) + 1) : nullptr;
+  w.cuc = varlen ? c.take<int32_t>(static_cast<size_t>(nseq) + 1) : nullptr;
+  w.sel = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
+  w.selh = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
+  w.pos = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
+  w.kst = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
+  w.hpos = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
 }
 
-dash_status select_impl(const float* scores, int64_t T, int kind, double keep, float thr, int keep_first,
-                        int keep_last, int32_t* idx, int32_t* halted, int32_t* count, cudaStream_t st) {
-  const int64_t lo = keep_first < T ? keep_first : T;
-  int64_t hi = keep_last > 0 ? T - keep_last : T;
-  if (hi < lo) hi = lo;
-  const int64_t n_mid = hi - lo;
-  const int64_t k_dyn = static_cast<int64_t>(std::floor(keep * static_cast<double>(n_mid)));
-  if (T == 0) return cudaMemsetAsync(count, 0, sizeof(int32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
-  TimedLaunch tl(DASH_K_SELECT, T, k_dyn, 0, st);
-  dash::rows::select_kernel<<<1, dash::rows::kSelThreads, 0, st>>>(scores, T, kind, k_dyn, thr, lo, hi, idx, halted,
-                                                                    count);
+dash_status select_impl(const float* scores, int64_t T, const int32_t* seg, int nseg, int kind, double keep,
+                        float thr, int keep_first, int keep_last, int32_t* idx, int32_t* halted, int32_t* count,
+                        cudaStream_t st) {
+  if (T == 0 || nseg == 0)
+    return cudaMemsetAsync(count, 0, sizeof(int32_t) * (nseg > 0 ? nseg : 1), st) == cudaSuccess ? DASH_OK
+                                                                                            : DASH_ERR_CUDA;
+  TimedLaunch tl(DASH_K_SELECT, T, nseg, 0, st);
+  dash::rows::select_kernel<<<nseg, dash::rows::kSelThreads, 0, st>>>(scores, T, seg, kind, keep, thr, keep_first,
+                                                                       keep_last, idx, halted, count);
+  return launch_status();
+}
+
+dash_status seq_layout(const int32_t* cu, int nseq, const int32_t* rows, int64_t M, const int32_t* kspace,
+                       int32_t* pos, int32_t* kstart, const DeviceInfo& di, cudaStream_t st) {
+  if (M == 0) return DASH_OK;
+  int64_t blocks = (M + 255) / 256;
+  if (blocks > di.num_sms * 8) blocks = di.num_sms * 8;
+  dash::rows::seq_layout_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(cu, nseq, rows, M, kspace, pos,
+                                                                               kstart);
   return launch_status();
 }
 
@@ -461,10 +496,186 @@ dash_status noalloc_scratch(void** out) {
   return DASH_OK;
 }
 
+// A wait that nothing will ever satisfy: the bounded wait must give up,
+// record kDevErrTimeout and let the kernel return (the failure path of every
+// pipelined kernel, exercised without faulting the GPU).
+__global__ void wait_timeout_selftest_kernel(int* done) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    dash::mbar_init(dash::smem_u32(&bar), 1);
+    dash::fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = dash::mbar_wait(dash::smem_u32(&bar), 0);
+  if (threadIdx.x == 0) done[0] = ok ? 1 : 2;
+}
+
 __global__ void exp2_fma_kernel(const float* __restrict__ x, int64_t n, float* __restrict__ y) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     y[i] = dash::attn::ex2_fma(x[i]);
+}
+
+
+dash_status check_config(const dash_dims* dims, const dash_config* cfg) {
+  if (cfg->mode != DASH_MODE_PRUNE && cfg->mode != DASH_MODE_HALT && cfg->mode != DASH_MODE_DENSE)
+    return DASH_ERR_INVALID_ARG;
+  if (cfg->mode != DASH_MODE_DENSE) {
+    if (cfg->halt_layer < 0 || cfg->halt_layer >= dims->n_layers) return DASH_ERR_INVALID_ARG;
+    if (cfg->select != DASH_SELECT_TOPK && cfg->select != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
+    if (cfg->score != DASH_SCORE_ABS && cfg->score != DASH_SCORE_REL) return DASH_ERR_INVALID_ARG;
+    if (cfg->select == DASH_SELECT_TOPK && !(cfg->keep_ratio >= 0.0 && cfg->keep_ratio <= 1.0))
+      return DASH_ERR_INVALID_ARG;
+    if (cfg->keep_first < 0 || cfg->keep_last < 0) return DASH_ERR_INVALID_ARG;
+  }
+  return DASH_OK;
+}
+
+// Single-shot DASH prefill over nseq independent sequences concatenated in H
+// (sequence s = rows [cu[s], cu[s+1]), cu in host memory): block-diagonal
+// causal attention, RoPE positions counted from each sequence's start, and a
+// separate selection per sequence ([DASH blog] §5.1: decisions are made per
+// sample).  nseq == 1 is the plain single-sequence prefill.
+dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, const int32_t* cu,
+                         int nseq, const dash_config* cfg, int32_t* idx_out, int64_t* K_out, int32_t* seq_counts,
+                         float* delta_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
+  if (!layers || !H || !cfg || !aligned16(H)) return DASH_ERR_INVALID_ARG;
+  const int64_t T = cu[nseq];
+  if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
+  dash_status s = check_config(dims, cfg);
+  if (s != DASH_OK) return s;
+  for (int l = 0; l < dims->n_layers; ++l)
+    if (!weights_ok(&layers[l])) return DASH_ERR_INVALID_ARG;
+  if (T == 0) {
+    if (K_out) *K_out = 0;
+    if (seq_counts)
+      for (int q = 0; q < nseq; ++q) seq_counts[q] = 0;
+    return DASH_OK;
+  }
+  Carver probe{nullptr};
+  PrefillWs sizes;
+  carve_prefill(*dims, T, nseq, probe, sizes);
+  if (!ws || ws_bytes < probe.off + 256) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  if ((s = device_info(&di)) != DASH_OK) return s;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  PrefillWs P;
+  carve_prefill(*dims, T, nseq, c, P);
+  cudaStream_t st = as_stream(stream);
+  bf16* h = reinterpret_cast<bf16*>(H);
+  const dash_dims& D = *dims;
+  const bool varlen = nseq > 1;
+  if ((s = rope_table(P.L.rope, T, D.head_dim, D.rope_theta, *di, st)) != DASH_OK) return s;
+
+  // Row layout of the full sequence(s): RoPE positions and key starts.
+  const int32_t* pos_full = nullptr;
+  const int32_t* kst_full = nullptr;
+  if (varlen) {
+    if (cudaMemcpyAsync(P.cu, cu, sizeof(int32_t) * (nseq + 1), cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DASH_ERR_CUDA;
+    if ((s = seq_layout(P.cu, nseq, nullptr, T, nullptr, P.pos, P.kst, *di, st)) != DASH_OK) return s;
+    pos_full = P.pos;
+    kst_full = P.kst;
+  }
+
+  auto run_layers = [&](int l0, int l1, bf16* rows, int64_t M, const int32_t* pos, const dash_halt_ctx* hc,
+                        const int32_t* kst, const int32_t* hpos, int delta_layer, float* delta) -> dash_status {
+    for (int l = l0; l < l1; ++l) {
+      g_timing.layer = l;
+      const dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, l == delta_layer ? delta : nullptr,
+                                       cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos);
+      g_timing.layer = -1;
+      if (r != DASH_OK) return r;
+    }
+    return DASH_OK;
+  };
+
+  if (cfg->mode == DASH_MODE_DENSE) {
+    if ((s = run_layers(0, D.n_layers, h, T, pos_full, nullptr, kst_full, nullptr, -1, nullptr)) != DASH_OK) return s;
+    if (K_out) *K_out = T;
+    if (seq_counts)
+      for (int q = 0; q < nseq; ++q) seq_counts[q] = cu[q + 1] - cu[q];
+    return DASH_OK;
+  }
+
+  // Layers 0..L_s on all T tokens; Δ from the halting layer's o_proj epilogue.
+  const int Ls = cfg->halt_layer;
+  float* delta = delta_out ? delta_out : P.delta;
+  if ((s = run_layers(0, Ls + 1, h, T, pos_full, nullptr, kst_full, nullptr, Ls, delta)) != DASH_OK) return s;
+
+  // One-shot selection of the active set S*, per sequence.
+  int32_t* idx = idx_out ? idx_out : P.idx;
+  std::vector<int32_t> counts(static_cast<size_t>(nseq));
+  if ((s = select_impl(delta, T, varlen ? P.cu : nullptr, nseq, cfg->select, cfg->keep_ratio, cfg->threshold,
+                       cfg->keep_first, cfg->keep_last, varlen ? P.sel : idx, varlen ? P.selh : P.halted, P.count,
+                       st)) != DASH_OK)
+    return s;
+  if (cudaMemcpyAsync(counts.data(), P.count, sizeof(int32_t) * nseq, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  int64_t K = 0;
+  for (int q = 0; q < nseq; ++q) {
+    if (counts[q] < 0) return DASH_ERR_NONFINITE;
+    K += counts[q];
+  }
+  if (K_out) *K_out = K;
+  if (seq_counts)
+    for (int q = 0; q < nseq; ++q) seq_counts[q] = counts[q];
+  if (varlen) {
+    // Pack the per-sequence regions into contiguous ascending lists.
+    std::vector<int32_t> cuc(static_cast<size_t>(nseq) + 1, 0);
+    int64_t hoff = 0;
+    for (int q = 0; q < nseq; ++q) {
+      const int64_t len = cu[q + 1] - cu[q], kq = counts[q];
+      cuc[q + 1] = cuc[q] + counts[q];
+      if (kq > 0 && cudaMemcpyAsync(idx + cuc[q], P.sel + cu[q], sizeof(int32_t) * kq, cudaMemcpyDeviceToDevice,
+                                    st) != cudaSuccess)
+        return DASH_ERR_CUDA;
+      if (len - kq > 0 && cudaMemcpyAsync(P.halted + hoff, P.selh + cu[q], sizeof(int32_t) * (len - kq),
+                                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return DASH_ERR_CUDA;
+      hoff += len - kq;
+    }
+    // (a copy from pageable host memory has consumed its source when it returns)
+    if (cudaMemcpyAsync(P.cuc, cuc.data(), sizeof(int32_t) * (nseq + 1), cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DASH_ERR_CUDA;
+  }
+
+  // Gather the active rows; later layers run on them only.
+  if ((s = move_rows(false, h, P.Hc, idx, K, T, D.d_model, *di, st)) != DASH_OK) return s;
+  if (cfg->mode == DASH_MODE_PRUNE) {
+    const int32_t* pos_c = idx;  // original positions
+    const int32_t* kst_c = nullptr;
+    if (varlen) {  // positions within each sequence; keys from the sequence's first active row
+      if ((s = seq_layout(P.cu, nseq, idx, K, P.cuc, P.pos, P.kst, *di, st)) != DASH_OK) return s;
+      pos_c = P.pos;
+      kst_c = P.kst;
+    }
+    if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_c, nullptr, kst_c, nullptr, -1, nullptr)) != DASH_OK)
+      return s;
+    if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16),
+                                 cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return DASH_ERR_CUDA;
+    return DASH_OK;
+  }
+  dash_halt_ctx hc;
+  hc.active_idx = idx;
+  hc.halted_idx = P.halted;
+  hc.h_full = H;
+  hc.T = T;
+  const int32_t* pos_a = idx;
+  const int32_t* kst_a = nullptr;
+  const int32_t* hpos = nullptr;
+  if (varlen) {
+    if ((s = seq_layout(P.cu, nseq, idx, K, nullptr, P.pos, P.kst, *di, st)) != DASH_OK) return s;
+    if ((s = seq_layout(P.cu, nseq, P.halted, T - K, nullptr, P.hpos, nullptr, *di, st)) != DASH_OK) return s;
+    pos_a = P.pos;
+    kst_a = P.kst;
+    hpos = P.hpos;
+  }
+  if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_a, &hc, kst_a, hpos, -1, nullptr)) != DASH_OK) return s;
+  return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
 }
 
 }  // namespace
@@ -530,7 +741,7 @@ dash_status dash_select(const float* scores, int64_t T, int32_t kind, double kee
   if (kind != DASH_SELECT_TOPK && kind != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
   if (keep_first < 0 || keep_last < 0) return DASH_ERR_INVALID_ARG;
   if (kind == DASH_SELECT_TOPK && !(keep_ratio >= 0.0 && keep_ratio <= 1.0)) return DASH_ERR_INVALID_ARG;
-  return select_impl(scores, T, kind, keep_ratio, threshold, keep_first, keep_last, idx, halted, count,
+  return select_impl(scores, T, nullptr, 1, kind, keep_ratio, threshold, keep_first, keep_last, idx, halted, count,
                      as_stream(stream));
 }
 
@@ -582,6 +793,14 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
                                      nullptr, N, ep, as_stream(stream), DASH_K_GEMM);
 }
 
+dash_status dash_selftest_wait_timeout(int32_t* done) {
+  if (!done) return DASH_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DASH_ERR_CUDA;
+  wait_timeout_selftest_kernel<<<1, 32>>>(done);
+  if (cudaGetLastError() != cudaSuccess) return DASH_ERR_CUDA;
+  return dash_device_error();
+}
+
 dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream) {
   if (n < 0) return DASH_ERR_SHAPE;
   if (n == 0) return DASH_OK;
@@ -592,7 +811,8 @@ dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream) {
 }
 
 dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf16* V, int64_t M, int64_t T_kv,
-                           int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos, dash_bf16* O, void* stream) {
+                           int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos, const int32_t* kstart,
+                           dash_bf16* O, void* stream) {
   if (M < 0 || T_kv < 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || (hd != 64 && hd != 128)) return DASH_ERR_SHAPE;
   if (M == 0) return DASH_OK;
   if (T_kv == 0) return DASH_ERR_SHAPE;
@@ -604,8 +824,8 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
   if (s != DASH_OK) return s;
   const int64_t qd = static_cast<int64_t>(hq) * hd, kvd = static_cast<int64_t>(hkv) * hd;
   return attention(reinterpret_cast<const bf16*>(Q), qd, reinterpret_cast<const bf16*>(K),
-                   reinterpret_cast<const bf16*>(V), kvd, M, T_kv, hq, hkv, hd, qpos, reinterpret_cast<bf16*>(O), qd,
-                   as_stream(stream));
+                   reinterpret_cast<const bf16*>(V), kvd, M, T_kv, hq, hkv, hd, qpos, kstart,
+                   reinterpret_cast<bf16*>(O), qd, as_stream(stream));
 }
 
 size_t dash_layer_workspace_size(const dash_dims* dims, int64_t M, int64_t T_kv, int64_t max_pos) {
@@ -666,105 +886,36 @@ size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_
   if (!dims_ok(dims) || T < 0 || !cfg) return 0;
   Carver c{nullptr};
   PrefillWs w;
-  carve_prefill(*dims, T, c, w);
+  carve_prefill(*dims, T, 1, c, w);
+  return c.off + 256;
+}
+
+size_t dash_prefill_varlen_workspace_size(const dash_dims* dims, int64_t T, int32_t nseq, const dash_config* cfg) {
+  if (!dims_ok(dims) || T < 0 || nseq < 1 || !cfg) return 0;
+  Carver c{nullptr};
+  PrefillWs w;
+  carve_prefill(*dims, T, nseq, c, w);
   return c.off + 256;
 }
 
 dash_status dash_prefill(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, int64_t T,
                          const dash_config* cfg, int32_t* idx_out, int64_t* K_out, float* delta_out, void* ws,
                          size_t ws_bytes, void* stream) {
-  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
-  if (!layers || !H || !cfg || !aligned16(H)) return DASH_ERR_INVALID_ARG;
   if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
-  if (cfg->mode != DASH_MODE_PRUNE && cfg->mode != DASH_MODE_HALT && cfg->mode != DASH_MODE_DENSE)
-    return DASH_ERR_INVALID_ARG;
-  if (cfg->mode != DASH_MODE_DENSE) {
-    if (cfg->halt_layer < 0 || cfg->halt_layer >= dims->n_layers) return DASH_ERR_INVALID_ARG;
-    if (cfg->select != DASH_SELECT_TOPK && cfg->select != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
-    if (cfg->score != DASH_SCORE_ABS && cfg->score != DASH_SCORE_REL) return DASH_ERR_INVALID_ARG;
-    if (cfg->select == DASH_SELECT_TOPK && !(cfg->keep_ratio >= 0.0 && cfg->keep_ratio <= 1.0))
-      return DASH_ERR_INVALID_ARG;
-    if (cfg->keep_first < 0 || cfg->keep_last < 0) return DASH_ERR_INVALID_ARG;
-  }
-  for (int l = 0; l < dims->n_layers; ++l)
-    if (!weights_ok(&layers[l])) return DASH_ERR_INVALID_ARG;
-  if (T == 0) {
-    if (K_out) *K_out = 0;
-    return DASH_OK;
-  }
-  const size_t need = dash_prefill_workspace_size(dims, T, cfg);
-  if (!ws || ws_bytes < need) return DASH_ERR_NO_MEMORY;
-  DeviceInfo* di;
-  dash_status s = device_info(&di);
-  if (s != DASH_OK) return s;
-  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
-  PrefillWs P;
-  carve_prefill(*dims, T, c, P);
-  cudaStream_t st = as_stream(stream);
-  bf16* h = reinterpret_cast<bf16*>(H);
-  const dash_dims& D = *dims;
-  if ((s = rope_table(P.L.rope, T, D.head_dim, D.rope_theta, *di, st)) != DASH_OK) return s;
+  const int32_t cu[2] = {0, static_cast<int32_t>(T)};
+  return prefill_impl(dims, layers, H, cu, 1, cfg, idx_out, K_out, nullptr, delta_out, ws, ws_bytes, stream);
+}
 
-  if (cfg->mode == DASH_MODE_DENSE) {
-    for (int l = 0; l < D.n_layers; ++l) {
-      g_timing.layer = l;
-      s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, nullptr, 0, P.L, st);
-      g_timing.layer = -1;
-      if (s != DASH_OK) return s;
-    }
-    if (K_out) *K_out = T;
-    return DASH_OK;
-  }
-
-  // Layers 0..L_s on all T tokens; Δ from the halting layer's o_proj epilogue.
-  const int Ls = cfg->halt_layer;
-  float* delta = delta_out ? delta_out : P.delta;
-  for (int l = 0; l <= Ls; ++l) {
-    g_timing.layer = l;
-    s = layer_impl(*di, D, layers[l], h, T, nullptr, nullptr, l == Ls ? delta : nullptr,
-                   cfg->score == DASH_SCORE_REL, P.L, st);
-    g_timing.layer = -1;
-    if (s != DASH_OK) return s;
-  }
-  // One-shot selection of the active set S*.
-  int32_t* idx = idx_out ? idx_out : P.idx;
-  if ((s = select_impl(delta, T, cfg->select, cfg->keep_ratio, cfg->threshold, cfg->keep_first, cfg->keep_last,
-                       idx, P.halted, P.count, st)) != DASH_OK)
-    return s;
-  int32_t K32 = 0;
-  if (cudaMemcpyAsync(&K32, P.count, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return DASH_ERR_CUDA;
-  if (K32 < 0) return DASH_ERR_NONFINITE;
-  const int64_t K = K32;
-  if (K_out) *K_out = K;
-
-  // Gather the active rows; later layers run on them only.
-  if ((s = move_rows(false, h, P.Hc, idx, K, T, D.d_model, *di, st)) != DASH_OK) return s;
-  if (cfg->mode == DASH_MODE_PRUNE) {
-    for (int l = Ls + 1; l < D.n_layers; ++l) {
-      g_timing.layer = l;
-      s = layer_impl(*di, D, layers[l], P.Hc, K, idx, nullptr, nullptr, 0, P.L, st);
-      g_timing.layer = -1;
-      if (s != DASH_OK) return s;
-    }
-    if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16), cudaMemcpyDeviceToDevice,
-                                 st) != cudaSuccess)
-      return DASH_ERR_CUDA;
-    return DASH_OK;
-  }
-  dash_halt_ctx hc;
-  hc.active_idx = idx;
-  hc.halted_idx = P.halted;
-  hc.h_full = H;
-  hc.T = T;
-  for (int l = Ls + 1; l < D.n_layers; ++l) {
-    g_timing.layer = l;
-    s = layer_impl(*di, D, layers[l], P.Hc, K, idx, &hc, nullptr, 0, P.L, st);
-    g_timing.layer = -1;
-    if (s != DASH_OK) return s;
-  }
-  return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
+dash_status dash_prefill_varlen(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H,
+                                const int32_t* cu_seqlens, int32_t nseq, const dash_config* cfg, int32_t* idx_out,
+                                int64_t* K_out, int32_t* seq_counts, float* delta_out, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (!cu_seqlens || nseq < 1) return DASH_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return DASH_ERR_INVALID_ARG;
+  for (int s = 0; s < nseq; ++s)
+    if (cu_seqlens[s + 1] < cu_seqlens[s]) return DASH_ERR_INVALID_ARG;
+  return prefill_impl(dims, layers, H, cu_seqlens, nseq, cfg, idx_out, K_out, seq_counts, delta_out, ws, ws_bytes,
+                      stream);
 }
 
 dash_status dash_timing_start(int32_t capacity) {

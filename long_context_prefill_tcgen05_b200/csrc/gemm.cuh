@@ -45,6 +45,7 @@ struct EpiArgs {
   const int32_t* pos;        // RoPE position of row m (NULL: m)
   const int32_t* kv_rowmap;  // k/v destination row of row m (NULL: m)
   const float4* rope;        // [max_pos, hd/2] float2 (cos, sin), read as float4 pairs
+  const float* row_scale;    // [M] or NULL: per-row factor on the accumulator (RMSNorm 1/rms)
   int col_offset;            // qkv column of this GEMM's column 0
   int hq, hkv, hd;
 };
@@ -143,11 +144,12 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
       tmem_ld32(tbase + BN / 2 + c, u);
       tmem_ld_wait();
       if (live) {
+        const float sc = ep.row_scale ? ep.row_scale[m] : 1.f;
         float o[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float gf = __uint_as_float(g[i]);
-          o[i] = gf / (1.f + __expf(-gf)) * __uint_as_float(u[i]);
+          const float gf = __uint_as_float(g[i]) * sc;
+          o[i] = gf / (1.f + __expf(-gf)) * (__uint_as_float(u[i]) * sc);
         }
         store32_bf16(ep.out + static_cast<int64_t>(m) * ep.ldo + tn * (BN / 2) + c, o);
       }
@@ -155,9 +157,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
   } else {  // kEpiQkv
     const int hd = ep.hd, half = hd >> 1;
     int p = 0, kvrow = 0;
+    float sc = 1.f;
     if (live) {
       p = ep.pos ? ep.pos[m] : m;
       kvrow = ep.kv_rowmap ? ep.kv_rowmap[m] : m;
+      if (ep.row_scale) sc = ep.row_scale[m];
     }
 #pragma unroll 1
     for (int hb = 0; hb < BN / hd; ++hb) {
@@ -186,8 +190,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float4 t = cs[i];  // (cos_2i, sin_2i, cos_2i+1, sin_2i+1)
-              const float a0 = __uint_as_float(x1[2 * i]), b0 = __uint_as_float(x2[2 * i]);
-              const float a1 = __uint_as_float(x1[2 * i + 1]), b1 = __uint_as_float(x2[2 * i + 1]);
+              const float a0 = __uint_as_float(x1[2 * i]) * sc, b0 = __uint_as_float(x2[2 * i]) * sc;
+              const float a1 = __uint_as_float(x1[2 * i + 1]) * sc, b1 = __uint_as_float(x2[2 * i + 1]) * sc;
               y1[2 * i] = a0 * t.x - b0 * t.y;
               y2[2 * i] = b0 * t.x + a0 * t.y;
               y1[2 * i + 1] = a1 * t.z - b1 * t.w;
@@ -206,7 +210,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
           if (live) {
             float o[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]) * sc;
             store32_bf16(dst + c, o);
           }
         }

@@ -32,10 +32,14 @@ __device__ __forceinline__ float sumsq8(const uint4& v) {
 // y[r] = x[src(r)] * rsqrt(mean(x^2) + eps) * g, one warp per row, fp32 math.
 // src(r) = rowmap[r] when a row map is given (halt mode normalises the frozen
 // rows straight from the full hidden-state buffer).
+// With row_scale given, the kernel writes y[r] = x[src(r)] * g and
+// row_scale[r] = rsqrt(mean(x^2) + eps) instead: the GEMM that consumes y
+// applies the scale to its fp32 accumulator, so the normalised activation is
+// never rounded to bf16 (x * g is exact in bf16 when g = 1).
 __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_rows,
                                const int32_t* __restrict__ rowmap, int64_t rows, int d,
                                const __nv_bfloat16* __restrict__ g, float eps,
-                               __nv_bfloat16* __restrict__ y) {
+                               __nv_bfloat16* __restrict__ y, float* __restrict__ row_scale) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
   if (r >= rows) return;
@@ -60,7 +64,11 @@ __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_ro
     }
   }
   ss = warp_sum(ss);
-  const float rs = rsqrtf(ss / static_cast<float>(d) + eps);
+  float rs = rsqrtf(ss / static_cast<float>(d) + eps);
+  if (row_scale) {
+    if (lane == 0) row_scale[r] = rs;
+    rs = 1.f;
+  }
   const uint4* gr = reinterpret_cast<const uint4*>(g);
   uint4* yr = reinterpret_cast<uint4*>(y + r * d);
 #pragma unroll
@@ -162,24 +170,38 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
   return res;
 }
 
-// Single-CTA selection over T scores.
+// Selection over T scores, one CTA per segment (one sequence of a varlen
+// batch; a single segment [0, T) when seg is NULL).  Within segment b,
+// [s0, s1) = [seg[b], seg[b+1]):
 //   kind 0 (top-k): among tokens in [lo, hi) choose the k_dyn best by
 //     (score desc, index asc); kind 1 (threshold): score >= thr.
-//   Tokens outside [lo, hi) (the forced first / last tokens) are always kept.
-// Writes the kept indices ascending to idx, the others to halted (optional),
-// and the count to count[0]; a NaN/Inf score writes count = -3 instead.
+//   Tokens outside [lo, hi) (the first keep_first / last keep_last tokens of
+//   the segment) are always kept; k_dyn = floor(keep * (hi - lo)) in double.
+// Writes the kept (absolute) indices ascending to idx[s0 ...], the others to
+// halted[s0 ...] (optional), and the count to count[b]; a NaN/Inf score in
+// the segment writes count[b] = -3 instead.
 // Top-k finds the k-th key by an 8-bit MSB-first radix select over
 // shared-memory histograms, then compacts in index order with block-wide
 // ballot prefix sums; among keys equal to the k-th, the lowest indices win.
 __global__ void __launch_bounds__(kSelThreads, 1)
-    select_kernel(const float* __restrict__ scores, int64_t T, int kind, int64_t k_dyn, float thr,
-                  int64_t lo, int64_t hi, int32_t* __restrict__ idx, int32_t* __restrict__ halted,
-                  int32_t* __restrict__ count) {
+    select_kernel(const float* __restrict__ scores_all, int64_t T_all, const int32_t* __restrict__ seg, int kind,
+                  double keep, float thr, int keep_first, int keep_last, int32_t* __restrict__ idx_all,
+                  int32_t* __restrict__ halted_all, int32_t* __restrict__ count_all) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[65];
   __shared__ uint32_t s_prefix, s_k;
   __shared__ int s_bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t s0 = seg ? seg[blockIdx.x] : 0;
+  const int64_t T = seg ? seg[blockIdx.x + 1] - s0 : T_all;
+  const float* scores = scores_all + s0;
+  int32_t* idx = idx_all + s0;
+  int32_t* halted = halted_all ? halted_all + s0 : nullptr;
+  int32_t* count = count_all + blockIdx.x;
+  const int64_t lo = keep_first < T ? keep_first : T;
+  int64_t hi = keep_last > 0 ? T - keep_last : T;
+  if (hi < lo) hi = lo;
+  const int64_t k_dyn = kind == 0 ? static_cast<int64_t>(floor(keep * static_cast<double>(hi - lo))) : 0;
 
   if (tid == 0) s_bad = 0;
   __syncthreads();
@@ -230,21 +252,14 @@ __global__ void __launch_bounds__(kSelThreads, 1)
           cnt[i] = hist[8 * lane + i];
           own += cnt[i];
         }
-        uint32_t above = 0;  // keys in bins of higher lanes
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t n = __shfl_down_sync(0xffffffffu, above + own, o);
-          // accumulate suffix sums of `own` over lanes > lane
-          (void)n;
-        }
-        // plain suffix sum: incl[l] = sum_{l' >= l} own[l']
+        // suffix sum over lanes: incl[l] = keys in bins of lanes >= l
         uint32_t incl = own;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t n = __shfl_down_sync(0xffffffffu, incl, o);
           if (lane + o < 32) incl += n;
         }
-        above = incl - own;
+        const uint32_t above = incl - own;  // keys in bins of higher lanes
         if (above < k && k <= incl) {
           uint32_t acc = above;
           int b = 7;
@@ -311,14 +326,36 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 #pragma unroll
     for (int i = 0; i < kSelPerThread; ++i) {
       if (!valid[i]) continue;
-      if (sel[i]) idx[ps++] = static_cast<int32_t>(t0 + i);
-      else if (halted) halted[ph++] = static_cast<int32_t>(t0 + i);
+      if (sel[i]) idx[ps++] = static_cast<int32_t>(s0 + t0 + i);
+      else if (halted) halted[ph++] = static_cast<int32_t>(s0 + t0 + i);
     }
     sel_base += tot_pk >> 16;
     hal_base += tot_pk & 0xffffu;
     eq_base += tot_eq;
   }
   if (tid == 0) count[0] = static_cast<int32_t>(sel_base);
+}
+
+// ---------------------------------------------------------- varlen layout
+// For each row i (original token orig = rows ? rows[i] : i) of a varlen batch
+// with sequence starts cu[0..nseq]: pos[i] = orig - cu[s] (the RoPE position
+// within its sequence s) and, when kstart is given, kstart[i] = kspace[s] (or
+// cu[s] without kspace): the first key the row may attend to.
+__global__ void seq_layout_kernel(const int32_t* __restrict__ cu, int nseq, const int32_t* __restrict__ rows,
+                                  int64_t M, const int32_t* __restrict__ kspace, int32_t* __restrict__ pos,
+                                  int32_t* __restrict__ kstart) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < M;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t orig = rows ? rows[i] : static_cast<int32_t>(i);
+    int a = 0, b = nseq;  // largest s with cu[s] <= orig
+    while (b - a > 1) {
+      const int mid = (a + b) >> 1;
+      if (cu[mid] <= orig) a = mid;
+      else b = mid;
+    }
+    if (pos) pos[i] = orig - cu[a];
+    if (kstart) kstart[i] = kspace ? kspace[a] : cu[a];
+  }
 }
 
 // -------------------------------------------------------- gather / scatter

@@ -68,10 +68,15 @@ _SIGS = {
                              c_vp, ctypes.POINTER(c_i64), c_vp, c_vp, c_sz, c_vp]),
     "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
     "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
-    "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "dash_prefill_varlen_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i64, c_i32, ctypes.POINTER(Config)]),
+    "dash_prefill_varlen": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp,
+                                    ctypes.POINTER(c_i32), c_i32, ctypes.POINTER(Config), c_vp,
+                                    ctypes.POINTER(c_i64), ctypes.POINTER(c_i32), c_vp, c_vp, c_sz, c_vp]),
     "dash_layer_forward_noalloc": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, c_vp,
                                            c_i64, ctypes.POINTER(HaltCtx), c_vp, c_i32, c_vp]),
     "dash_exp2_fma": (c_i32, [c_vp, c_i64, c_vp, c_vp]),
+    "dash_selftest_wait_timeout": (c_i32, [c_vp]),
     "dash_timing_start": (c_i32, [c_i32]),
     "dash_timing_stop": (c_i32, [ctypes.POINTER(LaunchRecord), c_i32]),
     "dash_kernel_name": (ctypes.c_char_p, [c_i32]),
@@ -222,10 +227,10 @@ def exp2_fma(x, stream=None):
     return y
 
 
-def attention(Q, K, V, hq, hkv, hd, qpos=None, out=None, stream=None):
+def attention(Q, K, V, hq, hkv, hd, qpos=None, kstart=None, out=None, stream=None):
     M = Q.shape[0]
     out = torch.empty(M, hq * hd, dtype=Q.dtype, device=Q.device) if out is None else out
-    _check(lib().dash_attention(_p(Q), _p(K), _p(V), M, K.shape[0], hq, hkv, hd, _p(qpos), _p(out),
+    _check(lib().dash_attention(_p(Q), _p(K), _p(V), M, K.shape[0], hq, hkv, hd, _p(qpos), _p(kstart), _p(out),
                                 _stream(stream)), "dash_attention")
     return out
 
@@ -276,6 +281,23 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
 def make_config(halt_layer=0, mode="prune", select="topk", keep=0.5, threshold=0.0, relative=False,
                 keep_first=0, keep_last=0):
     return Config(halt_layer, MODES[mode], SELECTS[select], int(relative), keep, threshold, keep_first, keep_last)
+
+
+def prefill_varlen(stack, H, cu_seqlens, cfg, idx_out=None, delta_out=None, stream=None):
+    """dash_prefill_varlen in place on H [T, d] for the sequences cu_seqlens
+    (host ints, length nseq + 1); returns (K, per-sequence active counts)."""
+    cu = [int(x) for x in cu_seqlens]
+    nseq = len(cu) - 1
+    T = H.shape[0]
+    need = lib().dash_prefill_varlen_workspace_size(ctypes.byref(stack.dims), T, nseq, ctypes.byref(cfg))
+    ws = workspace(need, H.device)
+    cu_arr = (c_i32 * (nseq + 1))(*cu)
+    counts = (c_i32 * nseq)()
+    K = c_i64(0)
+    _check(lib().dash_prefill_varlen(ctypes.byref(stack.dims), stack.layers, _p(H), cu_arr, nseq, ctypes.byref(cfg),
+                                     _p(idx_out), ctypes.byref(K), counts, _p(delta_out), _p(ws), ws.numel(),
+                                     _stream(stream)), "dash_prefill_varlen")
+    return K.value, list(counts)
 
 
 def prefill(stack, H, cfg, idx_out=None, delta_out=None, stream=None):

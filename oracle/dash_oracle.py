@@ -62,7 +62,7 @@ __all__ = [
     "rms_norm", "rope_inv_freq", "apply_rope", "causal_gqa_attention", "silu",
     "swiglu", "decoder_block", "dense_forward", "delta_scores", "forced_mask",
     "topk_count", "select_topk", "select_threshold", "gather_rows",
-    "scatter_rows", "dash_prefill", "OracleError",
+    "scatter_rows", "dash_prefill", "dash_prefill_varlen", "OracleError",
 ]
 
 
@@ -155,6 +155,8 @@ def decoder_block(h_q, q_pos, h_kv, kv_pos, w, dims):
     hq, hkv, hd = dims["n_heads"], dims["n_kv_heads"], dims["head_dim"]
     h_q = np.asarray(h_q, dtype=np.float64)
     h_kv = np.asarray(h_kv, dtype=np.float64)
+    if len(h_q) == 0:  # no active rows: nothing to update
+        return h_q.copy(), np.zeros_like(h_q)
     a_q = rms_norm(h_q, w["attn_norm"], eps)
     a_kv = rms_norm(h_kv, w["attn_norm"], eps)
     q = apply_rope((a_q @ w["wq"].T).reshape(len(h_q), hq, hd), q_pos, theta)
@@ -304,3 +306,36 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
         raise OracleError(f"unknown mode {mode!r}")
     return {"hidden": hidden, "idx": idx, "delta": delta,
             "halt_out": halt_out, "halt_in": h_in}
+
+
+def dash_prefill_varlen(h0, cu_seqlens, layers, dims, halt_layer, mode="prune", forced_idx=None, **kw):
+    """A batch of independent sequences ([DASH blog] §5.1: every sample takes
+    its own decision; gather/scatter must not mix samples).
+
+    Sequence s is rows [cu[s], cu[s+1]) of h0.  The result is, by definition,
+    the single-sequence prefill applied to each sequence on its own (RoPE
+    positions from 0, attention within the sequence, its own selection),
+    concatenated in order; idx holds absolute row numbers.  forced_idx, when
+    given, is a global ascending index list split by sequence.
+    """
+    cu = [int(x) for x in cu_seqlens]
+    h0 = np.asarray(h0, dtype=np.float64)
+    hidden, idx, delta, counts = [], [], [], []
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        f = None
+        if forced_idx is not None:
+            g = np.asarray(forced_idx)
+            f = g[(g >= a) & (g < b)] - a
+        if b == a:
+            counts.append(0)
+            continue
+        r = dash_prefill(h0[a:b], layers, dims, halt_layer, mode, forced_idx=f, **kw)
+        hidden.append(r["hidden"])
+        idx.append(r["idx"] + a)
+        delta.append(r["delta"])
+        counts.append(len(r["idx"]))
+    d = h0.shape[1]
+    return {"hidden": np.concatenate(hidden) if hidden else np.zeros((0, d)),
+            "idx": np.concatenate(idx).astype(np.int64) if idx else np.zeros(0, np.int64),
+            "delta": np.concatenate(delta) if delta else np.zeros(0), "counts": counts}

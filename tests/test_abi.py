@@ -88,8 +88,20 @@ def test_argument_errors_are_caught_on_the_host(L):
     assert L.dash_score(FAKE, None, 10, 64, 1, FAKE, None) == 1          # relative needs H
     assert L.dash_compact(FAKE, 10, FAKE, 5, 12, FAKE, None) == 2
     assert L.dash_linear(FAKE, 10, 100, FAKE, 128, FAKE, None) == 2      # K % 64
-    assert L.dash_attention(FAKE, FAKE, FAKE, 10, 10, 4, 2, 96, None, FAKE, None) == 2
-    assert L.dash_attention(FAKE, FAKE, FAKE, 20, 10, 4, 2, 64, None, FAKE, None) == 2  # M > T_kv causal
+    assert L.dash_attention(FAKE, FAKE, FAKE, 10, 10, 4, 2, 96, None, None, FAKE, None) == 2
+    assert L.dash_attention(FAKE, FAKE, FAKE, 20, 10, 4, 2, 64, None, None, FAKE, None) == 2  # M > T_kv causal
+
+    # varlen: cu_seqlens must start at 0 and not decrease
+    vcfg = dash.make_config(halt_layer=1)
+    bad_cu = (ctypes.c_int32 * 3)(0, 10, 5)
+    assert L.dash_prefill_varlen(ctypes.byref(dims), layers, FAKE, bad_cu, 2, ctypes.byref(vcfg), None, None, None,
+                                 None, None, 0, None) == 1
+    bad_cu0 = (ctypes.c_int32 * 3)(1, 10, 20)
+    assert L.dash_prefill_varlen(ctypes.byref(dims), layers, FAKE, bad_cu0, 2, ctypes.byref(vcfg), None, None, None,
+                                 None, None, 0, None) == 1
+    ok_cu = (ctypes.c_int32 * 3)(0, 10, 20)
+    assert L.dash_prefill_varlen(ctypes.byref(dims), layers, FAKE, ok_cu, 2, ctypes.byref(vcfg), None, None, None,
+                                 None, None, 0, None) == 4   # valid layout, no workspace
 
 
 def test_workspace_sizes_grow_with_tokens(L):

@@ -1,4 +1,5 @@
 """GPU parity of the building-block kernels against the CPU oracle, through the C ABI."""
+import ctypes
 import math
 
 import numpy as np
@@ -174,3 +175,35 @@ def test_exp2_fma_within_its_error_bound(gpu_lib):
     low = dash.exp2_fma(torch.tensor([-125.5, -127.0, -200.0, -float("inf")], device=DEV)).cpu().numpy()
     assert np.all(np.isfinite(low) & (low > 0) & (low < 1e-37))  # clamped far below any bf16 weight
     _no_device_error()
+
+
+@pytest.mark.parametrize("hd,hq,hkv,cu", [(64, 4, 2, [0, 300, 301, 700, 1030]), (128, 8, 2, [0, 256, 512, 900]),
+                                          (128, 4, 1, [0, 1, 129, 130, 400])])
+def test_attention_block_diagonal_matches_per_sequence_oracle(gpu_lib, hd, hq, hkv, cu):
+    T = cu[-1]
+    g = torch.Generator().manual_seed(T + hd)
+    Q = torch.randn(T, hq * hd, generator=g).to(torch.bfloat16)
+    K = torch.randn(T, hkv * hd, generator=g).to(torch.bfloat16)
+    V = torch.randn(T, hkv * hd, generator=g).to(torch.bfloat16)
+    kstart = torch.tensor(np.repeat(cu[:-1], np.diff(cu)), dtype=torch.int32)
+    got = to_np(dash.attention(Q.to(DEV), K.to(DEV), V.to(DEV), hq, hkv, hd, kstart=kstart.to(DEV)).cpu())
+    ref = np.concatenate([
+        O.causal_gqa_attention(to_np(Q[a:b]).reshape(b - a, hq, hd), to_np(K[a:b]).reshape(b - a, hkv, hd),
+                               to_np(V[a:b]).reshape(b - a, hkv, hd), np.arange(b - a), np.arange(b - a)
+                               ).reshape(b - a, -1)
+        for a, b in zip(cu[:-1], cu[1:])])
+    assert row_rel_err(got.reshape(T * hq, hd), ref.reshape(T * hq, hd)) < 2e-2
+    _no_device_error()
+
+
+def test_bounded_wait_gives_up_with_timeout_status(gpu_lib):
+    """A kernel waits on an mbarrier that nothing arrives on: the bounded wait
+    gives up (about 2 s), the TIMEOUT status reaches the host, and the
+    context stays usable."""
+    done = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert dash.lib().dash_selftest_wait_timeout(ctypes.c_void_p(done.data_ptr())) == 6
+    assert int(done.item()) == 2
+    assert dash.device_error() == 0                      # read and cleared
+    x = torch.randn(64, 256, device=DEV).to(torch.bfloat16)
+    y = dash.rmsnorm(x, torch.ones(256, dtype=torch.bfloat16, device=DEV), 1e-6)  # still works
+    assert torch.isfinite(y.float()).all()

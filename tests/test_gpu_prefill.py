@@ -260,3 +260,101 @@ def test_qwen_prefill_32k_properties(gpu_lib, mode):
     assert torch.isfinite(out.float()).all()
     del stack
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------- varlen batches
+CU_TINY = [0, 200, 201, 512, 641]   # ragged lengths, one of a single token
+
+
+def _prefill_varlen(stack, h0, cu, **kw):
+    H = h0.to(DEV).clone()
+    T = H.shape[0]
+    idx = torch.full((T,), -1, dtype=torch.int32, device=DEV)
+    delta = torch.empty(T, dtype=torch.float32, device=DEV)
+    K, counts = dash.prefill_varlen(stack, H, cu, dash.make_config(**kw), idx_out=idx, delta_out=delta)
+    assert dash.device_error() == 0
+    return H.cpu(), idx[:K].cpu().numpy(), delta.cpu().numpy(), K, counts
+
+
+@pytest.fixture(scope="module")
+def tiny_varlen(tiny):
+    dims, _, stack, L = tiny
+    h0, _ = inputs.make_hidden(CU_TINY[-1], dims.d_model, seed=9)
+    return dims, h0, stack, L
+
+
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+@pytest.mark.parametrize("keep,nf,nl", [(0.5, 0, 0), (0.4, 16, 8)])
+def test_prefill_varlen_tiny_matches_oracle(tiny_varlen, mode, keep, nf, nl):
+    dims, h0, stack, L = tiny_varlen
+    Hg, idx, delta, K, counts = _prefill_varlen(stack, h0, CU_TINY, halt_layer=1, mode=mode, keep=keep,
+                                                keep_first=nf, keep_last=nl)
+    free = O.dash_prefill_varlen(to_np(h0), CU_TINY, L, dims.as_dict(), 1, mode, keep=keep, keep_first=nf,
+                                 keep_last=nl)
+    assert counts == free["counts"] and K == sum(counts)
+    assert _rel(delta, free["delta"]) < DELTA_TOL
+    for s in range(len(CU_TINY) - 1):
+        a, b = CU_TINY[s], CU_TINY[s + 1]
+        mine = idx[(idx >= a) & (idx < b)]
+        assert np.array_equal(mine - a, O.select_topk(delta[a:b].astype(np.float64), keep, nf, nl))
+        ref = free["idx"][(free["idx"] >= a) & (free["idx"] < b)]
+        _check_sets(mine, ref, free["delta"], _topk_cut(free["delta"][a:b], keep, nf, nl))
+    forced = O.dash_prefill_varlen(to_np(h0), CU_TINY, L, dims.as_dict(), 1, mode, forced_idx=idx)
+    got = to_np(Hg[:K]) if mode == "prune" else to_np(Hg)
+    assert row_rel_err(got, forced["hidden"]) < HIDDEN_TOL
+
+
+def test_prefill_varlen_tiny_dense_and_threshold(tiny_varlen):
+    dims, h0, stack, L = tiny_varlen
+    Hd, _, _, K, counts = _prefill_varlen(stack, h0, CU_TINY, mode="dense")
+    assert K == CU_TINY[-1] and counts == list(np.diff(CU_TINY))
+    ref = O.dash_prefill_varlen(to_np(h0), CU_TINY, L, dims.as_dict(), 0, "halt", keep=1.0)
+    dense = np.concatenate([O.dense_forward(to_np(h0)[a:b], L, dims.as_dict())
+                            for a, b in zip(CU_TINY[:-1], CU_TINY[1:])])
+    assert row_rel_err(to_np(Hd), dense) < HIDDEN_TOL
+    thr = float(np.float32(np.quantile(ref["delta"], 0.6)))
+    Hg, idx, delta, K, counts = _prefill_varlen(stack, h0, CU_TINY, halt_layer=0, mode="halt", select="threshold",
+                                                threshold=thr)
+    assert np.array_equal(idx, O.select_threshold(delta.astype(np.float64), np.float32(thr)))
+    forced = O.dash_prefill_varlen(to_np(h0), CU_TINY, L, dims.as_dict(), 0, "halt", forced_idx=idx)
+    assert row_rel_err(to_np(Hg), forced["hidden"]) < HIDDEN_TOL
+
+
+def test_varlen_single_sequence_is_bitwise_plain_prefill(tiny):
+    dims, h0, stack, L = tiny
+    Ha, ia, da, Ka = _prefill(stack, h0, halt_layer=2, mode="prune", keep=0.5)
+    Hb, ib, db, Kb, _ = _prefill_varlen(stack, h0, [0, 512], halt_layer=2, mode="prune", keep=0.5)
+    assert Ka == Kb and np.array_equal(ia, ib) and np.array_equal(da, db) and torch.equal(Ha[:Ka], Hb[:Kb])
+
+
+@pytest.mark.slow
+def test_llama_varlen_two_layers_matches_oracle(gpu_lib):
+    dims = inputs.LLAMA8B
+    layers = inputs.make_layers(dims, seed=5, n_layers=2)
+    stack = dash.Stack(dims, _dev_layers(layers))
+    cu = [0, 256, 512, 640, 1024]
+    h0, _ = inputs.make_varlen_hidden(n_seq=4, seq_len=256, text_len=64, d=dims.d_model, seed=5)
+    Hg, idx, delta, K, counts = _prefill_varlen(stack, h0, cu, halt_layer=0, mode="prune", keep=0.4)
+    L = layers_np(layers)
+    forced = O.dash_prefill_varlen(to_np(h0), cu, L, dims.as_dict(), 0, "prune", forced_idx=idx)
+    assert counts == [math.floor(0.4 * n) for n in np.diff(cu)]
+    assert _rel(delta, forced["delta"]) < DELTA_TOL
+    assert row_rel_err(to_np(Hg[:K]), forced["hidden"]) < HIDDEN_TOL
+
+
+@pytest.mark.slow
+def test_llama_varlen_4x16k_properties(gpu_lib):
+    """The varlen workload: Llama-3.1-8B-shaped, 4 x 16384 tokens, halt at 13, keep 0.4, prune."""
+    dims = inputs.LLAMA8B
+    stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=DEV))
+    h0, cu = inputs.make_varlen_hidden(device=DEV)
+    cu = cu.tolist()
+    Hg, idx, delta, K, counts = _prefill_varlen(stack, h0, cu, halt_layer=13, mode="prune", keep=0.4)
+    assert counts == [6553] * 4 and K == 4 * 6553
+    for s in range(4):
+        a, b = cu[s], cu[s + 1]
+        mine = idx[(idx >= a) & (idx < b)]
+        assert np.array_equal(mine - a, O.select_topk(delta[a:b].astype(np.float64), 0.4))
+    assert torch.isfinite(Hg[:K].float()).all()
+    del stack
+    torch.cuda.empty_cache()

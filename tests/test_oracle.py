@@ -353,3 +353,19 @@ def test_golden_counts_from_the_pages():
             T, keep, nf, nl = int(a[0]), a[1], int(a[2]), int(a[3])
             got = O.topk_count(T, keep, nf, nl)
         assert got == int(expect), (kind, args)
+
+
+def test_varlen_oracle_is_per_sequence_and_order_independent(tiny_np):
+    dims_d, L, h0, _ = tiny_np
+    cu = [0, 70, 71, 200]
+    r = O.dash_prefill_varlen(h0[:200], cu, L, dims_d, 1, "prune", keep=0.5)
+    assert r["counts"] == [35, 0, 64]            # floor(0.5 * len) per sequence
+    # each sequence is the single-sequence prefill of its own rows
+    one = O.dash_prefill(h0[71:200], L, dims_d, 1, "prune", keep=0.5)
+    np.testing.assert_array_equal(r["idx"][35:], one["idx"] + 71)
+    np.testing.assert_allclose(r["hidden"][35:], one["hidden"], rtol=0, atol=0)
+    # swapping the sequences swaps the results: nothing crosses a boundary
+    sw = np.concatenate([h0[71:200], h0[0:71]])
+    r2 = O.dash_prefill_varlen(sw, [0, 129, 199, 200], L, dims_d, 1, "prune", keep=0.5)
+    np.testing.assert_allclose(r2["hidden"][:64], r["hidden"][35:], rtol=0, atol=0)
+    np.testing.assert_allclose(r2["hidden"][64:], r["hidden"][:35], rtol=0, atol=0)
