@@ -39,6 +39,10 @@ WORKLOADS = {
                         span_rows=6528, span_len=128, mode="halt", calibrate=True,
                         name="Qwen2.5-7B-shaped stack, T=131072, halt at layer 11, relative-delta threshold "
                              "calibrated to keep 30%, halt mode"),
+    "llama8b-varlen": dict(dims=inputs.LLAMA8B, T=65536, nseq=4, halt_layer=13, keep=0.4, select="topk",
+                           relative=False, span_rows=0, span_len=64, mode="prune", varlen=True,
+                           name="Llama-3.1-8B-shaped stack (32 layers, d=4096, 32q/8kv, hd=128, FFN 14336), varlen "
+                                "batch 4 x 16384 (2048 text + 14336 clustered rows each), halt at layer 13, keep 0.4"),
     "tiny": dict(dims=inputs.TINY, T=512, halt_layer=2, keep=0.5, select="topk", relative=False, span_rows=0,
                  span_len=64, mode="prune", name="tiny decoder stack (4 layers, d=256, 4q/2kv, hd=64, FFN 704), T=512"),
 }
@@ -259,8 +263,14 @@ def main():
     peaks = load_peaks()
 
     stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev))
-    h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=dev, span_rows=wl["span_rows"],
-                               span_len=wl["span_len"])
+    varlen = wl.get("varlen", False)
+    cu = None
+    if varlen:
+        h0, cu_t = inputs.make_varlen_hidden(n_seq=wl["nseq"], seq_len=T // wl["nseq"], d=dims.d_model, device=dev)
+        cu = cu_t.tolist()
+    else:
+        h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=dev, span_rows=wl["span_rows"],
+                                   span_len=wl["span_len"])
     H = torch.empty_like(h0)
     idx = torch.empty(T, dtype=torch.int32, device=dev)
     delta = torch.empty(T, dtype=torch.float32, device=dev)
@@ -269,16 +279,21 @@ def main():
         cal = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select="topk", keep=wl["keep"],
                                relative=wl["relative"])
         H.copy_(h0)
-        dash.prefill(stack, H, cal, idx_out=idx, delta_out=delta)
+        run(cal)
         kcal = math.floor(wl["keep"] * T)
         threshold = float(torch.sort(delta.cpu(), descending=True).values[kcal - 1])
     cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select=wl["select"], keep=wl["keep"],
                            threshold=threshold, relative=wl["relative"])
     cfg_dense = dash.make_config(mode="dense")
 
+    def run(c):
+        if varlen:
+            return dash.prefill_varlen(stack, H, cu, c, idx_out=idx, delta_out=delta)[0]
+        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
+
     def step(c):
         H.copy_(h0)
-        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
+        return run(c)
 
     def timed(c, k, record=False):
         torch.cuda.synchronize()
@@ -305,14 +320,23 @@ def main():
     clocks = clock.stop()
     dash.check_device()
     active = idx[:K].cpu().numpy()
-    halted_flops = costs.prefill_flops(dims, T, wl["halt_layer"], K, args.mode, active)
+    if varlen:
+        counts = [int(((active >= a) & (active < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
+        halted_flops = costs.varlen_prefill_flops(dims, cu, wl["halt_layer"], counts, args.mode, active)
+        seq_of = lambda i: max(s for s in range(len(cu) - 1) if cu[s] <= i)
+        pairs_by_rows = {T: sum(costs.causal_pairs(b - a) for a, b in zip(cu[:-1], cu[1:]))}
+        pairs_by_rows[K] = (sum(costs.causal_pairs(k) for k in counts) if args.mode == "prune"
+                            else int(sum(int(i) - cu[seq_of(int(i))] + 1 for i in active)))
+    else:
+        halted_flops = costs.prefill_flops(dims, T, wl["halt_layer"], K, args.mode, active)
+        pairs_by_rows = {T: costs.causal_pairs(T), K: int(sum(int(i) + 1 for i in active))
+                         if args.mode == "halt" else costs.causal_pairs(K)}
     value = world * T / (ms / 1e3)
 
     # per-kernel breakdown of the timed steps (CUDA events around every launch)
-    halt_pairs = int(sum(int(i) + 1 for i in active))
     per = {}
     for r in recs:
-        unit, amount = costs.launch_work(r, dims, halt_pairs)
+        unit, amount = costs.launch_work(r, dims, pairs_by_rows)
         p = per.setdefault(r["kind"], {"launches": 0, "ms": 0.0, "unit": unit, "work": 0})
         p["launches"] += 1
         p["ms"] += r["ms"]
@@ -343,20 +367,24 @@ def main():
     if not args.no_extra:
         step(cfg_dense)
         ms_d, _, _ = timed(cfg_dense, max(2, args.steps // 2))
-        dense_flops = costs.prefill_flops(dims, T)
+        dense_flops = costs.varlen_prefill_flops(dims, cu) if varlen else costs.prefill_flops(dims, T)
         other = "halt" if args.mode == "prune" else "prune"
         cfg_o = dash.make_config(halt_layer=wl["halt_layer"], mode=other, select=wl["select"], keep=wl["keep"],
                                  threshold=threshold, relative=wl["relative"])
         step(cfg_o)
         ms_o, K_o, _ = timed(cfg_o, max(2, args.steps // 2))
         act_o = idx[:K_o].cpu().numpy()
+        if varlen:
+            cnt_o = [int(((act_o >= a) & (act_o < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
+            flops_o = costs.varlen_prefill_flops(dims, cu, wl["halt_layer"], cnt_o, other, act_o)
+        else:
+            flops_o = costs.prefill_flops(dims, T, wl["halt_layer"], K_o, other, act_o)
         extra = {
             "dense": {"tokens_per_s": world * T / (ms_d / 1e3), "ms_per_step": ms_d,
                       "tflops": dense_flops / (ms_d / 1e3) / 1e12},
             other + "_mode": {"tokens_per_s": world * T / (ms_o / 1e3), "ms_per_step": ms_o, "K": K_o,
                               "speedup_vs_dense": ms_d / ms_o,
-                              "flop_bound": dense_flops / costs.prefill_flops(dims, T, wl["halt_layer"], K_o,
-                                                                              other, act_o)},
+                              "flop_bound": dense_flops / flops_o},
             "speedup_vs_dense": ms_d / ms,
             "flop_bound": dense_flops / halted_flops,
         }
@@ -366,7 +394,7 @@ def main():
         out_host = torch.empty(T, dims.d_model, dtype=torch.bfloat16).pin_memory()
         def e2e_step():
             H.copy_(h_host, non_blocking=True)
-            k = dash.prefill(stack, H, cfg, idx_out=idx, delta_out=delta)
+            k = run(cfg)
             rows = k if args.mode == "prune" else T
             out_host[:rows].copy_(H[:rows], non_blocking=True)
             return rows
@@ -389,8 +417,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, N(0,1) inputs)",
-        "config": {"workload": wl["name"], "model": "qwen2.5-7b-shaped random init" if dims is inputs.QWEN7B
-                   else "tiny", "global_batch": world, "seq_len": T, "halt_layer": wl["halt_layer"],
+        "config": {"workload": wl["name"], "model": {id(inputs.QWEN7B): "qwen2.5-7b-shaped random init",
+                                                       id(inputs.LLAMA8B): "llama-3.1-8b-shaped random init"}
+                   .get(id(dims), "tiny"), "global_batch": world * wl.get("nseq", 1), "seq_len": T, "halt_layer": wl["halt_layer"],
                    "keep": wl["keep"], "mode": args.mode, "select": wl["select"],
                    **({"threshold": threshold} if wl["select"] == "threshold" else {}),
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (13 GB of weights per step)"},

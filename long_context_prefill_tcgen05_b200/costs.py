@@ -44,14 +44,29 @@ def prefill_flops(dims, T, halt_layer=None, K=None, mode="dense", active_idx=Non
     return n_full * full + n_late * late
 
 
-def launch_work(rec, dims, halt_pairs=None):
-    """(unit, amount) of algorithmic work for one timed launch record."""
+def varlen_prefill_flops(dims, cu, halt_layer=None, counts=None, mode="dense", active_idx=None):
+    """prefill_flops summed over the independent sequences [cu[s], cu[s+1])."""
+    total = 0
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        act = None
+        if active_idx is not None:
+            act = [int(i) - a for i in active_idx if a <= int(i) < b]
+        total += prefill_flops(dims, b - a, halt_layer, None if counts is None else counts[s], mode, act)
+    return total
+
+
+def launch_work(rec, dims, pairs_by_rows=None):
+    """(unit, amount) of algorithmic work for one timed launch record.  Attention
+    launches whose visible pairs the library cannot count on the host (query
+    positions or per-sequence key starts) record k = -1; pairs_by_rows maps their
+    query-row count to the pairs of this run."""
     kind, m, n, k = rec["kind"], rec["m"], rec["n"], rec["k"]
     if kind.startswith("gemm"):
         return "flop", 2 * m * n * k
     if kind == "attention":
-        pairs = k if k >= 0 else halt_pairs
-        return "flop", attn_flops(dims, pairs or 0)
+        pairs = k if k >= 0 else (pairs_by_rows or {}).get(m, 0)
+        return "flop", attn_flops(dims, pairs)
     if kind == "rmsnorm":
         return "byte", 2 * m * n * 2
     if kind in ("gather", "scatter"):

@@ -217,7 +217,7 @@ dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16
   p.n_qblocks = static_cast<int>((M + 2 * dash::attn::BQ - 1) / (2 * dash::attn::BQ));
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
   const int64_t grid = static_cast<int64_t>(p.n_qblocks) * hq;
-  TimedLaunch tl(DASH_K_ATTENTION, M, T_kv, qpos ? -1 : M * (M + 1) / 2, st);
+  TimedLaunch tl(DASH_K_ATTENTION, M, T_kv, (qpos || kstart) ? -1 : M * (M + 1) / 2, st);
   attn_kernel<HD><<<static_cast<unsigned>(grid), dash::attn::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
   return launch_status();
 }
