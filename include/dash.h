@@ -106,6 +106,14 @@ typedef struct dash_config {
   float threshold;    /* threshold mode: keep t iff Δ_t >= threshold */
   int32_t keep_first; /* first tokens always kept (0 = none) */
   int32_t keep_last;  /* last tokens always kept (0 = none) */
+  /* Consecutive-layer monitoring ([DASH news] "层间更新动态监测": a token is
+   * stable when its update stays below the threshold over several
+   * consecutive layers).  Δ is taken at the monitor_layers layers ending at
+   * halt_layer and combined by maximum, so with threshold selection a token
+   * halts iff its Δ is below the threshold in every monitored layer; top-k
+   * ranks by the same maximum.  0 or 1 = the halting layer only; at most
+   * halt_layer + 1. */
+  int32_t monitor_layers;
 } dash_config;
 
 /* Human-readable name of a status code (static string). */

@@ -329,7 +329,7 @@ void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, C
 dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_layer_weights& w, bf16* H, int64_t M,
                        const int32_t* pos, const dash_halt_ctx* halt, float* delta, int relative,
                        const LayerWs& ws, cudaStream_t st, const int32_t* kstart = nullptr,
-                       const int32_t* halted_pos = nullptr) {
+                       const int32_t* halted_pos = nullptr, int delta_accumulate = 0) {
   if (M == 0) return DASH_OK;
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd, kvd = hkv * hd;
@@ -394,7 +394,8 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
     const int64_t blocks = (M + 255) / 256;
     TimedLaunch tl(DASH_K_SCORE, M, d / bn, 0, st);
     dash::rows::score_from_ssq_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(ws.ssq_u, ws.ssq_h, d / bn,
-                                                                                     M, relative, delta);
+                                                                                     M, relative, delta_accumulate,
+                                                                                     delta);
     if ((s = launch_status()) != DASH_OK) return s;
   }
   // a5: post-attention RMSNorm, gate/up GEMM with SwiGLU
@@ -527,6 +528,7 @@ dash_status check_config(const dash_dims* dims, const dash_config* cfg) {
     if (cfg->select == DASH_SELECT_TOPK && !(cfg->keep_ratio >= 0.0 && cfg->keep_ratio <= 1.0))
       return DASH_ERR_INVALID_ARG;
     if (cfg->keep_first < 0 || cfg->keep_last < 0) return DASH_ERR_INVALID_ARG;
+    if (cfg->monitor_layers < 0 || cfg->monitor_layers > cfg->halt_layer + 1) return DASH_ERR_INVALID_ARG;
   }
   return DASH_OK;
 }
@@ -579,12 +581,15 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
     kst_full = P.kst;
   }
 
+  // Δ is taken at the layers [delta_first, delta_last] and combined by maximum.
   auto run_layers = [&](int l0, int l1, bf16* rows, int64_t M, const int32_t* pos, const dash_halt_ctx* hc,
-                        const int32_t* kst, const int32_t* hpos, int delta_layer, float* delta) -> dash_status {
+                        const int32_t* kst, const int32_t* hpos, int delta_first, int delta_last,
+                        float* delta) -> dash_status {
     for (int l = l0; l < l1; ++l) {
       g_timing.layer = l;
-      const dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, l == delta_layer ? delta : nullptr,
-                                       cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos);
+      const bool take = l >= delta_first && l <= delta_last;
+      const dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, take ? delta : nullptr,
+                                       cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos, l > delta_first ? 1 : 0);
       g_timing.layer = -1;
       if (r != DASH_OK) return r;
     }
@@ -592,7 +597,8 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   };
 
   if (cfg->mode == DASH_MODE_DENSE) {
-    if ((s = run_layers(0, D.n_layers, h, T, pos_full, nullptr, kst_full, nullptr, -1, nullptr)) != DASH_OK) return s;
+    if ((s = run_layers(0, D.n_layers, h, T, pos_full, nullptr, kst_full, nullptr, -1, -1, nullptr)) != DASH_OK)
+      return s;
     if (K_out) *K_out = T;
     if (seq_counts)
       for (int q = 0; q < nseq; ++q) seq_counts[q] = cu[q + 1] - cu[q];
@@ -602,7 +608,9 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   // Layers 0..L_s on all T tokens; Δ from the halting layer's o_proj epilogue.
   const int Ls = cfg->halt_layer;
   float* delta = delta_out ? delta_out : P.delta;
-  if ((s = run_layers(0, Ls + 1, h, T, pos_full, nullptr, kst_full, nullptr, Ls, delta)) != DASH_OK) return s;
+  const int window = cfg->monitor_layers > 1 ? cfg->monitor_layers : 1;
+  if ((s = run_layers(0, Ls + 1, h, T, pos_full, nullptr, kst_full, nullptr, Ls - window + 1, Ls, delta)) != DASH_OK)
+    return s;
 
   // One-shot selection of the active set S*, per sequence.
   int32_t* idx = idx_out ? idx_out : P.idx;
@@ -652,7 +660,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
       pos_c = P.pos;
       kst_c = P.kst;
     }
-    if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_c, nullptr, kst_c, nullptr, -1, nullptr)) != DASH_OK)
+    if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_c, nullptr, kst_c, nullptr, -1, -1, nullptr)) != DASH_OK)
       return s;
     if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16),
                                  cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -674,7 +682,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
     kst_a = P.kst;
     hpos = P.hpos;
   }
-  if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_a, &hc, kst_a, hpos, -1, nullptr)) != DASH_OK) return s;
+  if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_a, &hc, kst_a, hpos, -1, -1, nullptr)) != DASH_OK) return s;
   return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
 }
 

@@ -114,9 +114,12 @@ __global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfl
 }
 
 // Δ from the o_proj epilogue's per-tile partial sums [ntiles, M], reduced in
-// a fixed order so the result is deterministic.
+// a fixed order so the result is deterministic.  With accumulate set, delta
+// keeps the maximum of its current value and the new Δ (consecutive-layer
+// monitoring).
 __global__ void score_from_ssq_kernel(const float* __restrict__ ssq_u, const float* __restrict__ ssq_h,
-                                      int ntiles, int64_t M, int relative, float* __restrict__ delta) {
+                                      int ntiles, int64_t M, int relative, int accumulate,
+                                      float* __restrict__ delta) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= M) return;
   float su = 0.f, sh = 0.f;
@@ -125,7 +128,7 @@ __global__ void score_from_ssq_kernel(const float* __restrict__ ssq_u, const flo
     for (int j = 0; j < ntiles; ++j) sh += ssq_h[j * M + t];
   const float dl = relative ? sqrtf(su) / sqrtf(sh) : sqrtf(su);
   if (!isfinite(dl)) flag_error(kDevErrNonfinite);
-  delta[t] = dl;
+  delta[t] = accumulate ? fmaxf(delta[t], dl) : dl;
 }
 
 // ------------------------------------------------------------------- select

@@ -40,7 +40,8 @@ class LayerWeights(ctypes.Structure):
 
 class Config(ctypes.Structure):
     _fields_ = [("halt_layer", c_i32), ("mode", c_i32), ("select", c_i32), ("score", c_i32),
-                ("keep_ratio", c_f64), ("threshold", c_f32), ("keep_first", c_i32), ("keep_last", c_i32)]
+                ("keep_ratio", c_f64), ("threshold", c_f32), ("keep_first", c_i32), ("keep_last", c_i32),
+                ("monitor_layers", c_i32)]
 
 
 class LaunchRecord(ctypes.Structure):
@@ -279,8 +280,9 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
 
 
 def make_config(halt_layer=0, mode="prune", select="topk", keep=0.5, threshold=0.0, relative=False,
-                keep_first=0, keep_last=0):
-    return Config(halt_layer, MODES[mode], SELECTS[select], int(relative), keep, threshold, keep_first, keep_last)
+                keep_first=0, keep_last=0, monitor_layers=1):
+    return Config(halt_layer, MODES[mode], SELECTS[select], int(relative), keep, threshold, keep_first, keep_last,
+                  monitor_layers)
 
 
 def prefill_varlen(stack, H, cu_seqlens, cfg, idx_out=None, delta_out=None, stream=None):

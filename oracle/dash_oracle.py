@@ -256,7 +256,7 @@ def scatter_rows(x_full, y, idx):
 
 def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
                  keep=0.5, threshold=None, relative=False, keep_first=0,
-                 keep_last=0, forced_idx=None):
+                 keep_last=0, forced_idx=None, monitor_layers=1):
     """Single-shot DASH prefill ([DASH blog] §2.3, §3.1; [DASH news]).
 
     Layers 0..halt_layer run on all T tokens (R6, R7).  After the halting
@@ -270,6 +270,12 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
       the active queries, which attend causally by original position.
       Returns hidden [T, d].
 
+    monitor_layers = W > 1 takes Δ at the W consecutive layers ending at the
+    halting layer and keeps their elementwise maximum ([DASH news]
+    "层间更新动态监测": a token is stable when its update stays below the
+    threshold over several consecutive layers; with threshold selection it
+    halts iff Δ_l < threshold in every monitored layer).
+
     forced_idx, when given, replaces the selection (teacher forcing in tests).
     Returns a dict with hidden, idx, delta, halt_out (halting layer output)
     and halt_in (its input).
@@ -277,11 +283,16 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
     h = np.asarray(h0, dtype=np.float64)
     T = len(h)
     pos = np.arange(T)
-    for l in range(halt_layer):
-        h, _ = decoder_block(h, pos, h, pos, layers[l], dims)
-    h_in = h
-    h, u = decoder_block(h, pos, h, pos, layers[halt_layer], dims)
-    delta = delta_scores(u, h_in, relative)
+    window = max(1, monitor_layers)
+    if window > halt_layer + 1:
+        raise OracleError("monitor window longer than the layers before halting")
+    delta = None
+    for l in range(halt_layer + 1):
+        h_in = h
+        h, u = decoder_block(h, pos, h, pos, layers[l], dims)
+        if l > halt_layer - window:
+            d_l = delta_scores(u, h_in, relative)
+            delta = d_l if delta is None else np.maximum(delta, d_l)
     if forced_idx is not None:
         idx = np.asarray(forced_idx, dtype=np.int64)
     elif select == "topk":

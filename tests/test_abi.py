@@ -71,6 +71,8 @@ def test_argument_errors_are_caught_on_the_host(L):
     assert call(dims, layers, FAKE, 512, bad) == 1                       # keep > 1
     bad = dash.make_config(halt_layer=1); bad.mode = 9
     assert call(dims, layers, FAKE, 512, bad) == 1                       # unknown mode
+    bad = dash.make_config(halt_layer=1, monitor_layers=3)
+    assert call(dims, layers, FAKE, 512, bad) == 1                       # window longer than layers 0..L_s
     holes = _fake_layers(4); holes[3] = dash.LayerWeights(*([FAKE] * 6 + [0]))
     assert call(dims, holes, FAKE, 512, cfg) == 1                        # a null weight
     assert call(dims, layers, FAKE, 512, cfg, None, 0) == 4              # no workspace

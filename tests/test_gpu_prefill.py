@@ -358,3 +358,24 @@ def test_llama_varlen_4x16k_properties(gpu_lib):
     assert torch.isfinite(Hg[:K].float()).all()
     del stack
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode,select,W", [("halt", "threshold", 2), ("prune", "topk", 3), ("prune", "threshold", 3)])
+def test_prefill_monitor_window_matches_oracle(tiny, mode, select, W):
+    dims, h0, stack, L = tiny
+    base = O.dash_prefill(to_np(h0), L, dims.as_dict(), 2, mode, keep=1.0, monitor_layers=W)
+    thr = float(np.float32(np.quantile(base["delta"], 0.5)))
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=2, mode=mode, select=select, keep=0.4, threshold=thr,
+                                 monitor_layers=W)
+    free = O.dash_prefill(to_np(h0), L, dims.as_dict(), 2, mode, select=select, keep=0.4, threshold=thr,
+                          monitor_layers=W)
+    assert _rel(delta, free["delta"]) < DELTA_TOL
+    if select == "topk":
+        assert np.array_equal(idx, O.select_topk(delta.astype(np.float64), 0.4))
+        _check_sets(idx, free["idx"], free["delta"], _topk_cut(free["delta"], 0.4))
+    else:
+        assert np.array_equal(idx, O.select_threshold(delta.astype(np.float64), np.float32(thr)))
+        _check_sets(idx, free["idx"], free["delta"], thr)
+    forced = O.dash_prefill(to_np(h0), L, dims.as_dict(), 2, mode, forced_idx=idx)
+    got = to_np(Hg[:K]) if mode == "prune" else to_np(Hg)
+    assert row_rel_err(got, forced["hidden"]) < HIDDEN_TOL

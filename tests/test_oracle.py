@@ -369,3 +369,26 @@ def test_varlen_oracle_is_per_sequence_and_order_independent(tiny_np):
     r2 = O.dash_prefill_varlen(sw, [0, 129, 199, 200], L, dims_d, 1, "prune", keep=0.5)
     np.testing.assert_allclose(r2["hidden"][:64], r["hidden"][35:], rtol=0, atol=0)
     np.testing.assert_allclose(r2["hidden"][64:], r["hidden"][:35], rtol=0, atol=0)
+
+
+def test_consecutive_layer_monitoring_brute_force(tiny_np):
+    # halted = tokens whose update is below the threshold in EVERY monitored
+    # layer, computed from per-layer deltas of directly run blocks
+    dims_d, L, h0, _ = tiny_np
+    h = h0[:150]
+    pos = np.arange(150)
+    per_layer, x = [], h
+    for l in range(3):
+        out, u = O.decoder_block(x, pos, x, pos, L[l], dims_d)
+        per_layer.append(np.linalg.norm(u, axis=1))
+        x = out
+    thr = float(np.median(per_layer[2]))
+    for W in (1, 2, 3):
+        r = O.dash_prefill(h, L, dims_d, 2, "halt", select="threshold", threshold=thr, monitor_layers=W)
+        stays = [t for t in range(150) if any(per_layer[l][t] >= thr for l in range(3 - W, 3))]
+        assert r["idx"].tolist() == stays
+    # top-k ranks by the window maximum
+    r = O.dash_prefill(h, L, dims_d, 2, "prune", keep=0.3, monitor_layers=2)
+    np.testing.assert_allclose(r["delta"], np.maximum(per_layer[1], per_layer[2]), rtol=1e-12)
+    with pytest.raises(O.OracleError):
+        O.dash_prefill(h, L, dims_d, 1, "prune", monitor_layers=3)
