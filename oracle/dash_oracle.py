@@ -53,6 +53,12 @@ Readings taken where the pages are silent or garbled:
       no selection is made.
   R15 the relative score divides by the norm of the halting layer's input
       residual stream H.
+  R17 generation after the prefill: the KV cache of a layer holds the keys
+      and values that layer's attention read during the prefill; a generated
+      token runs every layer and attends to that cache plus itself.
+  R18 a generated token's RoPE position continues the original numbering
+      (T for the first one after a T-token prompt), in prune mode too (R13).
+  (R16 is a reading of the pages that concerns no oracle function.)
 """
 import math
 
@@ -62,7 +68,8 @@ __all__ = [
     "rms_norm", "rope_inv_freq", "apply_rope", "causal_gqa_attention", "silu",
     "swiglu", "decoder_block", "dense_forward", "delta_scores", "forced_mask",
     "topk_count", "select_topk", "select_threshold", "gather_rows",
-    "scatter_rows", "dash_prefill", "dash_prefill_varlen", "OracleError",
+    "scatter_rows", "dash_prefill", "dash_prefill_varlen", "layer_kv",
+    "block_with_kv", "dash_decode", "OracleError",
 ]
 
 
@@ -140,6 +147,38 @@ def swiglu(gate, up):
     return silu(gate) * up
 
 
+def layer_kv(h_kv, kv_pos, w, dims):
+    """Keys (RoPE applied at kv_pos) and values of the rows h_kv [m, d] for one
+    layer: the entries a KV cache holds for them ([DASH blog] §2.1 block, R1-R4).
+    Returns k, v of shape [m, hkv, hd]."""
+    eps, theta = dims["rms_eps"], dims["rope_theta"]
+    hkv, hd = dims["n_kv_heads"], dims["head_dim"]
+    h_kv = np.asarray(h_kv, dtype=np.float64)
+    a_kv = rms_norm(h_kv, w["attn_norm"], eps)
+    k = apply_rope((a_kv @ w["wk"].T).reshape(len(h_kv), hkv, hd), kv_pos, theta)
+    v = (a_kv @ w["wv"].T).reshape(len(h_kv), hkv, hd)
+    return k, v
+
+
+def block_with_kv(h_q, q_pos, k, v, kv_pos, w, dims):
+    """The decoder block of the rows h_q (positions q_pos) attending to given
+    keys/values k, v [m, hkv, hd] at positions kv_pos.  Returns (out, U) as
+    decoder_block does."""
+    eps, theta = dims["rms_eps"], dims["rope_theta"]
+    hq, hd = dims["n_heads"], dims["head_dim"]
+    h_q = np.asarray(h_q, dtype=np.float64)
+    if len(h_q) == 0:  # no active rows: nothing to update
+        return h_q.copy(), np.zeros_like(h_q)
+    a_q = rms_norm(h_q, w["attn_norm"], eps)
+    q = apply_rope((a_q @ w["wq"].T).reshape(len(h_q), hq, hd), q_pos, theta)
+    o = causal_gqa_attention(q, k, v, q_pos, kv_pos).reshape(len(h_q), hq * hd)
+    u = o @ w["wo"].T
+    h1 = h_q + u
+    b = rms_norm(h1, w["ffn_norm"], eps)
+    f = swiglu(b @ w["wg"].T, b @ w["wu"].T) @ w["wd"].T
+    return h1 + f, u
+
+
 def decoder_block(h_q, q_pos, h_kv, kv_pos, w, dims):
     """One pre-norm decoder block ([DASH blog] §2.1; R1-R5).
 
@@ -150,24 +189,11 @@ def decoder_block(h_q, q_pos, h_kv, kv_pos, w, dims):
     Returns (out, U): out = H' + FFN(H'), H' = h_q + U, U = attention output
     after o_proj and before the residual add.
     """
-    eps = dims["rms_eps"]
-    theta = dims["rope_theta"]
-    hq, hkv, hd = dims["n_heads"], dims["n_kv_heads"], dims["head_dim"]
-    h_q = np.asarray(h_q, dtype=np.float64)
-    h_kv = np.asarray(h_kv, dtype=np.float64)
-    if len(h_q) == 0:  # no active rows: nothing to update
+    if len(h_q) == 0:
+        h_q = np.asarray(h_q, dtype=np.float64)
         return h_q.copy(), np.zeros_like(h_q)
-    a_q = rms_norm(h_q, w["attn_norm"], eps)
-    a_kv = rms_norm(h_kv, w["attn_norm"], eps)
-    q = apply_rope((a_q @ w["wq"].T).reshape(len(h_q), hq, hd), q_pos, theta)
-    k = apply_rope((a_kv @ w["wk"].T).reshape(len(h_kv), hkv, hd), kv_pos, theta)
-    v = (a_kv @ w["wv"].T).reshape(len(h_kv), hkv, hd)
-    o = causal_gqa_attention(q, k, v, q_pos, kv_pos).reshape(len(h_q), hq * hd)
-    u = o @ w["wo"].T
-    h1 = h_q + u
-    b = rms_norm(h1, w["ffn_norm"], eps)
-    f = swiglu(b @ w["wg"].T, b @ w["wu"].T) @ w["wd"].T
-    return h1 + f, u
+    k, v = layer_kv(h_kv, kv_pos, w, dims)
+    return block_with_kv(h_q, q_pos, k, v, kv_pos, w, dims)
 
 
 def dense_forward(h0, layers, dims, pos=None):
@@ -256,7 +282,7 @@ def scatter_rows(x_full, y, idx):
 
 def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
                  keep=0.5, threshold=None, relative=False, keep_first=0,
-                 keep_last=0, forced_idx=None, monitor_layers=1):
+                 keep_last=0, forced_idx=None, monitor_layers=1, return_kv=False):
     """Single-shot DASH prefill ([DASH blog] §2.3, §3.1; [DASH news]).
 
     Layers 0..halt_layer run on all T tokens (R6, R7).  After the halting
@@ -278,7 +304,10 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
 
     forced_idx, when given, replaces the selection (teacher forcing in tests).
     Returns a dict with hidden, idx, delta, halt_out (halting layer output)
-    and halt_in (its input).
+    and halt_in (its input).  With return_kv, "kv" holds per layer the tuple
+    (k, v, pos) of the keys/values that layer's attention read, in position
+    order: the KV cache the prefill leaves for generation (R17).  In prune
+    mode the layers after the halting layer hold the active rows only.
     """
     h = np.asarray(h0, dtype=np.float64)
     T = len(h)
@@ -287,9 +316,17 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
     if window > halt_layer + 1:
         raise OracleError("monitor window longer than the layers before halting")
     delta = None
+    kv = [] if return_kv else None
+
+    def block(h_q, q_pos, h_kv, kv_pos, w):
+        k, v = layer_kv(h_kv, kv_pos, w, dims)
+        if kv is not None:
+            kv.append((k, v, np.asarray(kv_pos, dtype=np.int64)))
+        return block_with_kv(h_q, q_pos, k, v, kv_pos, w, dims)
+
     for l in range(halt_layer + 1):
         h_in = h
-        h, u = decoder_block(h, pos, h, pos, layers[l], dims)
+        h, u = block(h, pos, h, pos, layers[l])
         if l > halt_layer - window:
             d_l = delta_scores(u, h_in, relative)
             delta = d_l if delta is None else np.maximum(delta, d_l)
@@ -305,18 +342,21 @@ def dash_prefill(h0, layers, dims, halt_layer, mode="prune", select="topk",
     if mode == "prune":
         hc = gather_rows(h, idx)
         for l in range(halt_layer + 1, len(layers)):
-            hc, _ = decoder_block(hc, idx, hc, idx, layers[l], dims)
+            hc, _ = block(hc, idx, hc, idx, layers[l])
         hidden = hc
     elif mode == "halt":
         hf = np.array(h, copy=True)
         for l in range(halt_layer + 1, len(layers)):
-            new_rows, _ = decoder_block(hf[idx], idx, hf, pos, layers[l], dims)
+            new_rows, _ = block(hf[idx], idx, hf, pos, layers[l])
             hf[idx] = new_rows
         hidden = hf
     else:
         raise OracleError(f"unknown mode {mode!r}")
-    return {"hidden": hidden, "idx": idx, "delta": delta,
-            "halt_out": halt_out, "halt_in": h_in}
+    out = {"hidden": hidden, "idx": idx, "delta": delta,
+           "halt_out": halt_out, "halt_in": h_in}
+    if kv is not None:
+        out["kv"] = kv
+    return out
 
 
 def dash_prefill_varlen(h0, cu_seqlens, layers, dims, halt_layer, mode="prune", forced_idx=None, **kw):
@@ -331,7 +371,7 @@ def dash_prefill_varlen(h0, cu_seqlens, layers, dims, halt_layer, mode="prune", 
     """
     cu = [int(x) for x in cu_seqlens]
     h0 = np.asarray(h0, dtype=np.float64)
-    hidden, idx, delta, counts = [], [], [], []
+    hidden, idx, delta, counts, kvs = [], [], [], [], []
     for s in range(len(cu) - 1):
         a, b = cu[s], cu[s + 1]
         f = None
@@ -340,13 +380,46 @@ def dash_prefill_varlen(h0, cu_seqlens, layers, dims, halt_layer, mode="prune", 
             f = g[(g >= a) & (g < b)] - a
         if b == a:
             counts.append(0)
+            kvs.append(None)
             continue
         r = dash_prefill(h0[a:b], layers, dims, halt_layer, mode, forced_idx=f, **kw)
+        kvs.append(r.get("kv"))
         hidden.append(r["hidden"])
         idx.append(r["idx"] + a)
         delta.append(r["delta"])
         counts.append(len(r["idx"]))
     d = h0.shape[1]
-    return {"hidden": np.concatenate(hidden) if hidden else np.zeros((0, d)),
-            "idx": np.concatenate(idx).astype(np.int64) if idx else np.zeros(0, np.int64),
-            "delta": np.concatenate(delta) if delta else np.zeros(0), "counts": counts}
+    out = {"hidden": np.concatenate(hidden) if hidden else np.zeros((0, d)),
+           "idx": np.concatenate(idx).astype(np.int64) if idx else np.zeros(0, np.int64),
+           "delta": np.concatenate(delta) if delta else np.zeros(0), "counts": counts}
+    if kw.get("return_kv"):
+        out["kv"] = kvs  # per sequence (positions within the sequence), None if empty
+    return out
+
+
+# ------------------------------------------------------------------- decode
+
+def dash_decode(x, pos, kv, layers, dims):
+    """Generation after a DASH prefill ([DASH blog] §3.1, generation stage, and
+    §5.1 on the KV cache): no pruning is applied to generated tokens, but in
+    every layer after the halting layer the cache holds only the active
+    tokens, so the new tokens attend to fewer keys.
+
+    x: [n, d] hidden states of n new tokens of one sequence at positions pos
+    (R18: the original numbering continues, e.g. T for the first generated
+    token).  kv: per layer (k, v, pos) as dash_prefill(return_kv=True)
+    returns it.  Every layer runs on the new rows; they attend to the cached
+    rows and causally to each other.  Returns (hidden [n, d], kv with the new
+    rows appended).
+    """
+    h = np.asarray(x, dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.int64)
+    new_kv = []
+    for w, (kc, vc, pc) in zip(layers, kv):
+        kn, vn = layer_kv(h, pos, w, dims)
+        k = np.concatenate([kc, kn])
+        v = np.concatenate([vc, vn])
+        p = np.concatenate([pc, pos])
+        h, _ = block_with_kv(h, pos, k, v, p, w, dims)
+        new_kv.append((k, v, p))
+    return h, new_kv

@@ -392,3 +392,87 @@ def test_consecutive_layer_monitoring_brute_force(tiny_np):
     np.testing.assert_allclose(r["delta"], np.maximum(per_layer[1], per_layer[2]), rtol=1e-12)
     with pytest.raises(O.OracleError):
         O.dash_prefill(h, L, dims_d, 1, "prune", monitor_layers=3)
+
+
+# ---------------------------------------------------------------- decode pins
+
+def test_prefill_cache_and_decode_match_transformers_kv_cache():
+    # transformers' own incremental decoding: its cache after the prompt and
+    # the hidden state of one generated token, against the oracle's dense
+    # prefill cache and dash_decode.
+    dims = inputs.TINY
+    layers_t = inputs.make_layers(dims, seed=3, n_layers=2)
+    gen = torch.Generator().manual_seed(8)
+    for w in layers_t:
+        w["attn_norm"] = (1 + 0.1 * torch.randn(dims.d_model, generator=gen)).to(torch.bfloat16)
+    L = layers_np(layers_t)
+    h = to_np(inputs.make_hidden(49, dims.d_model, seed=6)[0])
+    prompt, new = h[:48], h[48:]
+    r = O.dash_prefill(prompt, L, dims.as_dict(), halt_layer=1, mode="prune", keep=1.0, return_kv=True)
+    model = _hf_llama(dims, layers_t, 2)
+    with torch.no_grad():
+        out = model(inputs_embeds=torch.tensor(prompt)[None], position_ids=torch.arange(48)[None], use_cache=True)
+        cache = out.past_key_values
+        for l in range(2):
+            k, v, p = r["kv"][l]
+            assert np.array_equal(p, np.arange(48))
+            # rotated keys carry the fp32 angle error (about 6e-8 x angle, angles
+            # up to 47 rad here) times |k|: 1e-5 of max|k| bounds it; a wrong
+            # pairing, sign or position is off by order |k|.
+            ref_k = cache.layers[l].keys[0].numpy().transpose(1, 0, 2)
+            np.testing.assert_allclose(k, ref_k, rtol=0, atol=1e-5 * np.abs(ref_k).max())
+            np.testing.assert_allclose(v, cache.layers[l].values[0].numpy().transpose(1, 0, 2), **HF_TOL)
+        step = model(inputs_embeds=torch.tensor(new)[None], position_ids=torch.tensor([[48]]),
+                     past_key_values=cache, use_cache=True)
+    got, _ = O.dash_decode(new, [48], r["kv"], L, dims.as_dict())
+    np.testing.assert_allclose(got, step.last_hidden_state[0].numpy(), **HF_TOL)
+
+
+def test_decode_equals_dense_forward_of_the_longer_sequence(tiny_np):
+    # Two generated tokens on a dense cache, one at a time, are the last two
+    # rows of a dense forward over prompt + both tokens.
+    dims_d, L, h0, _ = tiny_np
+    h = h0[:66]
+    r = O.dash_prefill(h[:64], L, dims_d, halt_layer=len(L) - 1, mode="prune", keep=1.0, return_kv=True)
+    y1, kv = O.dash_decode(h[64:65], [64], r["kv"], L, dims_d)
+    y2, kv = O.dash_decode(h[65:66], [65], kv, L, dims_d)
+    ref = O.dense_forward(h, L, dims_d)
+    np.testing.assert_allclose(np.concatenate([y1, y2]), ref[64:], rtol=1e-11, atol=1e-11)
+    # several new tokens in one call attend causally among themselves
+    y12, _ = O.dash_decode(h[64:66], [64, 65], r["kv"], L, dims_d)
+    np.testing.assert_allclose(y12, ref[64:], rtol=1e-11, atol=1e-11)
+    assert all(len(k) == 66 for k, _, _ in kv)
+
+
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+def test_decode_on_pruned_cache_equals_prefill_with_the_new_token_active(tiny_np, mode):
+    # The generated token sees exactly what it would see as an extra active
+    # token of a prefill over prompt + token: the same rows in layers
+    # 0..L_s, and in later layers the active set (prune) or every row with
+    # the halted ones frozen (halt).
+    dims_d, L, h0, _ = tiny_np
+    T = 120
+    r = O.dash_prefill(h0[:T], L, dims_d, halt_layer=1, mode=mode, keep=0.4, return_kv=True)
+    idx = r["idx"]
+    K = len(idx)
+    rows = [len(k) for k, _, _ in r["kv"]]
+    late = K if mode == "prune" else T
+    assert rows == [T, T, late, late]
+    assert np.array_equal(r["kv"][2][2], idx if mode == "prune" else np.arange(T))
+    got, kv = O.dash_decode(h0[T:T + 1], [T], r["kv"], L, dims_d)
+    ext = O.dash_prefill(h0[:T + 1], L, dims_d, halt_layer=1, mode=mode,
+                         forced_idx=np.concatenate([idx, [T]]))
+    np.testing.assert_allclose(got, ext["hidden"][-1:], rtol=1e-11, atol=1e-11)
+    assert [len(k) for k, _, _ in kv] == [T + 1, T + 1, late + 1, late + 1]
+
+
+def test_varlen_prefill_returns_one_cache_per_sequence(tiny_np):
+    dims_d, L, h0, _ = tiny_np
+    cu = [0, 70, 70, 150]
+    r = O.dash_prefill_varlen(h0[:150], cu, L, dims_d, halt_layer=2, keep=0.5, return_kv=True)
+    assert r["kv"][1] is None
+    for s, (a, b) in enumerate([(0, 70), (70, 150)]):
+        kv = r["kv"][0 if s == 0 else 2]
+        one = O.dash_prefill(h0[a:b], L, dims_d, halt_layer=2, keep=0.5, return_kv=True)
+        for (k1, v1, p1), (k2, v2, p2) in zip(kv, one["kv"]):
+            assert np.array_equal(k1, k2) and np.array_equal(v1, v2) and np.array_equal(p1, p2)
