@@ -283,6 +283,65 @@ dash_status dash_prefill_varlen(const dash_dims* dims, const dash_layer_weights*
                                 int32_t* idx_out, int64_t* K_out, int32_t* seq_counts, float* delta_out,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------ KV cache and generation --
+ * [DASH blog] §3.1 (generation stage) and §5.1 (KV cache): generated tokens
+ * are not pruned, but the prefill caches keys/values only for the tokens
+ * each layer attended over -- in prune mode the active tokens alone in every
+ * layer after L_s -- so each generated token attends to fewer keys there.
+ *
+ * One dash_kv_cache describes one layer of one sequence.  The arrays are
+ * caller-owned device memory; `len` is a HOST field the library updates. */
+typedef struct dash_kv_cache {
+  dash_bf16* k;     /* [capacity, n_kv_heads*head_dim]: keys, RoPE applied, 16-byte aligned */
+  dash_bf16* v;     /* [capacity, n_kv_heads*head_dim]: values, 16-byte aligned */
+  int32_t* pos;     /* [capacity] original position of each cached row, or NULL */
+  int64_t capacity; /* rows allocated */
+  int64_t len;      /* rows filled (host field, set by the library) */
+} dash_kv_cache;
+
+#define DASH_DECODE_MAX_SEQ 8
+
+/* dash_prefill that also fills caches[0 .. n_layers): layer l's cache gets
+ * the keys/values that layer's attention read, in position order, and
+ * len = their count:
+ *   layers 0..L_s (and every layer in dense mode)  T rows, pos 0..T-1
+ *   later layers, prune                            K rows, pos = idx_out
+ *   later layers, halt                             T rows (halted rows' keys
+ *                                                  from their frozen state)
+ * Capacities are checked on the host before any launch (top-k selection),
+ * or, with threshold selection, for the later layers right after the
+ * selection (DASH_ERR_SHAPE, before those layers run). */
+dash_status dash_prefill_kv(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, int64_t T,
+                            const dash_config* cfg, int32_t* idx_out, int64_t* K_out, float* delta_out,
+                            dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream);
+
+/* dash_prefill_varlen that also fills caches[s * n_layers + l] (sequence-
+ * major) for every sequence s, positions counted from the sequence start. */
+dash_status dash_prefill_varlen_kv(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H,
+                                   const int32_t* cu_seqlens, int32_t nseq, const dash_config* cfg,
+                                   int32_t* idx_out, int64_t* K_out, int32_t* seq_counts, float* delta_out,
+                                   dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes for dash_decode_step with up to nseq sequences. */
+size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq);
+
+/* One generation step: one new token for each of nseq (<= DASH_DECODE_MAX_SEQ)
+ * sequences runs through every layer.
+ *   X      [nseq, d_model] bf16: the new tokens' input hidden states; on
+ *          return the hidden states after the last layer (no final norm).
+ *   pos    HOST [nseq]: RoPE position of each new token; it must exceed
+ *          every position already in that sequence's cache (the token
+ *          attends to all cached rows and itself).
+ *   caches HOST array [nseq * n_layers] (sequence-major): each layer appends
+ *          the token's key/value (and position) at row len, then len += 1;
+ *          every cache needs len < capacity and len + 1 <= 2^31 - 1.
+ * Layer l: RMSNorm -> QKV GEMV with RoPE and the cache append -> attention
+ * over the cache -> o_proj + residual -> RMSNorm -> gate/up GEMV with SwiGLU
+ * -> down + residual.  Requires (n_heads / n_kv_heads) <= 16. */
+dash_status dash_decode_step(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X,
+                             int32_t nseq, const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,19 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
                            int64_t T_kv, int32_t hq, int32_t hkv, int32_t hd, const int32_t* qpos,
                            const int32_t* kstart, dash_bf16* O, void* stream);
 
+/* Attention of one new query row per sequence over that sequence's cache
+ * (the generation-step attention of dash_decode_step; [DASH blog] §3.1,
+ * generation stage):  O[s, h, :] = softmax_j(Q[s, h, :] . k_j / sqrt(hd)) v_j
+ * over the rows j < caches[s].len of caches[s] (kv head h / (hq / hkv)).
+ *   Q, O: [nseq, hq*hd] bf16; caches: HOST array [nseq] (only k, v, len
+ *   are read; 1 <= len <= 2^31 - 1).  nseq <= DASH_DECODE_MAX_SEQ,
+ *   hq / hkv <= 16, nseq * hkv <= 64, hd 64 or 128.
+ *   ws: dash_decode_attention_workspace_size(hd) bytes. */
+size_t dash_decode_attention_workspace_size(int32_t hd);
+dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_kv_cache* caches, int32_t hq,
+                                  int32_t hkv, int32_t hd, dash_bf16* O, void* ws, size_t ws_bytes,
+                                  void* stream);
+
 /* The FMA-pipe exponential the attention softmax uses for half of its
  * elements (no page counterpart; exported so tests can hold it to its error
  * bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
@@ -61,14 +74,16 @@ typedef enum dash_kernel_kind {
   DASH_K_ROPE_TABLE = 0, DASH_K_RMSNORM = 1, DASH_K_GEMM_QKV = 2, DASH_K_GEMM_KV_HALTED = 3,
   DASH_K_ATTENTION = 4, DASH_K_GEMM_O = 5, DASH_K_SCORE = 6, DASH_K_GEMM_GATE_UP = 7,
   DASH_K_GEMM_DOWN = 8, DASH_K_SELECT = 9, DASH_K_GATHER = 10, DASH_K_SCATTER = 11,
-  DASH_K_GEMM = 12, DASH_K_COUNT = 13
+  DASH_K_GEMM = 12, DASH_K_KV_STORE = 13, DASH_K_DEC_GEMV_QKV = 14, DASH_K_DEC_ATTENTION = 15,
+  DASH_K_DEC_COMBINE = 16, DASH_K_DEC_GEMV_O = 17, DASH_K_DEC_GEMV_GATE_UP = 18, DASH_K_DEC_GEMV_DOWN = 19,
+  DASH_K_COUNT = 20
 } dash_kernel_kind;
 
 typedef struct dash_launch_record {
   int32_t kind;   /* dash_kernel_kind */
   int32_t layer;  /* decoder layer, -1 outside the layer loop */
-  int64_t m;      /* rows (GEMM M, attention query rows, selection T) */
-  int64_t n;      /* GEMM N, attention key rows */
+  int64_t m;      /* rows (GEMM M, attention query rows, selection T, decode sequences) */
+  int64_t n;      /* GEMM N, attention key rows (decode: cached keys summed over sequences) */
   int64_t k;      /* GEMM K, attention causal (query, key) pairs */
   float ms;       /* device time between the two events */
 } dash_launch_record;

@@ -11,6 +11,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemm.cuh"
 #include "rowops.cuh"
 
@@ -518,6 +519,45 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, int64_t n, float* _
 }
 
 
+// ---------------------------------------------------------------- KV cache
+dash_status kv_store(const bf16* Kb, const bf16* Vb, int kvd, int64_t a, int64_t rows, const int32_t* pos_src,
+                     const dash_kv_cache& c, const DeviceInfo& di, cudaStream_t st) {
+  if (rows == 0) return DASH_OK;
+  const int warps = 8;
+  int64_t blocks = (rows + warps - 1) / warps;
+  const int64_t cap = static_cast<int64_t>(di.num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  TimedLaunch tl(DASH_K_KV_STORE, rows, kvd, 0, st);
+  dash::decode::kv_store_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
+      Kb, Vb, kvd, a, rows, pos_src, reinterpret_cast<bf16*>(c.k), reinterpret_cast<bf16*>(c.v), c.pos);
+  return launch_status();
+}
+
+bool cache_ok(const dash_kv_cache& c) {
+  return c.k && c.v && aligned16(c.k) && aligned16(c.v) && c.capacity >= 0 && c.len >= 0 && c.len <= c.capacity &&
+         (!c.pos || (reinterpret_cast<uintptr_t>(c.pos) & 3u) == 0);
+}
+
+// Capacities a prefill needs: every layer holds its sequence's T_s rows,
+// except the layers after L_s in prune mode, which hold K_s rows (known here
+// for top-k selection; checked after the selection for threshold selection).
+dash_status check_prefill_caches(const dash_dims& D, const dash_config& cfg, const int32_t* cu, int nseq,
+                                 const dash_kv_cache* caches) {
+  for (int q = 0; q < nseq; ++q) {
+    const int64_t Tq = cu[q + 1] - cu[q];
+    for (int l = 0; l < D.n_layers; ++l) {
+      const dash_kv_cache& c = caches[static_cast<size_t>(q) * D.n_layers + l];
+      if (!cache_ok(c)) return DASH_ERR_INVALID_ARG;
+      int64_t need = Tq;
+      if (cfg.mode == DASH_MODE_PRUNE && l > cfg.halt_layer)
+        need = cfg.select == DASH_SELECT_TOPK ? dash_topk_count(Tq, cfg.keep_ratio, cfg.keep_first, cfg.keep_last)
+                                              : 0;
+      if (c.capacity < need) return DASH_ERR_SHAPE;
+    }
+  }
+  return DASH_OK;
+}
+
 dash_status check_config(const dash_dims* dims, const dash_config* cfg) {
   if (cfg->mode != DASH_MODE_PRUNE && cfg->mode != DASH_MODE_HALT && cfg->mode != DASH_MODE_DENSE)
     return DASH_ERR_INVALID_ARG;
@@ -540,7 +580,8 @@ dash_status check_config(const dash_dims* dims, const dash_config* cfg) {
 // sample).  nseq == 1 is the plain single-sequence prefill.
 dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, const int32_t* cu,
                          int nseq, const dash_config* cfg, int32_t* idx_out, int64_t* K_out, int32_t* seq_counts,
-                         float* delta_out, void* ws, size_t ws_bytes, void* stream) {
+                         float* delta_out, void* ws, size_t ws_bytes, void* stream,
+                         dash_kv_cache* caches = nullptr) {
   if (!dims_ok(dims)) return DASH_ERR_SHAPE;
   if (!layers || !H || !cfg || !aligned16(H)) return DASH_ERR_INVALID_ARG;
   const int64_t T = cu[nseq];
@@ -549,7 +590,10 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   if (s != DASH_OK) return s;
   for (int l = 0; l < dims->n_layers; ++l)
     if (!weights_ok(&layers[l])) return DASH_ERR_INVALID_ARG;
+  if (caches && (s = check_prefill_caches(*dims, *cfg, cu, nseq, caches)) != DASH_OK) return s;
   if (T == 0) {
+    if (caches)
+      for (int q = 0; q < nseq * dims->n_layers; ++q) caches[q].len = 0;
     if (K_out) *K_out = 0;
     if (seq_counts)
       for (int q = 0; q < nseq; ++q) seq_counts[q] = 0;
@@ -581,6 +625,15 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
     kst_full = P.kst;
   }
 
+  // KV cache rows of each sequence after a layer: kv_start/kv_rows index the
+  // layer's K/V buffers; kv_pos (NULL: row order) gives their positions.
+  std::vector<int64_t> kv_start(static_cast<size_t>(nseq)), kv_rows(static_cast<size_t>(nseq));
+  for (int q = 0; q < nseq; ++q) {
+    kv_start[q] = cu[q];
+    kv_rows[q] = cu[q + 1] - cu[q];
+  }
+  const int32_t* kv_pos = nullptr;
+
   // Δ is taken at the layers [delta_first, delta_last] and combined by maximum.
   auto run_layers = [&](int l0, int l1, bf16* rows, int64_t M, const int32_t* pos, const dash_halt_ctx* hc,
                         const int32_t* kst, const int32_t* hpos, int delta_first, int delta_last,
@@ -588,8 +641,13 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
     for (int l = l0; l < l1; ++l) {
       g_timing.layer = l;
       const bool take = l >= delta_first && l <= delta_last;
-      const dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, take ? delta : nullptr,
-                                       cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos, l > delta_first ? 1 : 0);
+      dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, take ? delta : nullptr,
+                                 cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos, l > delta_first ? 1 : 0);
+      for (int q = 0; r == DASH_OK && caches && q < nseq; ++q) {
+        dash_kv_cache& c = caches[static_cast<size_t>(q) * D.n_layers + l];
+        r = kv_store(P.L.Kb, P.L.Vb, D.n_kv_heads * D.head_dim, kv_start[q], kv_rows[q], kv_pos, c, *di, st);
+        c.len = kv_rows[q];
+      }
       g_timing.layer = -1;
       if (r != DASH_OK) return r;
     }
@@ -660,6 +718,17 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
       pos_c = P.pos;
       kst_c = P.kst;
     }
+    if (caches) {  // later layers cache the active rows only
+      int64_t a = 0;
+      for (int q = 0; q < nseq; ++q) {
+        kv_start[q] = a;
+        kv_rows[q] = counts[q];
+        a += counts[q];
+        for (int l = Ls + 1; l < D.n_layers; ++l)
+          if (caches[static_cast<size_t>(q) * D.n_layers + l].capacity < counts[q]) return DASH_ERR_SHAPE;
+      }
+      kv_pos = pos_c;
+    }
     if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_c, nullptr, kst_c, nullptr, -1, -1, nullptr)) != DASH_OK)
       return s;
     if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16),
@@ -686,6 +755,227 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   return move_rows(true, P.Hc, h, idx, K, T, D.d_model, *di, st);
 }
 
+
+// ------------------------------------------------------------ generation
+namespace dec = dash::decode;
+
+struct DecodeWs {
+  bf16* Xn;        // [n, d] x * g of the current norm
+  float* rs;       // [n] its 1/rms
+  bf16* Q;         // [n, hq*hd]
+  bf16* O;         // [n, hq*hd] attention output
+  bf16* Act;       // [n, F]
+  float* part_o;   // [kMaxCtas, 16, hd]
+  float* part_ml;  // [kMaxCtas, 16, 2]
+};
+
+void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
+  const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
+  w.Xn = c.take<bf16>(static_cast<size_t>(n) * D.d_model);
+  w.rs = c.take<float>(static_cast<size_t>(n));
+  w.Q = c.take<bf16>(n * qd);
+  w.O = c.take<bf16>(n * qd);
+  w.Act = c.take<bf16>(static_cast<size_t>(n) * D.ffn_dim);
+  w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * D.head_dim);
+  w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
+}
+
+template <int EPI, int NS>
+dash_status launch_gemv_ns(const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
+  if (gp.tasks == 0) return DASH_OK;
+  const unsigned blocks = static_cast<unsigned>((gp.tasks + dec::kGemvWarps - 1) / dec::kGemvWarps);
+  TimedLaunch tl(kind, gp.n, n_out, gp.K, st);
+  dec::gemv_kernel<EPI, NS><<<blocks, 32 * dec::kGemvWarps, 0, st>>>(gp);
+  return launch_status();
+}
+
+template <int EPI>
+dash_status launch_gemv(const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
+  if (gp.n <= 1) return launch_gemv_ns<EPI, 1>(gp, kind, n_out, st);
+  if (gp.n <= 2) return launch_gemv_ns<EPI, 2>(gp, kind, n_out, st);
+  if (gp.n <= 4) return launch_gemv_ns<EPI, 4>(gp, kind, n_out, st);
+  return launch_gemv_ns<EPI, 8>(gp, kind, n_out, st);
+}
+
+// Split-key decode attention of one layer: the CTA count is held to one
+// wave (at most one CTA per SM, at most kMaxCtas) by giving each CTA a run of
+// tiles_per_cta key tiles of one (sequence, kv head) segment.
+template <int HD>
+dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n, const int64_t* len,
+                                const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st) {
+  using C = dec::ACfg<HD>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(dec::decode_attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  const int hkv = D.n_kv_heads, kvd = hkv * HD;
+  dec::AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  dec::AttnParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  int64_t total_tiles = 0, max_tiles = 0, keys = 0;
+  for (int q = 0; q < n; ++q) {
+    const dash_kv_cache& c = *layer_caches[q];
+    if (!make_map(&maps.k[q], c.k, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV) ||
+        !make_map(&maps.v[q], c.v, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV))
+      return DASH_ERR_INVALID_ARG;
+    ap.len[q] = static_cast<int>(len[q]);
+    const int64_t t = (len[q] + dec::BKV - 1) / dec::BKV;
+    total_tiles += t * hkv;
+    max_tiles = t > max_tiles ? t : max_tiles;
+    keys += len[q];
+  }
+  const int64_t cap = di.num_sms < dec::kMaxCtas ? di.num_sms : dec::kMaxCtas;
+  int64_t per = (total_tiles + cap - 1) / cap;
+  if (per < 1) per = 1;
+  auto ctas_for = [&](int64_t tpc) {
+    int64_t c = 0;
+    for (int q = 0; q < n; ++q) c += hkv * (((len[q] + dec::BKV - 1) / dec::BKV + tpc - 1) / tpc);
+    return c;
+  };
+  while (ctas_for(per) > cap && per < max_tiles) ++per;
+  const int64_t nctas = ctas_for(per);
+  if (nctas > dec::kMaxCtas) return DASH_ERR_SHAPE;
+  int c0 = 0;
+  for (int q = 0; q < n; ++q) {
+    const int64_t chunks = ((len[q] + dec::BKV - 1) / dec::BKV + per - 1) / per;
+    for (int h = 0; h < hkv; ++h) {
+      ap.seg_cta0[q * hkv + h] = c0;
+      c0 += static_cast<int>(chunks);
+    }
+  }
+  ap.seg_cta0[n * hkv] = c0;
+  ap.q = w.Q;
+  ap.part_o = w.part_o;
+  ap.part_ml = w.part_ml;
+  ap.n = n;
+  ap.hq = D.n_heads;
+  ap.hkv = hkv;
+  ap.group = D.n_heads / hkv;
+  ap.tiles_per_cta = static_cast<int>(per);
+  ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
+  {
+    TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, 0, st);
+    dec::decode_attn_kernel<HD><<<static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st>>>(maps, ap);
+  }
+  dash_status s = launch_status();
+  if (s != DASH_OK) return s;
+  TimedLaunch tl(DASH_K_DEC_COMBINE, n, nctas, 0, st);
+  dec::decode_combine_kernel<HD><<<static_cast<unsigned>(n * D.n_heads), HD, 0, st>>>(ap, w.O);
+  return launch_status();
+}
+
+dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X, int n,
+                        const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream) {
+  if (!dims_ok(dims)) return DASH_ERR_SHAPE;
+  const dash_dims& D = *dims;
+  if (n < 1 || n > dec::kMaxSeq) return DASH_ERR_SHAPE;
+  if (D.n_heads / D.n_kv_heads > dec::kGroupPad || n * D.n_kv_heads > dec::kMaxSegs) return DASH_ERR_SHAPE;
+  if (!layers || !X || !aligned16(X) || !pos || !caches) return DASH_ERR_INVALID_ARG;
+  for (int l = 0; l < D.n_layers; ++l)
+    if (!weights_ok(&layers[l])) return DASH_ERR_INVALID_ARG;
+  for (int q = 0; q < n; ++q) {
+    if (pos[q] < 0) return DASH_ERR_INVALID_ARG;
+    for (int l = 0; l < D.n_layers; ++l) {
+      const dash_kv_cache& c = caches[static_cast<size_t>(q) * D.n_layers + l];
+      if (!cache_ok(c)) return DASH_ERR_INVALID_ARG;
+      if (c.len >= c.capacity || c.len + 1 > INT32_MAX) return DASH_ERR_SHAPE;
+    }
+  }
+  Carver probe{nullptr};
+  DecodeWs sizes;
+  carve_decode(D, n, probe, sizes);
+  if (!ws || ws_bytes < probe.off + 256) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  if (di->num_sms < dec::kMaxSegs) return DASH_ERR_SHAPE;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  DecodeWs w;
+  carve_decode(D, n, c, w);
+  cudaStream_t st = as_stream(stream);
+  bf16* x = reinterpret_cast<bf16*>(X);
+  const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
+  const int qd = hq * hd;
+
+  for (int l = 0; l < D.n_layers; ++l) {
+    g_timing.layer = l;
+    const dash_layer_weights& lw = layers[l];
+    const dash_kv_cache* lc[dec::kMaxSeq];
+    int64_t len[dec::kMaxSeq];
+    dec::GemvParams qkv;
+    std::memset(&qkv, 0, sizeof(qkv));
+    for (int q = 0; q < n; ++q) {
+      lc[q] = &caches[static_cast<size_t>(q) * D.n_layers + l];
+      qkv.seq.k[q] = reinterpret_cast<bf16*>(lc[q]->k);
+      qkv.seq.v[q] = reinterpret_cast<bf16*>(lc[q]->v);
+      qkv.seq.pos[q] = lc[q]->pos;
+      qkv.seq.row[q] = lc[q]->len;
+      qkv.seq.p[q] = pos[q];
+      len[q] = lc[q]->len + 1;
+    }
+    // RMSNorm -> QKV with RoPE, appended to the caches
+    if ((s = rmsnorm(x, n, nullptr, n, d, cb(lw.attn_norm), D.rms_eps, w.Xn, st, w.rs)) != DASH_OK) break;
+    qkv.W = cb(lw.w_qkv);
+    qkv.x = w.Xn;
+    qkv.xs = w.rs;
+    qkv.n = n;
+    qkv.K = d;
+    qkv.tasks = (hq + 2 * hkv) * hd / 2;
+    qkv.q = w.Q;
+    qkv.hq = hq;
+    qkv.hkv = hkv;
+    qkv.hd = hd;
+    qkv.theta = D.rope_theta;
+    if ((s = launch_gemv<dec::kGvQkv>(qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
+    // attention over each sequence's cache (including the new row)
+    s = hd == 128 ? decode_attention_hd<128>(*di, D, n, len, lc, w, st)
+                  : decode_attention_hd<64>(*di, D, n, len, lc, w, st);
+    if (s != DASH_OK) break;
+    // o_proj + residual
+    dec::GemvParams o;
+    std::memset(&o, 0, sizeof(o));
+    o.W = cb(lw.w_o);
+    o.x = w.O;
+    o.n = n;
+    o.K = qd;
+    o.tasks = d / 2;
+    o.out = x;
+    o.ldo = d;
+    if ((s = launch_gemv<dec::kGvResid>(o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
+    // RMSNorm -> gate/up with SwiGLU
+    if ((s = rmsnorm(x, n, nullptr, n, d, cb(lw.ffn_norm), D.rms_eps, w.Xn, st, w.rs)) != DASH_OK) break;
+    dec::GemvParams gu;
+    std::memset(&gu, 0, sizeof(gu));
+    gu.W = cb(lw.w_gate);
+    gu.W2 = cb(lw.w_up);
+    gu.x = w.Xn;
+    gu.xs = w.rs;
+    gu.n = n;
+    gu.K = d;
+    gu.tasks = F;
+    gu.out = w.Act;
+    gu.ldo = F;
+    if ((s = launch_gemv<dec::kGvSwiglu>(gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
+    // down + residual
+    dec::GemvParams dn;
+    std::memset(&dn, 0, sizeof(dn));
+    dn.W = cb(lw.w_down);
+    dn.x = w.Act;
+    dn.n = n;
+    dn.K = F;
+    dn.tasks = d / 2;
+    dn.out = x;
+    dn.ldo = d;
+    if ((s = launch_gemv<dec::kGvResid>(dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
+    for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
+  }
+  g_timing.layer = -1;
+  return s;
+}
 }  // namespace
 
 // =================================================================== C ABI
@@ -926,6 +1216,86 @@ dash_status dash_prefill_varlen(const dash_dims* dims, const dash_layer_weights*
                       stream);
 }
 
+dash_status dash_prefill_kv(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H, int64_t T,
+                            const dash_config* cfg, int32_t* idx_out, int64_t* K_out, float* delta_out,
+                            dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
+  if (!caches) return DASH_ERR_INVALID_ARG;
+  const int32_t cu[2] = {0, static_cast<int32_t>(T)};
+  return prefill_impl(dims, layers, H, cu, 1, cfg, idx_out, K_out, nullptr, delta_out, ws, ws_bytes, stream,
+                      caches);
+}
+
+dash_status dash_prefill_varlen_kv(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* H,
+                                   const int32_t* cu_seqlens, int32_t nseq, const dash_config* cfg,
+                                   int32_t* idx_out, int64_t* K_out, int32_t* seq_counts, float* delta_out,
+                                   dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream) {
+  if (!cu_seqlens || nseq < 1 || !caches) return DASH_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return DASH_ERR_INVALID_ARG;
+  for (int s = 0; s < nseq; ++s)
+    if (cu_seqlens[s + 1] < cu_seqlens[s]) return DASH_ERR_INVALID_ARG;
+  return prefill_impl(dims, layers, H, cu_seqlens, nseq, cfg, idx_out, K_out, seq_counts, delta_out, ws, ws_bytes,
+                      stream, caches);
+}
+
+size_t dash_decode_attention_workspace_size(int32_t hd) {
+  if (hd != 64 && hd != 128) return 0;
+  return static_cast<size_t>(dash::decode::kMaxCtas) * dash::decode::kGroupPad * (hd + 2) * sizeof(float) + 1024;
+}
+
+dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_kv_cache* caches, int32_t hq,
+                                  int32_t hkv, int32_t hd, dash_bf16* O, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  namespace dec = dash::decode;
+  if (nseq < 1 || nseq > dec::kMaxSeq || hkv <= 0 || hq <= 0 || hq % hkv != 0 || (hd != 64 && hd != 128) ||
+      hq / hkv > dec::kGroupPad || nseq * hkv > dec::kMaxSegs || (hq * hd) % 8 != 0)
+    return DASH_ERR_SHAPE;
+  if (!Q || !O || !caches || !aligned16(Q) || !aligned16(O)) return DASH_ERR_INVALID_ARG;
+  const dash_kv_cache* lc[dec::kMaxSeq];
+  int64_t len[dec::kMaxSeq];
+  for (int q = 0; q < nseq; ++q) {
+    if (!caches[q].k || !caches[q].v || !aligned16(caches[q].k) || !aligned16(caches[q].v))
+      return DASH_ERR_INVALID_ARG;
+    if (caches[q].len < 1 || caches[q].len > INT32_MAX) return DASH_ERR_SHAPE;
+    lc[q] = &caches[q];
+    len[q] = caches[q].len;
+  }
+  const size_t need = dash_decode_attention_workspace_size(hd);
+  if (!ws || ws_bytes < need) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  if (di->num_sms < dec::kMaxSegs) return DASH_ERR_SHAPE;
+  dash_dims D{};
+  D.n_layers = 1;
+  D.n_heads = hq;
+  D.n_kv_heads = hkv;
+  D.head_dim = hd;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  DecodeWs w{};
+  w.Q = const_cast<bf16*>(reinterpret_cast<const bf16*>(Q));
+  w.O = reinterpret_cast<bf16*>(O);
+  w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * hd);
+  w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
+  cudaStream_t st = as_stream(stream);
+  return hd == 128 ? decode_attention_hd<128>(*di, D, nseq, len, lc, w, st)
+                   : decode_attention_hd<64>(*di, D, nseq, len, lc, w, st);
+}
+
+size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq) {
+  if (!dims_ok(dims) || nseq < 1 || nseq > dash::decode::kMaxSeq) return 0;
+  Carver c{nullptr};
+  DecodeWs w;
+  carve_decode(*dims, nseq, c, w);
+  return c.off + 256;
+}
+
+dash_status dash_decode_step(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X,
+                             int32_t nseq, const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes,
+                             void* stream) {
+  return decode_impl(dims, layers, X, nseq, pos, caches, ws, ws_bytes, stream);
+}
+
 dash_status dash_timing_start(int32_t capacity) {
   if (capacity <= 0) return DASH_ERR_INVALID_ARG;
   g_timing.recs.clear();
@@ -956,7 +1326,10 @@ int32_t dash_timing_stop(dash_launch_record* out, int32_t cap) {
 const char* dash_kernel_name(int32_t kind) {
   static const char* names[DASH_K_COUNT] = {"rope_table", "rmsnorm", "gemm_qkv_rope", "gemm_kv_halted",
                                             "attention", "gemm_o_resid_delta", "score", "gemm_gate_up_swiglu",
-                                            "gemm_down_resid", "select", "gather", "scatter", "gemm"};
+                                            "gemm_down_resid", "select", "gather", "scatter", "gemm",
+                                            "kv_store", "gemv_qkv_rope_append", "decode_attention",
+                                            "decode_combine", "gemv_o_resid", "gemv_gate_up_swiglu",
+                                            "gemv_down_resid"};
   return kind >= 0 && kind < DASH_K_COUNT ? names[kind] : "unknown";
 }
 

@@ -1,0 +1,601 @@
+// Generation on the KV cache a DASH prefill leaves behind (sm_100a).
+//
+// The DASH blog post (§3.1, generation stage; §5.1, KV cache) notes that
+// generated tokens are not pruned, but every layer past the halting layer
+// cached only the active tokens, so a new token attends to fewer keys.  One
+// step runs one new token per sequence (n <= kMaxSeq) through a layer:
+//
+//   gemv_kernel<kGvQkv>     q/k/v = rmsnorm(x) W_qkv^T, RoPE on q and k, the
+//                           new k/v (and position) appended to each cache
+//   decode_attn_kernel      split-key attention over each cache on tcgen05
+//   decode_combine_kernel   merge of the per-CTA partial softmax results
+//   gemv_kernel<kGvResid>   x += o W_o^T
+//   gemv_kernel<kGvSwiglu>  act = silu(rmsnorm(x) W_g^T) * (rmsnorm(x) W_u^T)
+//   gemv_kernel<kGvResid>   x += act W_d^T
+//
+// With n <= 8 rows the projections are HBM-bound on the weights (2 bytes
+// per multiply-add), so they run on the CUDA cores: one warp streams two
+// weight rows with 16-byte loads and keeps n dot products per row.
+//
+// The attention is HBM-bound on the cache.  Its query group (hq / hkv <= 16
+// heads) is too small for a tcgen05 M dimension, so the kernel puts the keys
+// on M instead:
+//   S^T [128 keys, 16]  = K_tile [128 keys, hd] . Q^T          (A = K, K-major)
+//   O^T [hd, 16]       += V_tile^T [hd, 128 keys] . P^T          (A = V^T, MN-major)
+// with the group padded to N = 16 columns.  TMEM lane r holds key r of the
+// tile for S^T and dimension r for O^T, so the four softmax warps own both.
+// K/V tiles arrive by TMA (128B swizzle, no multicast) in a 3-stage ring.
+#pragma once
+
+#include "common.cuh"
+
+namespace dash {
+namespace decode {
+
+constexpr int kMaxSeq = 8;
+constexpr int kMaxSegs = 64;   // sequences x kv heads in one launch
+constexpr int kMaxCtas = 256;  // decode-attention CTAs (partial-result slots)
+constexpr int kGroupPad = 16;  // query heads per kv head, padded (MMA N)
+constexpr int BKV = 128;       // keys per tile (MMA M)
+constexpr int kStages = 3;
+constexpr int kAttnThreads = 192;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units, as in the prefill softmax
+
+// =================================================================== GEMV
+enum GemvEpi : int { kGvQkv = 0, kGvResid = 1, kGvSwiglu = 2 };
+
+struct SeqSlots {
+  __nv_bfloat16* k[kMaxSeq];  // cache arrays of this layer
+  __nv_bfloat16* v[kMaxSeq];
+  int32_t* pos[kMaxSeq];      // may be NULL
+  int64_t row[kMaxSeq];       // row the new token's k/v go to
+  int32_t p[kMaxSeq];         // RoPE position of the new token
+};
+
+struct GemvParams {
+  const __nv_bfloat16* W;   // [rows, K] row-major
+  const __nv_bfloat16* W2;  // kGvSwiglu: up-projection [rows, K]
+  const __nv_bfloat16* x;   // [n, K]
+  const float* xs;          // [n] factor on each dot product (RMSNorm 1/rms) or NULL
+  int n, K, tasks;
+  __nv_bfloat16* out;  // kGvResid: residual stream [n, ldo] (in/out); kGvSwiglu: act [n, ldo]
+  int64_t ldo;
+  __nv_bfloat16* q;  // kGvQkv: [n, hq*hd]
+  int hq, hkv, hd;
+  double theta;
+  SeqSlots seq;
+};
+
+constexpr int kGemvWarps = 8;
+
+__device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
+  float a = bf16_lo(w.x) * bf16_lo(x.x);
+  float b = bf16_hi(w.x) * bf16_hi(x.x);
+  a = fmaf(bf16_lo(w.y), bf16_lo(x.y), a);
+  b = fmaf(bf16_hi(w.y), bf16_hi(x.y), b);
+  a = fmaf(bf16_lo(w.z), bf16_lo(x.z), a);
+  b = fmaf(bf16_hi(w.z), bf16_hi(x.z), b);
+  a = fmaf(bf16_lo(w.w), bf16_lo(x.w), a);
+  b = fmaf(bf16_hi(w.w), bf16_hi(x.w), b);
+  return a + b;
+}
+
+__device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Each warp owns one task = two weight rows (r0, r1) and all n inputs:
+//   kGvQkv     rows (i, i + hd/2) of one q/k/v head: the RoPE pair
+//   kGvSwiglu  row t of W (gate) and row t of W2 (up)
+//   kGvResid   rows (2t, 2t + 1)
+template <int EPI, int NS>
+__global__ void __launch_bounds__(32 * kGemvWarps) gemv_kernel(const GemvParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int task = blockIdx.x * kGemvWarps + warp;
+  if (task >= p.tasks) return;
+  const int K = p.K;
+  int head = 0, i = 0;
+  const __nv_bfloat16* w0;
+  const __nv_bfloat16* w1;
+  if constexpr (EPI == kGvQkv) {
+    const int half = p.hd >> 1;
+    head = task / half;
+    i = task - head * half;
+    w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
+    w1 = w0 + static_cast<int64_t>(half) * K;
+  } else if constexpr (EPI == kGvSwiglu) {
+    w0 = p.W + static_cast<int64_t>(task) * K;
+    w1 = p.W2 + static_cast<int64_t>(task) * K;
+  } else {
+    w0 = p.W + static_cast<int64_t>(2 * task) * K;
+    w1 = w0 + K;
+  }
+  const uint4* wa = reinterpret_cast<const uint4*>(w0);
+  const uint4* wb = reinterpret_cast<const uint4*>(w1);
+  const uint4* xv = reinterpret_cast<const uint4*>(p.x);
+  const int nv = K >> 3;
+  constexpr int U = NS <= 2 ? 4 : 2;  // 16-byte chunks per row in flight per lane
+  float a0[NS], a1[NS];
+#pragma unroll
+  for (int m = 0; m < NS; ++m) a0[m] = a1[m] = 0.f;
+  for (int c0 = lane; c0 < nv; c0 += 32 * U) {
+    uint4 ra[U], rb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nv) {
+        ra[u] = __ldcs(wa + c);  // weights stream through once per step
+        rb[u] = __ldcs(wb + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nv) {
+#pragma unroll
+        for (int m = 0; m < NS; ++m) {
+          if (m < p.n) {
+            const uint4 xm = __ldg(xv + static_cast<int64_t>(m) * nv + c);
+            a0[m] += dot8(ra[u], xm);
+            a1[m] += dot8(rb[u], xm);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NS; ++m) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a0[m] += __shfl_xor_sync(0xffffffffu, a0[m], o);
+      a1[m] += __shfl_xor_sync(0xffffffffu, a1[m], o);
+    }
+  }
+  // Epilogue: lane m finishes input row m.
+#pragma unroll
+  for (int m = 0; m < NS; ++m) {
+    if (m >= p.n || lane != m) continue;
+    const float sc = p.xs ? p.xs[m] : 1.f;
+    const float y0 = a0[m] * sc, y1 = a1[m] * sc;
+    if constexpr (EPI == kGvQkv) {
+      const int hd = p.hd, half = hd >> 1;
+      float o0 = y0, o1 = y1;
+      if (head < p.hq + p.hkv) {  // rotate-half RoPE at the token's position (fp64 angle)
+        const double inv = pow(p.theta, -2.0 * i / static_cast<double>(hd));
+        double sn, cs;
+        sincos(static_cast<double>(p.seq.p[m]) * inv, &sn, &cs);
+        const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+        o0 = y0 * c - y1 * s;
+        o1 = y1 * c + y0 * s;
+      }
+      __nv_bfloat16* dst;
+      if (head < p.hq) {
+        dst = p.q + static_cast<int64_t>(m) * p.hq * hd + head * hd;
+      } else {
+        const int kvd = p.hkv * hd;
+        const bool is_k = head < p.hq + p.hkv;
+        const int h = is_k ? head - p.hq : head - p.hq - p.hkv;
+        dst = (is_k ? p.seq.k[m] : p.seq.v[m]) + p.seq.row[m] * kvd + h * hd;
+        if (head == p.hq && i == 0 && p.seq.pos[m]) p.seq.pos[m][p.seq.row[m]] = p.seq.p[m];
+      }
+      dst[i] = __float2bfloat16_rn(o0);
+      dst[i + half] = __float2bfloat16_rn(o1);
+    } else if constexpr (EPI == kGvSwiglu) {
+      p.out[static_cast<int64_t>(m) * p.ldo + task] = __float2bfloat16_rn(y0 / (1.f + __expf(-y0)) * y1);
+    } else {
+      __nv_bfloat16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
+      const float r0 = bf16_to_f(o[0]) + y0, r1 = bf16_to_f(o[1]) + y1;
+      *reinterpret_cast<uint32_t*>(o) = pack_bf16(r0, r1);
+    }
+  }
+}
+
+// ========================================================= decode attention
+struct AttnParams {
+  const __nv_bfloat16* q;  // [n, hq*HD], RoPE applied
+  float* part_o;           // [kMaxCtas, 16, HD]: unnormalised O of each CTA
+  float* part_ml;          // [kMaxCtas, 16, 2]: (running max in log2 units, sum)
+  int n, hq, hkv, group, tiles_per_cta;
+  int len[kMaxSeq];                // keys of each sequence (cache rows incl. the new one)
+  int seg_cta0[kMaxSegs + 1];      // first CTA of segment s * hkv + h; [nseg] = CTA count
+  float scale_log2;                // log2(e) / sqrt(HD)
+};
+
+struct AttnMaps {
+  CUtensorMap k[kMaxSeq];  // [len, hkv*HD] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap v[kMaxSeq];
+};
+
+template <int HD>
+struct ACfg {
+  static constexpr int kPanels = HD / 64;
+  static constexpr int kTile = BKV * HD * 2;  // one K or V tile
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kStages * kTile;
+  // HD = 64: V^T has only 64 rows; the MMA (M = 128) reads its second 64-row
+  // panel from here (zeros), and those O^T rows are never used.
+  static constexpr int kOffZero = 2 * kStages * kTile;
+  static constexpr int kZeroBytes = HD == 64 ? BKV * 128 : 0;
+  static constexpr int kOffQ = kOffZero + kZeroBytes;   // [16, HD] K-major, kPanels x 2 KB
+  static constexpr int kOffP = kOffQ + kPanels * 2048;  // [16, 128 keys] K-major, 2 x 2 KB
+  static constexpr int kOffRed = kOffP + 4096;          // [2][4 warps][16] floats
+  static constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 4;
+  // full[kStages], empty[kStages], q_ready, s_full[2], p_full, pv_done, red[2], drain
+  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 1 + 1 + 2 + 1;
+  static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 64;  // S^T buffers [0,16) [16,32), O^T [32,48)
+};
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Byte offset of element (row, col) in a K-major 128B-swizzled operand whose
+// 64-column panels are `panel_bytes` apart (rows of 128 bytes, 8-row atoms).
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col, int panel_bytes) {
+  const int pn = col >> 6, cc = col & 63;
+  return pn * panel_bytes + row * 128 + ((((cc >> 3) ^ (row & 7)) & 7) << 4) + ((cc & 7) << 1);
+}
+
+// One CTA = a run of up to tiles_per_cta key tiles of one (sequence, kv head)
+// segment.  Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.
+// Warps 2..5: Q staging, softmax (lane r = key r of the tile), and the
+// epilogue (lane r = dimension r of O^T), writing the CTA's partial result.
+template <int HD>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    decode_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  using C = ACfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int b = blockIdx.x;
+  const int nseg = p.n * p.hkv;
+  int seg = 0;
+  while (seg + 1 < nseg && p.seg_cta0[seg + 1] <= b) ++seg;
+  const int s = seg / p.hkv, kvh = seg - s * p.hkv;
+  const int L = p.len[s];
+  const int tiles = (L + BKV - 1) / BKV;
+  const int t0 = (b - p.seg_cta0[seg]) * p.tiles_per_cta;
+  const int nt = min(t0 + p.tiles_per_cta, tiles) - t0;
+  if (nt <= 0) return;  // uniform for the whole CTA
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = smem_u32(bars + kStages);
+  const uint32_t bar_q = smem_u32(bars + 2 * kStages);
+  const uint32_t bar_sfull = bar_q + 8;   // [2]
+  const uint32_t bar_pfull = bar_q + 24;
+  const uint32_t bar_pvdone = bar_q + 32;
+  const uint32_t bar_red = bar_q + 40;    // [2]
+  const uint32_t bar_drain = bar_q + 56;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    mbar_init(bar_q, 128);
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sfull + 8, 1);
+    mbar_init(bar_pfull, 128);
+    mbar_init(bar_pvdone, 1);
+    mbar_init(bar_red, 128);
+    mbar_init(bar_red + 8, 128);
+    mbar_init(bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (HD == 64) {  // zero panel read as the upper half of V^T
+    uint4* z = reinterpret_cast<uint4*>(smem + C::kOffZero);
+    for (int i = threadIdx.x; i < C::kZeroBytes / 16; i += kAttnThreads) z[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&maps.k[s]);
+    prefetch_tmap(&maps.v[s]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t armed = 0, par = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int st = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!mbar_wait(bar_empty + 8 * st, ph ^ 1u)) break;
+        const uint32_t sk = smem_u32(smem + C::kOffK + st * C::kTile);
+        const uint32_t sv = smem_u32(smem + C::kOffV + st * C::kTile);
+        mbar_arrive_expect_tx(bar_full + 8 * st, 2 * C::kTile);
+        const int row = (t0 + i) * BKV;
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d(&maps.k[s], sk + pn * (BKV * 128), bar_full + 8 * st, kvh * HD + pn * 64, row);
+          tma_load_2d(&maps.v[s], sv + pn * (BKV * 128), bar_full + 8 * st, kvh * HD + pn * 64, row);
+        }
+        armed |= 1u << st;
+        par = (par & ~(1u << st)) | (ph << st);
+      }
+      for (int st = 0; st < kStages; ++st)
+        if ((armed >> st) & 1u) mbar_wait_drain(bar_full + 8 * st, (par >> st) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    const uint32_t idesc_s = umma_idesc_bf16(BKV, kGroupPad, false, false);
+    const uint32_t idesc_o = umma_idesc_bf16(BKV, kGroupPad, true, false);
+    const uint32_t sq = smem_u32(smem + C::kOffQ);
+    const uint32_t sp = smem_u32(smem + C::kOffP);
+    const uint32_t sz = smem_u32(smem + C::kOffZero);
+    auto issue_s = [&](int i) {  // S^T_i = K_i Q^T
+      const int st = i % kStages;
+      if (!mbar_wait(bar_full + 8 * st, (i / kStages) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sk = smem_u32(smem + C::kOffK + st * C::kTile);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t oa = (kk >> 2) * (BKV * 128) + (kk & 3) * 32;
+          const uint32_t ob = (kk >> 2) * 2048 + (kk & 3) * 32;
+          umma_bf16_ss(tmem_base + (i & 1) * kGroupPad, umma_desc_sw128(sk + oa, 16, 1024),
+                       umma_desc_sw128(sq + ob, 16, 1024), idesc_s, kk != 0 ? 1u : 0u);
+        }
+        umma_commit(bar_sfull + 8 * (i & 1));
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int i) {  // O^T += V_i^T P_i^T
+      if (!mbar_wait(bar_pfull, i & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const int st = i % kStages;
+        const uint32_t sv = smem_u32(smem + C::kOffV + st * C::kTile);
+        const uint32_t lbo = HD == 128 ? BKV * 128 : sz - sv;  // stride of V^T's two 64-row panels
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint32_t ob = (kk >> 2) * 2048 + (kk & 3) * 32;
+          umma_bf16_ss(tmem_base + 2 * kGroupPad, umma_desc_sw128(sv + kk * 16 * 128, lbo, 1024),
+                       umma_desc_sw128(sp + ob, 16, 1024), idesc_o, (i != 0 || kk != 0) ? 1u : 0u);
+        }
+        umma_commit(bar_pvdone);
+        umma_commit(bar_empty + 8 * st);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = mbar_wait(bar_q, 0);
+    if (ok) ok = issue_s(0);
+    for (int i = 0; ok && i < nt; ++i) {
+      if (i + 1 < nt) ok = issue_s(i + 1);
+      if (ok) ok = issue_pv(i);
+    }
+    if (lane == 0) umma_commit(bar_drain);
+    __syncwarp();
+    mbar_wait_drain(bar_drain, 0);
+  } else {
+    // ---------------------------------------------- Q staging, softmax, epilogue
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int G = p.group;
+    // Q of this kv head's group, rows G..15 zero, K-major 128B-swizzled.
+    {
+      const __nv_bfloat16* qs = p.q + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
+      constexpr int kChunks = kGroupPad * HD / 8;
+      for (int ch = r; ch < kChunks; ch += 128) {
+        const int g = ch / (HD / 8), c = ch - g * (HD / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (g < G) v = *reinterpret_cast<const uint4*>(qs + g * HD + c * 8);
+        *reinterpret_cast<uint4*>(smem + C::kOffQ + sw128_offset(g, c * 8, 2048)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_q);
+    }
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    const float sc = p.scale_log2;
+    float m_run[kGroupPad], l_part[kGroupPad];
+#pragma unroll
+    for (int g = 0; g < kGroupPad; ++g) {
+      m_run[g] = -INFINITY;
+      l_part[g] = 0.f;
+    }
+    bool ok = true;
+    for (int i = 0; i < nt; ++i) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull + 8 * (i & 1), (i >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t u[kGroupPad];
+      tmem_ld16(tmem_base + lane_off + (i & 1) * kGroupPad, u);
+      tmem_ld_wait();
+      const bool valid = (t0 + i) * BKV + r < L;
+      float sv[kGroupPad], mx[kGroupPad];
+#pragma unroll
+      for (int g = 0; g < kGroupPad; ++g) {
+        sv[g] = valid ? __uint_as_float(u[g]) * sc : -INFINITY;
+        mx[g] = sv[g];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int g = 0; g < kGroupPad; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
+      // tile maximum per head over the four warps (mbarrier exchange)
+      float* rb = red + (i & 1) * 64;
+      if (lane < kGroupPad) {
+        float v = mx[0];
+#pragma unroll
+        for (int g = 1; g < kGroupPad; ++g) v = lane == g ? mx[g] : v;
+        rb[wq * 16 + lane] = v;
+      }
+      mbar_arrive(bar_red + 8 * (i & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_red + 8 * (i & 1), (i >> 1) & 1));
+      if (!ok) break;
+      bool rescale = false;
+      float alpha[kGroupPad];
+#pragma unroll
+      for (int g = 0; g < kGroupPad; ++g) {
+        const float mt = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
+        alpha[g] = 1.f;
+        if (i == 0) {
+          m_run[g] = mt;  // the first tile of a run always holds a valid key
+        } else if (mt > m_run[g] + kRescaleThreshold) {
+          rescale = true;
+        }
+        mx[g] = mt;
+      }
+      if (rescale) {  // identical decision in every thread (same inputs)
+#pragma unroll
+        for (int g = 0; g < kGroupPad; ++g) {
+          const float mn = fmaxf(m_run[g], mx[g]);
+          alpha[g] = mn == m_run[g] ? 1.f : ex2f(m_run[g] - mn);
+          m_run[g] = mn;
+          l_part[g] *= alpha[g];
+        }
+      }
+      uint16_t pb[kGroupPad];
+#pragma unroll
+      for (int g = 0; g < kGroupPad; ++g) {
+        const float e = valid ? ex2f(sv[g] - m_run[g]) : 0.f;
+        const __nv_bfloat16 eb = __float2bfloat16_rn(e);
+        l_part[g] += e;
+        pb[g] = *reinterpret_cast<const uint16_t*>(&eb);
+      }
+      // P^T buffer and O^T are free once P_(i-1) V_(i-1) is done.
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone, (i - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (rescale) {
+        uint32_t o[kGroupPad];
+        tmem_ld16(tmem_base + lane_off + 2 * kGroupPad, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < kGroupPad; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+        tmem_st16(tmem_base + lane_off + 2 * kGroupPad, o);
+        tmem_st_wait();
+      }
+#pragma unroll
+      for (int g = 0; g < kGroupPad; ++g)
+        *reinterpret_cast<uint16_t*>(smem + C::kOffP + sw128_offset(g, r, 2048)) = pb[g];
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_pfull);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone, (nt - 1) & 1));
+    if (ok) {
+      tc_fence_after();
+      uint32_t o[kGroupPad];
+      tmem_ld16(tmem_base + lane_off + 2 * kGroupPad, o);
+      tmem_ld_wait();
+      // sum of each head's exponentials over the CTA's keys
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < kGroupPad; ++g) l_part[g] += __shfl_xor_sync(0xffffffffu, l_part[g], off);
+      float* rb = red + (nt & 1) * 64;  // the buffer tile nt would use: free now
+      if (lane < kGroupPad) {
+        float v = l_part[0];
+#pragma unroll
+        for (int g = 1; g < kGroupPad; ++g) v = lane == g ? l_part[g] : v;
+        rb[wq * 16 + lane] = v;
+      }
+      mbar_arrive(bar_red + 8 * (nt & 1));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_red + 8 * (nt & 1), (nt >> 1) & 1));
+      if (ok) {
+        float* po = p.part_o + static_cast<int64_t>(b) * kGroupPad * HD;
+        if (r < HD)
+#pragma unroll
+          for (int g = 0; g < kGroupPad; ++g)
+            if (g < G) po[g * HD + r] = __uint_as_float(o[g]);
+        if (r < G) {
+          float mr = m_run[0], lr = 0.f;
+#pragma unroll
+          for (int g = 0; g < kGroupPad; ++g)
+            if (g == r) {
+              mr = m_run[g];
+              lr = (rb[g] + rb[16 + g]) + (rb[32 + g] + rb[48 + g]);
+            }
+          float* pm = p.part_ml + (static_cast<int64_t>(b) * kGroupPad + r) * 2;
+          pm[0] = mr;
+          pm[1] = lr;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// O[s, head, :] = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c over the CTAs c
+// of the head's segment (M = max m_c).  One block of HD threads per (s, head).
+template <int HD>
+__global__ void decode_combine_kernel(const AttnParams p, __nv_bfloat16* __restrict__ out) {
+  const int s = blockIdx.x / p.hq, head = blockIdx.x - s * p.hq;
+  const int kvh = head / p.group, g = head - kvh * p.group;
+  const int seg = s * p.hkv + kvh;
+  const int c0 = p.seg_cta0[seg], c1 = p.seg_cta0[seg + 1];
+  const int d = threadIdx.x;
+  float M = -INFINITY;
+  for (int c = c0; c < c1; ++c) M = fmaxf(M, p.part_ml[(static_cast<int64_t>(c) * kGroupPad + g) * 2]);
+  float l = 0.f, acc = 0.f;
+  for (int c = c0; c < c1; ++c) {
+    const float* ml = p.part_ml + (static_cast<int64_t>(c) * kGroupPad + g) * 2;
+    const float w = ex2f(ml[0] - M);
+    l = fmaf(w, ml[1], l);
+    acc = fmaf(w, p.part_o[(static_cast<int64_t>(c) * kGroupPad + g) * HD + d], acc);
+  }
+  out[static_cast<int64_t>(s) * p.hq * HD + head * HD + d] = __float2bfloat16_rn(acc / l);
+}
+
+// ============================================================ cache store
+// Rows [a, a + rows) of the prefill's per-layer K/V buffers -> cache rows
+// [0, rows); pos[r] = pos_src[a + r] (or r when pos_src is NULL).
+__global__ void kv_store_kernel(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
+                                int kvd, int64_t a, int64_t rows, const int32_t* __restrict__ pos_src,
+                                __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
+                                int32_t* __restrict__ pos) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int nv = kvd >> 3;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * wpb + warp; r < rows; r += gridDim.x * wpb) {
+    const uint4* sk = reinterpret_cast<const uint4*>(Kb + (a + r) * kvd);
+    const uint4* svv = reinterpret_cast<const uint4*>(Vb + (a + r) * kvd);
+    uint4* dk = reinterpret_cast<uint4*>(k + r * kvd);
+    uint4* dv = reinterpret_cast<uint4*>(v + r * kvd);
+    for (int c = lane; c < nv; c += 32) {
+      dk[c] = sk[c];
+      dv[c] = svv[c];
+    }
+    if (pos && lane == 0) pos[r] = pos_src ? pos_src[a + r] : static_cast<int32_t>(r);
+  }
+}
+
+}  // namespace decode
+}  // namespace dash

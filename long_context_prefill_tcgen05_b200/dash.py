@@ -52,6 +52,10 @@ class HaltCtx(ctypes.Structure):
     _fields_ = [("active_idx", c_vp), ("halted_idx", c_vp), ("h_full", c_vp), ("T", c_i64)]
 
 
+class KVCacheDesc(ctypes.Structure):
+    _fields_ = [("k", c_vp), ("v", c_vp), ("pos", c_vp), ("capacity", c_i64), ("len", c_i64)]
+
+
 _SIGS = {
     "dash_status_string": (ctypes.c_char_p, [c_i32]),
     "dash_device_error": (c_i32, []),
@@ -77,6 +81,19 @@ _SIGS = {
     "dash_layer_forward_noalloc": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64, c_vp,
                                            c_i64, ctypes.POINTER(HaltCtx), c_vp, c_i32, c_vp]),
     "dash_exp2_fma": (c_i32, [c_vp, c_i64, c_vp, c_vp]),
+    "dash_prefill_kv": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i64,
+                                ctypes.POINTER(Config), c_vp, ctypes.POINTER(c_i64), c_vp,
+                                ctypes.POINTER(KVCacheDesc), c_vp, c_sz, c_vp]),
+    "dash_prefill_varlen_kv": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp,
+                                       ctypes.POINTER(c_i32), c_i32, ctypes.POINTER(Config), c_vp,
+                                       ctypes.POINTER(c_i64), ctypes.POINTER(c_i32), c_vp,
+                                       ctypes.POINTER(KVCacheDesc), c_vp, c_sz, c_vp]),
+    "dash_decode_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i32]),
+    "dash_decode_attention_workspace_size": (c_sz, [c_i32]),
+    "dash_decode_attention": (c_i32, [c_vp, c_i32, ctypes.POINTER(KVCacheDesc), c_i32, c_i32, c_i32, c_vp, c_vp,
+                                      c_sz, c_vp]),
+    "dash_decode_step": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp, c_i32,
+                                 ctypes.POINTER(c_i32), ctypes.POINTER(KVCacheDesc), c_vp, c_sz, c_vp]),
     "dash_selftest_wait_timeout": (c_i32, [c_vp]),
     "dash_timing_start": (c_i32, [c_i32]),
     "dash_timing_stop": (c_i32, [ctypes.POINTER(LaunchRecord), c_i32]),
@@ -311,3 +328,94 @@ def prefill(stack, H, cfg, idx_out=None, delta_out=None, stream=None):
     _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _p(H), T, ctypes.byref(cfg), _p(idx_out),
                               ctypes.byref(K), _p(delta_out), _p(ws), ws.numel(), _stream(stream)), "dash_prefill")
     return K.value
+
+
+# ------------------------------------------------------------- KV cache
+class KVCache:
+    """Caller-owned KV caches for nseq sequences x n_layers layers.
+
+    capacity: rows per cache, one int for all, or a list per layer.  The
+    descriptor array ``desc`` (dash_kv_cache[nseq * n_layers], sequence-
+    major) is what the library reads and whose ``len`` fields it updates.
+    """
+
+    def __init__(self, stack, nseq=1, capacity=0, device="cuda", with_pos=True):
+        L = stack.n_layers
+        caps = [int(capacity)] * L if isinstance(capacity, int) else [int(c) for c in capacity]
+        kvd = stack.dims.n_kv_heads * stack.dims.head_dim
+        self.nseq, self.n_layers = nseq, L
+        self.k, self.v, self.pos = [], [], []
+        self.desc = (KVCacheDesc * (nseq * L))()
+        for s in range(nseq):
+            for l in range(L):
+                k = torch.zeros(max(caps[l], 1), kvd, dtype=torch.bfloat16, device=device)
+                v = torch.zeros_like(k)
+                p = torch.full((max(caps[l], 1),), -1, dtype=torch.int32, device=device) if with_pos else None
+                self.k.append(k)
+                self.v.append(v)
+                self.pos.append(p)
+                self.desc[s * L + l] = KVCacheDesc(k.data_ptr(), v.data_ptr(), p.data_ptr() if with_pos else None,
+                                                   caps[l], 0)
+
+    def lens(self, s=0):
+        return [self.desc[s * self.n_layers + l].len for l in range(self.n_layers)]
+
+    def layer(self, s, l):
+        """(k [len, kvd], v, pos [len] or None) of sequence s, layer l."""
+        i = s * self.n_layers + l
+        n = self.desc[i].len
+        return self.k[i][:n], self.v[i][:n], (self.pos[i][:n] if self.pos[i] is not None else None)
+
+
+def prefill_kv(stack, H, cfg, cache, idx_out=None, delta_out=None, stream=None):
+    """dash_prefill_kv: dash_prefill that also fills cache (KVCache, nseq = 1); returns K."""
+    T = H.shape[0]
+    need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
+    ws = workspace(need, H.device)
+    K = c_i64(0)
+    _check(lib().dash_prefill_kv(ctypes.byref(stack.dims), stack.layers, _p(H), T, ctypes.byref(cfg), _p(idx_out),
+                                 ctypes.byref(K), _p(delta_out), cache.desc, _p(ws), ws.numel(), _stream(stream)),
+           "dash_prefill_kv")
+    return K.value
+
+
+def prefill_varlen_kv(stack, H, cu_seqlens, cfg, cache, idx_out=None, delta_out=None, stream=None):
+    """dash_prefill_varlen_kv; returns (K, per-sequence active counts)."""
+    cu = [int(x) for x in cu_seqlens]
+    nseq = len(cu) - 1
+    T = H.shape[0]
+    need = lib().dash_prefill_varlen_workspace_size(ctypes.byref(stack.dims), T, nseq, ctypes.byref(cfg))
+    ws = workspace(need, H.device)
+    cu_arr = (c_i32 * (nseq + 1))(*cu)
+    counts = (c_i32 * nseq)()
+    K = c_i64(0)
+    _check(lib().dash_prefill_varlen_kv(ctypes.byref(stack.dims), stack.layers, _p(H), cu_arr, nseq,
+                                        ctypes.byref(cfg), _p(idx_out), ctypes.byref(K), counts, _p(delta_out),
+                                        cache.desc, _p(ws), ws.numel(), _stream(stream)), "dash_prefill_varlen_kv")
+    return K.value, list(counts)
+
+
+def decode_step(stack, X, pos, cache, stream=None):
+    """dash_decode_step in place on X [nseq, d]: one new token per sequence at
+    the host positions pos; appends to cache (KVCache)."""
+    n = X.shape[0]
+    need = lib().dash_decode_workspace_size(ctypes.byref(stack.dims), n)
+    ws = workspace(need, X.device)
+    pos_arr = (c_i32 * n)(*[int(p) for p in pos])
+    _check(lib().dash_decode_step(ctypes.byref(stack.dims), stack.layers, _p(X), n, pos_arr, cache.desc, _p(ws),
+                                  ws.numel(), _stream(stream)), "dash_decode_step")
+    return X
+
+
+def decode_attention(Q, kv, hq, hkv, hd, out=None, stream=None):
+    """dash_decode_attention: Q [nseq, hq*hd]; kv = list of (K [len, hkv*hd], V) per sequence."""
+    n = Q.shape[0]
+    out = torch.empty_like(Q) if out is None else out
+    desc = (KVCacheDesc * n)()
+    for s, (k, v) in enumerate(kv):
+        desc[s] = KVCacheDesc(k.data_ptr(), v.data_ptr(), None, k.shape[0], k.shape[0])
+    need = lib().dash_decode_attention_workspace_size(hd)
+    ws = workspace(need, Q.device)
+    _check(lib().dash_decode_attention(_p(Q), n, desc, hq, hkv, hd, _p(out), _p(ws), ws.numel(), _stream(stream)),
+           "dash_decode_attention")
+    return out

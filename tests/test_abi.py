@@ -117,3 +117,58 @@ def test_workspace_sizes_grow_with_tokens(L):
     # activations for T = 32768 fit well inside one GPU's memory
     assert 1 << 30 < big < 8 << 30
     assert L.dash_layer_workspace_size(ctypes.byref(dims), 100, 50, 100) == 0  # T_kv < M rejected
+
+
+def _cache_arr(n, k=FAKE, v=FAKE, cap=1024, ln=0):
+    arr = (dash.KVCacheDesc * n)()
+    for i in range(n):
+        arr[i] = dash.KVCacheDesc(k, v, None, cap, ln)
+    return arr
+
+
+def test_kv_cache_and_decode_argument_errors(L):
+    dims = _dims()
+    layers = _fake_layers(4)
+    cfg = dash.make_config(halt_layer=1, mode="prune", keep=0.5)
+    K = ctypes.c_int64(0)
+    pre = lambda caches, T=512, c=cfg: L.dash_prefill_kv(ctypes.byref(dims), layers, FAKE, T, ctypes.byref(c), None,
+                                                         ctypes.byref(K), None, caches, None, 0, None)
+    assert pre(None) == 1                                                  # caches required
+    assert pre(_cache_arr(4, cap=511)) == 2                                # layer 0 holds T = 512 rows
+    small = _cache_arr(4, cap=512)
+    small[3].capacity = 255                                                # K = 256 rows after L_s
+    assert pre(small) == 2
+    small[3].capacity = 256
+    assert pre(small) == 4                                                 # capacities fine, no workspace
+    halt = dash.make_config(halt_layer=1, mode="halt", keep=0.5)
+    assert pre(small, c=halt) == 2                                         # halt keeps T rows in every layer
+    assert pre(_cache_arr(4, k=FAKE + 8)) == 1                             # misaligned cache
+    assert pre(_cache_arr(4, ln=2000)) == 1                                # len > capacity
+    # an empty prompt resets the lengths without touching the device
+    emp = _cache_arr(4, ln=7)
+    assert pre(emp, T=0) == 0 and [c.len for c in emp] == [0] * 4
+
+    ws = L.dash_decode_workspace_size(ctypes.byref(dims), 2)
+    assert ws > 0 and L.dash_decode_workspace_size(ctypes.byref(dims), 9) == 0
+    pos = (ctypes.c_int32 * 2)(10, 20)
+    dec = lambda n, caches, p=pos, w=None, wb=0: L.dash_decode_step(ctypes.byref(dims), layers, FAKE, n, p, caches,
+                                                                     w, wb, None)
+    assert dec(0, _cache_arr(8)) == 2                                      # no sequences
+    assert dec(9, _cache_arr(36)) == 2                                     # more than DASH_DECODE_MAX_SEQ
+    assert dec(2, None) == 1
+    assert dec(2, _cache_arr(8), p=None) == 1
+    assert dec(2, _cache_arr(8, cap=5, ln=5)) == 2                         # a full cache
+    assert dec(2, _cache_arr(8, ln=3)) == 4                                # valid, no workspace
+    assert dec(2, _cache_arr(8, ln=3), w=FAKE, wb=ws - 1) == 4             # one byte short
+    neg = (ctypes.c_int32 * 2)(-1, 3)
+    assert dec(2, _cache_arr(8), p=neg) == 1                               # negative position
+    # decode attention op
+    cs = _cache_arr(2, ln=100)
+    att = lambda n, hq, hkv, hd, caches=cs, w=None, wb=0: L.dash_decode_attention(FAKE, n, caches, hq, hkv, hd, FAKE,
+                                                                                  w, wb, None)
+    assert att(2, 4, 2, 96) == 2                                           # head_dim
+    assert att(2, 68, 2, 64) == 2                                          # group of 34 > 16
+    assert att(9, 4, 2, 64) == 2                                           # too many sequences
+    assert att(2, 4, 2, 64, caches=_cache_arr(2, ln=0)) == 2               # an empty cache
+    assert att(2, 4, 2, 64) == 4                                           # no workspace
+    assert L.dash_decode_attention_workspace_size(64) > 0 and L.dash_decode_attention_workspace_size(80) == 0
