@@ -232,6 +232,72 @@ def run_reference(args, world, rank):
                               "d2h_bytes_per_step": 0}}), flush=True)
 
 
+# --------------------------------------------------------------- decode
+def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, steps=16, warmup=3):
+    """Generation after the prefill: ms per step (one new token per sequence)
+    on the cache a DASH prefill leaves (prune mode: later layers hold the
+    active tokens only) against the dense prefill's cache."""
+    nseq = len(cu) - 1 if cu else 1
+    T_max = max(b - a for a, b in zip(cu[:-1], cu[1:])) if cu else h0.shape[0]
+    total = warmup + 2 * steps  # warm-up, a plain timed run, a run with per-kernel events
+    g = torch.Generator(device=dev).manual_seed(99)
+    out = {}
+    for name, c in (("dash_cache", cfg_cache), ("dense_cache", cfg_dense)):
+        cache = dash.KVCache(stack, nseq, T_max + total, device=dev)
+        H = h0.clone()
+        if cu:
+            dash.prefill_varlen_kv(stack, H, cu, c, cache)
+        else:
+            dash.prefill_kv(stack, H, c, cache)
+        del H
+        starts = [cu[s + 1] - cu[s] for s in range(nseq)] if cu else [h0.shape[0]]
+        xs = torch.randn(total, nseq, dims.d_model, generator=g, device=dev).to(torch.bfloat16)
+        for j in range(warmup):
+            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
+        torch.cuda.synchronize()
+        base = [cache.lens(s) for s in range(nseq)]  # rows per layer before the timed steps
+        step_bytes = sum(costs.decode_step_bytes(dims, [[b + 1 + j for b in base[s]] for s in range(nseq)])
+                         for j in range(steps)) / steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for j in range(warmup, warmup + steps):
+            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        dash.timing_start()
+        for j in range(warmup + steps, total):
+            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
+        torch.cuda.synchronize()
+        recs = dash.timing_stop()
+        per = {}
+        for r in recs:
+            unit, amount = costs.launch_work(r, dims)
+            q = per.setdefault(r["kind"], {"ms": 0.0, "bytes": 0, "launches": 0})
+            q["ms"] += r["ms"]
+            q["bytes"] += amount
+            q["launches"] += 1
+        dom = max(per, key=lambda k: per[k]["ms"])
+        gbs = per[dom]["bytes"] / (per[dom]["ms"] / 1e3) / 1e9
+        out[name] = {"ms_per_step": ms, "tokens_per_s": nseq / (ms / 1e3),
+                     "cached_rows_per_layer": cache.lens(0),
+                     "step_gb": step_bytes / 1e9, "step_gbs": step_bytes / (ms / 1e3) / 1e9,
+                     "step_frac_of_hbm": step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "gpu_launches_per_step": len(recs) // steps,
+                     "kernels": {k: {"ms_per_step": v["ms"] / steps, "launches_per_step": v["launches"] // steps,
+                                     "gbs": v["bytes"] / (v["ms"] / 1e3) / 1e9 if v["ms"] else 0.0}
+                                 for k, v in sorted(per.items(), key=lambda kv: -kv[1]["ms"])},
+                     "roofline": {"bound": "hbm", "kernel": dom, "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}}
+        del cache, xs
+        torch.cuda.empty_cache()
+    out["speedup_vs_dense_cache"] = out["dense_cache"]["ms_per_step"] / out["dash_cache"]["ms_per_step"]
+    out["sequences"] = nseq
+    out["steps"] = steps
+    out["warmup"] = warmup
+    return out
+
+
 # ------------------------------------------------------------------ ours
 def main():
     ap = argparse.ArgumentParser()
@@ -243,6 +309,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the dense / other-mode / e2e legs")
+    ap.add_argument("--no-decode", action="store_true", help="skip the generation leg")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.impl == "reference":
@@ -412,6 +479,12 @@ def main():
         extra["e2e"] = {"value": world * T / (ms_e / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": T * dims.d_model * 2, "d2h_bytes_per_step": rows * dims.d_model * 2}
     dash.check_device()
+    if not args.no_decode:
+        # the cache of a prune-mode prefill with the workload's selection
+        cfg_cache = dash.make_config(halt_layer=wl["halt_layer"], mode="prune", select=wl["select"],
+                                     keep=wl["keep"], threshold=threshold, relative=wl["relative"])
+        extra["decode"] = decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks)
+        dash.check_device()
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -56,6 +56,22 @@ def varlen_prefill_flops(dims, cu, halt_layer=None, counts=None, mode="dense", a
     return total
 
 
+def layer_weight_bytes(dims):
+    """bf16 bytes of one decoder layer's weights (projections and norm gains)."""
+    d, hd, F = dims.d_model, dims.head_dim, dims.ffn_dim
+    qd, kvd = dims.n_heads * hd, dims.n_kv_heads * hd
+    return 2 * (d * (qd + 2 * kvd) + qd * d + 2 * F * d + F * d + 2 * d)
+
+
+def decode_step_bytes(dims, cache_lens):
+    """HBM bytes one generation step must move: every layer's weights once,
+    plus, per sequence and layer, the cached keys/values it attends over
+    (cache_lens[s][l] rows after the append) and the appended row."""
+    kvd = dims.n_kv_heads * dims.head_dim
+    kv = sum(sum(lens) for lens in cache_lens) * kvd * 2 * 2
+    return dims.n_layers * layer_weight_bytes(dims) + kv
+
+
 def launch_work(rec, dims, pairs_by_rows=None):
     """(unit, amount) of algorithmic work for one timed launch record.  Attention
     launches whose visible pairs the library cannot count on the host (query
@@ -77,4 +93,12 @@ def launch_work(rec, dims, pairs_by_rows=None):
         return "byte", m * 4 + m * 4
     if kind == "rope_table":
         return "byte", m * n * 8
+    if kind.startswith("gemv"):          # weights [n, k] once, m input rows, m output rows
+        return "byte", 2 * (n * k + m * k + m * n)
+    if kind == "decode_attention":       # n cached rows (summed over sequences), K and V
+        return "byte", n * dims.n_kv_heads * dims.head_dim * 2 * 2
+    if kind == "decode_combine":         # n CTAs' partial results for m sequences
+        return "byte", n * 16 * (dims.head_dim + 2) * 4
+    if kind == "kv_store":               # m rows of K and V read and written
+        return "byte", m * n * 2 * 2 * 2
     return "byte", 0
