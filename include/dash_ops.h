@@ -75,8 +75,7 @@ typedef enum dash_kernel_kind {
   DASH_K_ATTENTION = 4, DASH_K_GEMM_O = 5, DASH_K_SCORE = 6, DASH_K_GEMM_GATE_UP = 7,
   DASH_K_GEMM_DOWN = 8, DASH_K_SELECT = 9, DASH_K_GATHER = 10, DASH_K_SCATTER = 11,
   DASH_K_GEMM = 12, DASH_K_KV_STORE = 13, DASH_K_DEC_GEMV_QKV = 14, DASH_K_DEC_ATTENTION = 15,
-  DASH_K_DEC_COMBINE = 16, DASH_K_DEC_GEMV_O = 17, DASH_K_DEC_GEMV_GATE_UP = 18, DASH_K_DEC_GEMV_DOWN = 19,
-  DASH_K_COUNT = 20
+  DASH_K_DEC_GEMV_O = 16, DASH_K_DEC_GEMV_GATE_UP = 17, DASH_K_DEC_GEMV_DOWN = 18, DASH_K_COUNT = 19
 } dash_kernel_kind;
 
 typedef struct dash_launch_record {
@@ -84,7 +83,7 @@ typedef struct dash_launch_record {
   int32_t layer;  /* decoder layer, -1 outside the layer loop */
   int64_t m;      /* rows (GEMM M, attention query rows, selection T, decode sequences) */
   int64_t n;      /* GEMM N, attention key rows (decode: cached keys summed over sequences) */
-  int64_t k;      /* GEMM K, attention causal (query, key) pairs */
+  int64_t k;      /* GEMM K, attention causal (query, key) pairs (decode: CTAs) */
   float ms;       /* device time between the two events */
 } dash_launch_record;
 

@@ -97,8 +97,6 @@ def launch_work(rec, dims, pairs_by_rows=None):
         return "byte", 2 * (n * k + m * k + m * n)
     if kind == "decode_attention":       # n cached rows (summed over sequences), K and V
         return "byte", n * dims.n_kv_heads * dims.head_dim * 2 * 2
-    if kind == "decode_combine":         # n CTAs' partial results for m sequences
-        return "byte", n * 16 * (dims.head_dim + 2) * 4
     if kind == "kv_store":               # m rows of K and V read and written
         return "byte", m * n * 2 * 2 * 2
     return "byte", 0

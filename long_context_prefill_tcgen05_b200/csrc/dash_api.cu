@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "dash.h"
@@ -760,8 +761,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
 namespace dec = dash::decode;
 
 struct DecodeWs {
-  bf16* Xn;        // [n, d] x * g of the current norm
-  float* rs;       // [n] its 1/rms
+  int* counters;   // [kMaxSegs] finished decode-attention CTAs per segment
   bf16* Q;         // [n, hq*hd]
   bf16* O;         // [n, hq*hd] attention output
   bf16* Act;       // [n, F]
@@ -771,8 +771,7 @@ struct DecodeWs {
 
 void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
-  w.Xn = c.take<bf16>(static_cast<size_t>(n) * D.d_model);
-  w.rs = c.take<float>(static_cast<size_t>(n));
+  w.counters = c.take<int>(dec::kMaxSegs);
   w.Q = c.take<bf16>(n * qd);
   w.O = c.take<bf16>(n * qd);
   w.Act = c.take<bf16>(static_cast<size_t>(n) * D.ffn_dim);
@@ -780,21 +779,59 @@ void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
 }
 
+// Launch with programmatic dependent launch: the kernel may be scheduled
+// while its predecessor on the stream finishes; it waits (griddepcontrol)
+// before reading that predecessor's results.
+template <typename... ExpTypes, typename... ActTypes>
+cudaError_t launch_pdl(void (*kernel)(ExpTypes...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       ActTypes&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<ActTypes>(args)...);
+}
+
+constexpr size_t kGemvSmemMax = 160 * 1024;  // x staged in shared memory up to this size
+
 template <int EPI, int NS>
-dash_status launch_gemv_ns(const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
+dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out,
+                           cudaStream_t st) {
   if (gp.tasks == 0) return DASH_OK;
-  const unsigned blocks = static_cast<unsigned>((gp.tasks + dec::kGemvWarps - 1) / dec::kGemvWarps);
+  constexpr bool kNorm = EPI != dec::kGvResid;
+  const size_t xbytes = static_cast<size_t>(gp.n) * gp.K * 2;
+  const bool stage = kNorm || xbytes <= kGemvSmemMax;
+  if (kNorm && xbytes > kGemvSmemMax) return DASH_ERR_SHAPE;
+  dec::GemvParams q = gp;
+  q.stage_x = !kNorm && stage;
+  const size_t smem = stage ? xbytes : 0;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(dec::gemv_kernel<EPI, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(kGemvSmemMax));
+  });
+  if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  // one CTA per SM (tasks strided over the grid), so every SM streams weights
+  const unsigned grid = static_cast<unsigned>(gp.tasks < di.num_sms ? gp.tasks : di.num_sms);
   TimedLaunch tl(kind, gp.n, n_out, gp.K, st);
-  dec::gemv_kernel<EPI, NS><<<blocks, 32 * dec::kGemvWarps, 0, st>>>(gp);
+  if (launch_pdl(dec::gemv_kernel<EPI, NS>, grid, 32 * dec::kGemvWarps, smem, st, q) != cudaSuccess)
+    return DASH_ERR_CUDA;
   return launch_status();
 }
 
 template <int EPI>
-dash_status launch_gemv(const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
-  if (gp.n <= 1) return launch_gemv_ns<EPI, 1>(gp, kind, n_out, st);
-  if (gp.n <= 2) return launch_gemv_ns<EPI, 2>(gp, kind, n_out, st);
-  if (gp.n <= 4) return launch_gemv_ns<EPI, 4>(gp, kind, n_out, st);
-  return launch_gemv_ns<EPI, 8>(gp, kind, n_out, st);
+dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
+  if (gp.n <= 1) return launch_gemv_ns<EPI, 1>(di, gp, kind, n_out, st);
+  if (gp.n <= 2) return launch_gemv_ns<EPI, 2>(di, gp, kind, n_out, st);
+  if (gp.n <= 4) return launch_gemv_ns<EPI, 4>(di, gp, kind, n_out, st);
+  return launch_gemv_ns<EPI, 8>(di, gp, kind, n_out, st);
 }
 
 // Split-key decode attention of one layer: the CTA count is held to one
@@ -849,6 +886,8 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   }
   ap.seg_cta0[n * hkv] = c0;
   ap.q = w.Q;
+  ap.out = w.O;
+  ap.counters = w.counters;
   ap.part_o = w.part_o;
   ap.part_ml = w.part_ml;
   ap.n = n;
@@ -857,14 +896,10 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   ap.group = D.n_heads / hkv;
   ap.tiles_per_cta = static_cast<int>(per);
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
-  {
-    TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, 0, st);
-    dec::decode_attn_kernel<HD><<<static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st>>>(maps, ap);
-  }
-  dash_status s = launch_status();
-  if (s != DASH_OK) return s;
-  TimedLaunch tl(DASH_K_DEC_COMBINE, n, nctas, 0, st);
-  dec::decode_combine_kernel<HD><<<static_cast<unsigned>(n * D.n_heads), HD, 0, st>>>(ap, w.O);
+  TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, nctas, st);
+  if (launch_pdl(dec::decode_attn_kernel<HD>, static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st,
+                 maps, ap) != cudaSuccess)
+    return DASH_ERR_CUDA;
   return launch_status();
 }
 
@@ -900,6 +935,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
   bf16* x = reinterpret_cast<bf16*>(X);
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd;
+  if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
 
   for (int l = 0; l < D.n_layers; ++l) {
     g_timing.layer = l;
@@ -917,11 +953,11 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
       qkv.seq.p[q] = pos[q];
       len[q] = lc[q]->len + 1;
     }
-    // RMSNorm -> QKV with RoPE, appended to the caches
-    if ((s = rmsnorm(x, n, nullptr, n, d, cb(lw.attn_norm), D.rms_eps, w.Xn, st, w.rs)) != DASH_OK) break;
+    // RMSNorm (fused) -> QKV with RoPE, appended to the caches
     qkv.W = cb(lw.w_qkv);
-    qkv.x = w.Xn;
-    qkv.xs = w.rs;
+    qkv.x = x;
+    qkv.gain = cb(lw.attn_norm);
+    qkv.eps = static_cast<float>(D.rms_eps);
     qkv.n = n;
     qkv.K = d;
     qkv.tasks = (hq + 2 * hkv) * hd / 2;
@@ -930,7 +966,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     qkv.hkv = hkv;
     qkv.hd = hd;
     qkv.theta = D.rope_theta;
-    if ((s = launch_gemv<dec::kGvQkv>(qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvQkv>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
     // attention over each sequence's cache (including the new row)
     s = hd == 128 ? decode_attention_hd<128>(*di, D, n, len, lc, w, st)
                   : decode_attention_hd<64>(*di, D, n, len, lc, w, st);
@@ -945,21 +981,21 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     o.tasks = d / 2;
     o.out = x;
     o.ldo = d;
-    if ((s = launch_gemv<dec::kGvResid>(o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
-    // RMSNorm -> gate/up with SwiGLU
-    if ((s = rmsnorm(x, n, nullptr, n, d, cb(lw.ffn_norm), D.rms_eps, w.Xn, st, w.rs)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
+    // RMSNorm (fused) -> gate/up with SwiGLU
     dec::GemvParams gu;
     std::memset(&gu, 0, sizeof(gu));
     gu.W = cb(lw.w_gate);
     gu.W2 = cb(lw.w_up);
-    gu.x = w.Xn;
-    gu.xs = w.rs;
+    gu.x = x;
+    gu.gain = cb(lw.ffn_norm);
+    gu.eps = static_cast<float>(D.rms_eps);
     gu.n = n;
     gu.K = d;
     gu.tasks = F;
     gu.out = w.Act;
     gu.ldo = F;
-    if ((s = launch_gemv<dec::kGvSwiglu>(gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvSwiglu>(*di, gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
     // down + residual
     dec::GemvParams dn;
     std::memset(&dn, 0, sizeof(dn));
@@ -970,7 +1006,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     dn.tasks = d / 2;
     dn.out = x;
     dn.ldo = d;
-    if ((s = launch_gemv<dec::kGvResid>(dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
     for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
   }
   g_timing.layer = -1;
@@ -1240,7 +1276,8 @@ dash_status dash_prefill_varlen_kv(const dash_dims* dims, const dash_layer_weigh
 
 size_t dash_decode_attention_workspace_size(int32_t hd) {
   if (hd != 64 && hd != 128) return 0;
-  return static_cast<size_t>(dash::decode::kMaxCtas) * dash::decode::kGroupPad * (hd + 2) * sizeof(float) + 1024;
+  return static_cast<size_t>(dash::decode::kMaxCtas) * dash::decode::kGroupPad * (hd + 2) * sizeof(float) +
+         dash::decode::kMaxSegs * sizeof(int) + 1024;
 }
 
 dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_kv_cache* caches, int32_t hq,
@@ -1275,9 +1312,11 @@ dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_k
   DecodeWs w{};
   w.Q = const_cast<bf16*>(reinterpret_cast<const bf16*>(Q));
   w.O = reinterpret_cast<bf16*>(O);
+  w.counters = c.take<int>(dec::kMaxSegs);
   w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * hd);
   w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
   cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
   return hd == 128 ? decode_attention_hd<128>(*di, D, nseq, len, lc, w, st)
                    : decode_attention_hd<64>(*di, D, nseq, len, lc, w, st);
 }
@@ -1328,8 +1367,7 @@ const char* dash_kernel_name(int32_t kind) {
                                             "attention", "gemm_o_resid_delta", "score", "gemm_gate_up_swiglu",
                                             "gemm_down_resid", "select", "gather", "scatter", "gemm",
                                             "kv_store", "gemv_qkv_rope_append", "decode_attention",
-                                            "decode_combine", "gemv_o_resid", "gemv_gate_up_swiglu",
-                                            "gemv_down_resid"};
+                                            "gemv_o_resid", "gemv_gate_up_swiglu", "gemv_down_resid"};
   return kind >= 0 && kind < DASH_K_COUNT ? names[kind] : "unknown";
 }
 

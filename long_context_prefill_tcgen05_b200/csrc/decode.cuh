@@ -7,15 +7,19 @@
 //
 //   gemv_kernel<kGvQkv>     q/k/v = rmsnorm(x) W_qkv^T, RoPE on q and k, the
 //                           new k/v (and position) appended to each cache
-//   decode_attn_kernel      split-key attention over each cache on tcgen05
-//   decode_combine_kernel   merge of the per-CTA partial softmax results
+//   decode_attn_kernel      split-key attention over each cache on tcgen05; the
+//                           last CTA of each (sequence, kv head) merges the
+//                           partial softmax results
 //   gemv_kernel<kGvResid>   x += o W_o^T
 //   gemv_kernel<kGvSwiglu>  act = silu(rmsnorm(x) W_g^T) * (rmsnorm(x) W_u^T)
 //   gemv_kernel<kGvResid>   x += act W_d^T
 //
 // With n <= 8 rows the projections are HBM-bound on the weights (2 bytes
 // per multiply-add), so they run on the CUDA cores: one warp streams two
-// weight rows with 16-byte loads and keeps n dot products per row.
+// weight rows with 16-byte loads and keeps n dot products per row; one
+// 16-warp CTA per SM takes the row pairs strided over the grid, so the
+// weights spread evenly over the SMs.  Every kernel of the step is launched
+// with programmatic dependent launch (griddepcontrol) to hide launch gaps.
 //
 // The attention is HBM-bound on the cache.  Its query group (hq / hkv <= 16
 // heads) is too small for a tcgen05 M dimension, so the kernel puts the keys
@@ -53,11 +57,13 @@ struct SeqSlots {
 };
 
 struct GemvParams {
-  const __nv_bfloat16* W;   // [rows, K] row-major
-  const __nv_bfloat16* W2;  // kGvSwiglu: up-projection [rows, K]
-  const __nv_bfloat16* x;   // [n, K]
-  const float* xs;          // [n] factor on each dot product (RMSNorm 1/rms) or NULL
+  const __nv_bfloat16* W;     // [rows, K] row-major
+  const __nv_bfloat16* W2;    // kGvSwiglu: up-projection [rows, K]
+  const __nv_bfloat16* x;     // [n, K]
+  const __nv_bfloat16* gain;  // kGvQkv / kGvSwiglu: RMSNorm gain [K] (the norm is fused)
+  float eps;
   int n, K, tasks;
+  int stage_x;                // kGvResid: copy x to shared memory first (it fits)
   __nv_bfloat16* out;  // kGvResid: residual stream [n, ldo] (in/out); kGvSwiglu: act [n, ldo]
   int64_t ldo;
   __nv_bfloat16* q;  // kGvQkv: [n, hq*hd]
@@ -66,7 +72,13 @@ struct GemvParams {
   SeqSlots seq;
 };
 
-constexpr int kGemvWarps = 8;
+constexpr int kGemvWarps = 16;  // one CTA per SM; warps take tasks strided over the grid
+
+// Programmatic dependent launch: let the next kernel of the stream be
+// scheduled now, and wait until the previous one has finished and its
+// writes are visible.  (No-ops for a launch without the PDL attribute.)
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
   float a = bf16_lo(w.x) * bf16_lo(x.x);
@@ -80,110 +92,179 @@ __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
   return a + b;
 }
 
+__device__ __forceinline__ float sumsq8(const uint4& v) {
+  float s = 0.f;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s = fmaf(bf16_lo(w[e]), bf16_lo(w[e]), fmaf(bf16_hi(w[e]), bf16_hi(w[e]), s));
+  return s;
+}
+
+__device__ __forceinline__ uint4 mul8(const uint4& x, const uint4& g) {
+  return make_uint4(pack_bf16(bf16_lo(x.x) * bf16_lo(g.x), bf16_hi(x.x) * bf16_hi(g.x)),
+                    pack_bf16(bf16_lo(x.y) * bf16_lo(g.y), bf16_hi(x.y) * bf16_hi(g.y)),
+                    pack_bf16(bf16_lo(x.z) * bf16_lo(g.z), bf16_hi(x.z) * bf16_hi(g.z)),
+                    pack_bf16(bf16_lo(x.w) * bf16_lo(g.w), bf16_hi(x.w) * bf16_hi(g.w)));
+}
+
 __device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// Each warp owns one task = two weight rows (r0, r1) and all n inputs:
+// Streaming read of weights: not kept in L1, 256-byte L2 fetch granularity.
+__device__ __forceinline__ uint4 ldg_stream(const uint4* ptr) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(ptr));
+  return v;
+}
+
+// Each task = two weight rows (r0, r1) against all n inputs:
 //   kGvQkv     rows (i, i + hd/2) of one q/k/v head: the RoPE pair
 //   kGvSwiglu  row t of W (gate) and row t of W2 (up)
 //   kGvResid   rows (2t, 2t + 1)
+// With the norm fused (kGvQkv, kGvSwiglu) the CTA first computes each
+// input row's 1/rms and stages x * gain as bf16 in shared memory (exact for
+// unit gains); the 1/rms multiplies the finished dot products, as the
+// prefill's GEMM epilogues do.  kGvResid stages x as is when it fits.
 template <int EPI, int NS>
-__global__ void __launch_bounds__(32 * kGemvWarps) gemv_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvParams p) {
+  constexpr bool kNorm = EPI != kGvResid;
+  extern __shared__ uint4 xg_smem[];  // kNorm: [n][K/8]
+  __shared__ float red[kGemvWarps][kMaxSeq];
+  __shared__ float rs_s[kMaxSeq];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int task = blockIdx.x * kGemvWarps + warp;
-  if (task >= p.tasks) return;
-  const int K = p.K;
-  int head = 0, i = 0;
-  const __nv_bfloat16* w0;
-  const __nv_bfloat16* w1;
-  if constexpr (EPI == kGvQkv) {
-    const int half = p.hd >> 1;
-    head = task / half;
-    i = task - head * half;
-    w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
-    w1 = w0 + static_cast<int64_t>(half) * K;
-  } else if constexpr (EPI == kGvSwiglu) {
-    w0 = p.W + static_cast<int64_t>(task) * K;
-    w1 = p.W2 + static_cast<int64_t>(task) * K;
-  } else {
-    w0 = p.W + static_cast<int64_t>(2 * task) * K;
-    w1 = w0 + K;
-  }
-  const uint4* wa = reinterpret_cast<const uint4*>(w0);
-  const uint4* wb = reinterpret_cast<const uint4*>(w1);
-  const uint4* xv = reinterpret_cast<const uint4*>(p.x);
-  const int nv = K >> 3;
-  constexpr int U = NS <= 2 ? 4 : 2;  // 16-byte chunks per row in flight per lane
-  float a0[NS], a1[NS];
+  const int K = p.K, nv = K >> 3;
+  const uint4* xg = reinterpret_cast<const uint4*>(p.x);
+  if constexpr (kNorm) {
+    float ss[NS];
 #pragma unroll
-  for (int m = 0; m < NS; ++m) a0[m] = a1[m] = 0.f;
-  for (int c0 = lane; c0 < nv; c0 += 32 * U) {
-    uint4 ra[U], rb[U];
+    for (int m = 0; m < NS; ++m) ss[m] = 0.f;
+    const uint4* gv = reinterpret_cast<const uint4*>(p.gain);
+    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+      const uint4 g = __ldg(gv + c);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < nv) {
-        ra[u] = __ldcs(wa + c);  // weights stream through once per step
-        rb[u] = __ldcs(wb + c);
-      }
+      for (int m = 0; m < NS; ++m)
+        if (m < p.n) {
+          const uint4 v = __ldg(xg + static_cast<int64_t>(m) * nv + c);
+          ss[m] += sumsq8(v);
+          xg_smem[m * nv + c] = mul8(v, g);
+        }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < nv) {
+    for (int m = 0; m < NS; ++m) {
 #pragma unroll
-        for (int m = 0; m < NS; ++m) {
-          if (m < p.n) {
-            const uint4 xm = __ldg(xv + static_cast<int64_t>(m) * nv + c);
-            a0[m] += dot8(ra[u], xm);
-            a1[m] += dot8(rb[u], xm);
+      for (int o = 16; o > 0; o >>= 1) ss[m] += __shfl_xor_sync(0xffffffffu, ss[m], o);
+      if (lane == 0) red[warp][m] = ss[m];
+    }
+    __syncthreads();
+    if (threadIdx.x < p.n) {
+      float t = 0.f;
+      for (int w = 0; w < kGemvWarps; ++w) t += red[w][threadIdx.x];
+      rs_s[threadIdx.x] = rsqrtf(t / static_cast<float>(K) + p.eps);
+    }
+    __syncthreads();
+    xg = xg_smem;
+  } else if (p.stage_x) {
+    for (int c = threadIdx.x; c < p.n * nv; c += blockDim.x) xg_smem[c] = __ldg(xg + c);
+    __syncthreads();
+    xg = xg_smem;
+  }
+  const bool from_smem = kNorm || p.stage_x;
+  constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
+  const int stride = gridDim.x * kGemvWarps;
+  for (int task = blockIdx.x + gridDim.x * warp; task < p.tasks; task += stride) {
+    int head = 0, i = 0;
+    const __nv_bfloat16* w0;
+    const __nv_bfloat16* w1;
+    if constexpr (EPI == kGvQkv) {
+      const int half = p.hd >> 1;
+      head = task / half;
+      i = task - head * half;
+      w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
+      w1 = w0 + static_cast<int64_t>(half) * K;
+    } else if constexpr (EPI == kGvSwiglu) {
+      w0 = p.W + static_cast<int64_t>(task) * K;
+      w1 = p.W2 + static_cast<int64_t>(task) * K;
+    } else {
+      w0 = p.W + static_cast<int64_t>(2 * task) * K;
+      w1 = w0 + K;
+    }
+    const uint4* wa = reinterpret_cast<const uint4*>(w0);
+    const uint4* wb = reinterpret_cast<const uint4*>(w1);
+    float a0[NS], a1[NS];
+#pragma unroll
+    for (int m = 0; m < NS; ++m) a0[m] = a1[m] = 0.f;
+    for (int c0 = lane; c0 < nv; c0 += 32 * U) {
+      uint4 ra[U], rb[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nv) {
+          ra[u] = ldg_stream(wa + c);  // weights stream through once per step
+          rb[u] = ldg_stream(wb + c);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nv) {
+#pragma unroll
+          for (int m = 0; m < NS; ++m) {
+            if (m < p.n) {
+              const uint4 xm = from_smem ? xg[m * nv + c] : __ldg(xg + static_cast<int64_t>(m) * nv + c);
+              a0[m] += dot8(ra[u], xm);
+              a1[m] += dot8(rb[u], xm);
+            }
           }
         }
       }
     }
-  }
 #pragma unroll
-  for (int m = 0; m < NS; ++m) {
+    for (int m = 0; m < NS; ++m) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      a0[m] += __shfl_xor_sync(0xffffffffu, a0[m], o);
-      a1[m] += __shfl_xor_sync(0xffffffffu, a1[m], o);
+      for (int o = 16; o > 0; o >>= 1) {
+        a0[m] += __shfl_xor_sync(0xffffffffu, a0[m], o);
+        a1[m] += __shfl_xor_sync(0xffffffffu, a1[m], o);
+      }
     }
-  }
-  // Epilogue: lane m finishes input row m.
+    // Epilogue: lane m finishes input row m.
 #pragma unroll
-  for (int m = 0; m < NS; ++m) {
-    if (m >= p.n || lane != m) continue;
-    const float sc = p.xs ? p.xs[m] : 1.f;
-    const float y0 = a0[m] * sc, y1 = a1[m] * sc;
-    if constexpr (EPI == kGvQkv) {
-      const int hd = p.hd, half = hd >> 1;
-      float o0 = y0, o1 = y1;
-      if (head < p.hq + p.hkv) {  // rotate-half RoPE at the token's position (fp64 angle)
-        const double inv = pow(p.theta, -2.0 * i / static_cast<double>(hd));
-        double sn, cs;
-        sincos(static_cast<double>(p.seq.p[m]) * inv, &sn, &cs);
-        const float c = static_cast<float>(cs), s = static_cast<float>(sn);
-        o0 = y0 * c - y1 * s;
-        o1 = y1 * c + y0 * s;
-      }
-      __nv_bfloat16* dst;
-      if (head < p.hq) {
-        dst = p.q + static_cast<int64_t>(m) * p.hq * hd + head * hd;
+    for (int m = 0; m < NS; ++m) {
+      if (m >= p.n || lane != m) continue;
+      const float sc = kNorm ? rs_s[m] : 1.f;
+      const float y0 = a0[m] * sc, y1 = a1[m] * sc;
+      if constexpr (EPI == kGvQkv) {
+        const int hd = p.hd, half = hd >> 1;
+        float o0 = y0, o1 = y1;
+        if (head < p.hq + p.hkv) {  // rotate-half RoPE at the token's position (fp64 angle)
+          const double inv = pow(p.theta, -2.0 * i / static_cast<double>(hd));
+          double sn, cs;
+          sincos(static_cast<double>(p.seq.p[m]) * inv, &sn, &cs);
+          const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+          o0 = y0 * c - y1 * s;
+          o1 = y1 * c + y0 * s;
+        }
+        __nv_bfloat16* dst;
+        if (head < p.hq) {
+          dst = p.q + static_cast<int64_t>(m) * p.hq * hd + head * hd;
+        } else {
+          const int kvd = p.hkv * hd;
+          const bool is_k = head < p.hq + p.hkv;
+          const int h = is_k ? head - p.hq : head - p.hq - p.hkv;
+          dst = (is_k ? p.seq.k[m] : p.seq.v[m]) + p.seq.row[m] * kvd + h * hd;
+          if (head == p.hq && i == 0 && p.seq.pos[m]) p.seq.pos[m][p.seq.row[m]] = p.seq.p[m];
+        }
+        dst[i] = __float2bfloat16_rn(o0);
+        dst[i + half] = __float2bfloat16_rn(o1);
+      } else if constexpr (EPI == kGvSwiglu) {
+        p.out[static_cast<int64_t>(m) * p.ldo + task] = __float2bfloat16_rn(y0 / (1.f + __expf(-y0)) * y1);
       } else {
-        const int kvd = p.hkv * hd;
-        const bool is_k = head < p.hq + p.hkv;
-        const int h = is_k ? head - p.hq : head - p.hq - p.hkv;
-        dst = (is_k ? p.seq.k[m] : p.seq.v[m]) + p.seq.row[m] * kvd + h * hd;
-        if (head == p.hq && i == 0 && p.seq.pos[m]) p.seq.pos[m][p.seq.row[m]] = p.seq.p[m];
+        __nv_bfloat16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
+        const float r0 = bf16_to_f(o[0]) + y0, r1 = bf16_to_f(o[1]) + y1;
+        *reinterpret_cast<uint32_t*>(o) = pack_bf16(r0, r1);
       }
-      dst[i] = __float2bfloat16_rn(o0);
-      dst[i + half] = __float2bfloat16_rn(o1);
-    } else if constexpr (EPI == kGvSwiglu) {
-      p.out[static_cast<int64_t>(m) * p.ldo + task] = __float2bfloat16_rn(y0 / (1.f + __expf(-y0)) * y1);
-    } else {
-      __nv_bfloat16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
-      const float r0 = bf16_to_f(o[0]) + y0, r1 = bf16_to_f(o[1]) + y1;
-      *reinterpret_cast<uint32_t*>(o) = pack_bf16(r0, r1);
     }
   }
 }
@@ -191,8 +272,11 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_kernel(const GemvParams 
 // ========================================================= decode attention
 struct AttnParams {
   const __nv_bfloat16* q;  // [n, hq*HD], RoPE applied
-  float* part_o;           // [kMaxCtas, 16, HD]: unnormalised O of each CTA
-  float* part_ml;          // [kMaxCtas, 16, 2]: (running max in log2 units, sum)
+  __nv_bfloat16* out;      // [n, hq*HD]
+  float* part_o;           // [CTA c][g < group][HD]: unnormalised O of each CTA (a segment's CTAs adjacent)
+  float* part_ml;          // [CTA c][16][2]: (running max in log2 units, sum); 128 bytes per CTA, so
+                           // a segment's block starts 16-byte aligned for the bulk copy
+  int* counters;           // [kMaxSegs] finished CTAs per segment (zero before the launch; left zero)
   int n, hq, hkv, group, tiles_per_cta;
   int len[kMaxSeq];                // keys of each sequence (cache rows incl. the new one)
   int seg_cta0[kMaxSegs + 1];      // first CTA of segment s * hkv + h; [nseg] = CTA count
@@ -215,11 +299,11 @@ struct ACfg {
   static constexpr int kOffZero = 2 * kStages * kTile;
   static constexpr int kZeroBytes = HD == 64 ? BKV * 128 : 0;
   static constexpr int kOffQ = kOffZero + kZeroBytes;   // [16, HD] K-major, kPanels x 2 KB
-  static constexpr int kOffP = kOffQ + kPanels * 2048;  // [16, 128 keys] K-major, 2 x 2 KB
-  static constexpr int kOffRed = kOffP + 4096;          // [2][4 warps][16] floats
+  static constexpr int kOffP = kOffQ + kPanels * 2048;  // 2 buffers of [16, 128 keys] K-major, 2 x 2 KB each
+  static constexpr int kOffRed = kOffP + 2 * 4096;      // [2][4 warps][16] floats
   static constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 4;
-  // full[kStages], empty[kStages], q_ready, s_full[2], p_full, pv_done, red[2], drain
-  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 1 + 1 + 2 + 1;
+  // full[kStages], empty[kStages], q_ready, s_full[2], p_full[2], pv_done[2], red[2], drain, pub, merge
+  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
   static constexpr uint32_t kTmemCols = 64;  // S^T buffers [0,16) [16,32), O^T [32,48)
 };
@@ -253,6 +337,107 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int panel_byt
   return pn * panel_bytes + row * 128 + ((((cc >> 3) ^ (row & 7)) & 7) << 4) + ((cc & 7) << 1);
 }
 
+
+// Bulk async copy global -> shared (no tensor map), completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Merge of one (sequence, kv head) segment's partial results by all threads
+// of its last CTA (after the CTA's final barrier; the K/V stages are free):
+//   M_g = max_c m_cg,  w_cg = 2^(m_cg - M_g) / sum_c' 2^(m_c'g - M_g) l_c'g,
+//   O_g = sum_c w_cg o_cg.
+// A segment's partial results are adjacent in memory, so they come into
+// shared memory by a few large bulk async copies (one L2 round trip each).
+template <int HD>
+__device__ void merge_segment(const AttnParams& p, int seg, int s, int kvh, uint8_t* scratch, int scratch_bytes,
+                              uint32_t bar) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int G = p.group;
+  const int c0 = p.seg_cta0[seg], nch = p.seg_cta0[seg + 1] - c0;
+  float2* ml = reinterpret_cast<float2*>(scratch);                         // [nch][16] (m, l)
+  float* wt = reinterpret_cast<float*>(scratch + kMaxCtas * kGroupPad * 8);  // [nch][G] weights
+  float* os = wt + kMaxCtas * kGroupPad;                                    // [chunk][G][HD]
+  const int row_bytes = G * HD * 4;
+  const int chunk = (scratch_bytes - kMaxCtas * kGroupPad * 12) / row_bytes;
+  const float* po = p.part_o + static_cast<int64_t>(c0) * G * HD;
+  uint32_t phase = 0;
+  if (t == 0) {
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");  // other CTAs' partials -> the async proxy
+    const uint32_t ml_bytes = nch * kGroupPad * 8;  // source offset c0 * 128 bytes: 16-byte aligned
+    const int cn = min(chunk, nch);
+    mbar_arrive_expect_tx(bar, ml_bytes + cn * row_bytes);
+    bulk_load(smem_u32(ml), p.part_ml + static_cast<int64_t>(c0) * kGroupPad * 2, ml_bytes, bar);
+    bulk_load(smem_u32(os), po, cn * row_bytes, bar);
+  }
+  constexpr int kOut4 = kGroupPad * HD / 4;
+  constexpr int kMaxOut = (kOut4 + kAttnThreads - 1) / kAttnThreads;
+  float4 acc[kMaxOut];
+#pragma unroll
+  for (int j = 0; j < kMaxOut; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int n4 = G * HD / 4;
+  for (int cs = 0; cs < nch; cs += chunk) {
+    const int cn = min(chunk, nch - cs);
+    if (cs > 0) {
+      __syncthreads();  // previous chunk consumed
+      if (t == 0) {
+        mbar_arrive_expect_tx(bar, cn * row_bytes);
+        bulk_load(smem_u32(os), po + static_cast<int64_t>(cs) * G * HD, cn * row_bytes, bar);
+      }
+    }
+    mbar_wait(bar, phase);
+    phase ^= 1u;
+    if (cs == 0) {
+      for (int g = warp; g < G; g += kAttnThreads / 32) {
+        float M = -INFINITY;
+        for (int c = lane; c < nch; c += 32) M = fmaxf(M, ml[c * kGroupPad + g].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int c = lane; c < nch; c += 32) L = fmaf(ex2f(ml[c * kGroupPad + g].x - M), ml[c * kGroupPad + g].y, L);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float inv = 1.f / L;
+        for (int c = lane; c < nch; c += 32) wt[c * G + g] = ex2f(ml[c * kGroupPad + g].x - M) * inv;
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxOut; ++j) {
+      const int i = t + j * kAttnThreads;  // float4 output: head g, dimensions 4 * (i % (HD/4))
+      if (i < n4) {
+        const int g = i / (HD / 4);
+        float4 a = acc[j];
+        const float4* src = reinterpret_cast<const float4*>(os) + i;
+#pragma unroll 4
+        for (int c = 0; c < cn; ++c) {
+          const float w = wt[(cs + c) * G + g];
+          const float4 o = src[c * n4];
+          a.x = fmaf(w, o.x, a.x);
+          a.y = fmaf(w, o.y, a.y);
+          a.z = fmaf(w, o.z, a.z);
+          a.w = fmaf(w, o.w, a.w);
+        }
+        acc[j] = a;
+      }
+    }
+  }
+  __nv_bfloat16* dst = p.out + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
+#pragma unroll
+  for (int j = 0; j < kMaxOut; ++j) {
+    const int i = t + j * kAttnThreads;
+    if (i < n4) {
+      uint2 v;
+      v.x = pack_bf16(acc[j].x, acc[j].y);
+      v.y = pack_bf16(acc[j].z, acc[j].w);
+      *reinterpret_cast<uint2*>(dst + 4 * i) = v;
+    }
+  }
+}
+
 // One CTA = a run of up to tiles_per_cta key tiles of one (sequence, kv head)
 // segment.  Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.
 // Warps 2..5: Q staging, softmax (lane r = key r of the tile), and the
@@ -264,6 +449,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  pdl_trigger();
+  pdl_wait();  // q and the appended cache row come from the previous kernel
   const int b = blockIdx.x;
   const int nseg = p.n * p.hkv;
   int seg = 0;
@@ -279,12 +466,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_empty = smem_u32(bars + kStages);
   const uint32_t bar_q = smem_u32(bars + 2 * kStages);
-  const uint32_t bar_sfull = bar_q + 8;   // [2]
-  const uint32_t bar_pfull = bar_q + 24;
-  const uint32_t bar_pvdone = bar_q + 32;
-  const uint32_t bar_red = bar_q + 40;    // [2]
-  const uint32_t bar_drain = bar_q + 56;
+  const uint32_t bar_sfull = bar_q + 8;    // [2] S^T buffer b holds tile i (i & 1 == b)
+  const uint32_t bar_pfull = bar_q + 24;   // [2] P^T buffer b written for tile i
+  const uint32_t bar_pvdone = bar_q + 40;  // [2] P^T(i) V(i) finished, buffer i & 1 free
+  const uint32_t bar_red = bar_q + 56;     // [2]
+  const uint32_t bar_drain = bar_q + 72;
+  const uint32_t bar_pub = bar_q + 80;    // 128 epilogue threads published their partials
+  const uint32_t bar_merge = bar_q + 88;  // bulk copies of the merge
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  int* ticket = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -296,10 +486,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar_sfull, 1);
     mbar_init(bar_sfull + 8, 1);
     mbar_init(bar_pfull, 128);
+    mbar_init(bar_pfull + 8, 128);
     mbar_init(bar_pvdone, 1);
+    mbar_init(bar_pvdone + 8, 1);
     mbar_init(bar_red, 128);
     mbar_init(bar_red + 8, 128);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_pub, 128);
+    mbar_init(bar_merge, 1);
+    *ticket = 0;
     fence_mbar_init();
   }
   if (HD == 64) {  // zero panel read as the upper half of V^T
@@ -368,7 +563,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       return true;
     };
     auto issue_pv = [&](int i) {  // O^T += V_i^T P_i^T
-      if (!mbar_wait(bar_pfull, i & 1)) return false;
+      if (!mbar_wait(bar_pfull + 8 * (i & 1), (i >> 1) & 1)) return false;
       tc_fence_after();
       if (lane == 0) {
         const int st = i % kStages;
@@ -378,9 +573,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint32_t ob = (kk >> 2) * 2048 + (kk & 3) * 32;
           umma_bf16_ss(tmem_base + 2 * kGroupPad, umma_desc_sw128(sv + kk * 16 * 128, lbo, 1024),
-                       umma_desc_sw128(sp + ob, 16, 1024), idesc_o, (i != 0 || kk != 0) ? 1u : 0u);
+                       umma_desc_sw128(sp + (i & 1) * 4096 + ob, 16, 1024), idesc_o,
+                       (i != 0 || kk != 0) ? 1u : 0u);
         }
-        umma_commit(bar_pvdone);
+        umma_commit(bar_pvdone + 8 * (i & 1));
         umma_commit(bar_empty + 8 * st);
       }
       __syncwarp();
@@ -482,12 +678,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_part[g] += e;
         pb[g] = *reinterpret_cast<const uint16_t*>(&eb);
       }
-      // P^T buffer and O^T are free once P_(i-1) V_(i-1) is done.
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone, (i - 1) & 1));
+      // P^T buffer i & 1 is free once P_(i-2) V_(i-2) is done; a rescale of
+      // O^T also needs P_(i-1) V_(i-1) done.  (Each pv_done barrier is at
+      // most one completion ahead of these waits.)
+      if (i >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + 8 * (i & 1), ((i >> 1) - 1) & 1));
         if (!ok) break;
-        tc_fence_after();
       }
+      if (rescale) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1));
+        if (!ok) break;
+      }
+      tc_fence_after();
       if (rescale) {
         uint32_t o[kGroupPad];
         tmem_ld16(tmem_base + lane_off + 2 * kGroupPad, o);
@@ -499,12 +701,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
 #pragma unroll
       for (int g = 0; g < kGroupPad; ++g)
-        *reinterpret_cast<uint16_t*>(smem + C::kOffP + sw128_offset(g, r, 2048)) = pb[g];
+        *reinterpret_cast<uint16_t*>(smem + C::kOffP + (i & 1) * 4096 + sw128_offset(g, r, 2048)) = pb[g];
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar_pfull);
+      mbar_arrive(bar_pfull + 8 * (i & 1));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone, (nt - 1) & 1));
+    // MMAs complete in order: PV(nt-1) done means all are.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + 8 * ((nt - 1) & 1), ((nt - 1) >> 1) & 1));
     if (ok) {
       tc_fence_after();
       uint32_t o[kGroupPad];
@@ -525,7 +728,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(bar_red + 8 * (nt & 1));
       ok = __all_sync(0xffffffffu, mbar_wait(bar_red + 8 * (nt & 1), (nt >> 1) & 1));
       if (ok) {
-        float* po = p.part_o + static_cast<int64_t>(b) * kGroupPad * HD;
+        float* po = p.part_o + static_cast<int64_t>(b) * G * HD;
         if (r < HD)
 #pragma unroll
           for (int g = 0; g < kGroupPad; ++g)
@@ -542,6 +745,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pm[0] = mr;
           pm[1] = lr;
         }
+        // The last CTA of the segment to finish merges every CTA's partial
+        // result, after the CTA's final barrier.
+        // (The fence of the counting thread, after it has seen every
+        // thread's stores through the mbarrier, orders them before its atomic.)
+        mbar_arrive(bar_pub);
+        if (r == 0) {
+          const int c0 = p.seg_cta0[seg], c1 = p.seg_cta0[seg + 1];
+          if (mbar_wait(bar_pub, 0)) {
+            __threadfence();
+            *ticket = atomicAdd(&p.counters[seg], 1) == c1 - c0 - 1 ? 1 : 0;
+          }
+        }
       }
     }
   }
@@ -551,27 +766,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-}
-
-// O[s, head, :] = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c over the CTAs c
-// of the head's segment (M = max m_c).  One block of HD threads per (s, head).
-template <int HD>
-__global__ void decode_combine_kernel(const AttnParams p, __nv_bfloat16* __restrict__ out) {
-  const int s = blockIdx.x / p.hq, head = blockIdx.x - s * p.hq;
-  const int kvh = head / p.group, g = head - kvh * p.group;
-  const int seg = s * p.hkv + kvh;
-  const int c0 = p.seg_cta0[seg], c1 = p.seg_cta0[seg + 1];
-  const int d = threadIdx.x;
-  float M = -INFINITY;
-  for (int c = c0; c < c1; ++c) M = fmaxf(M, p.part_ml[(static_cast<int64_t>(c) * kGroupPad + g) * 2]);
-  float l = 0.f, acc = 0.f;
-  for (int c = c0; c < c1; ++c) {
-    const float* ml = p.part_ml + (static_cast<int64_t>(c) * kGroupPad + g) * 2;
-    const float w = ex2f(ml[0] - M);
-    l = fmaf(w, ml[1], l);
-    acc = fmaf(w, p.part_o[(static_cast<int64_t>(c) * kGroupPad + g) * HD + d], acc);
+  if (*ticket == 1) {  // uniform: written before the barrier above
+    merge_segment<HD>(p, seg, s, kvh, smem + C::kOffK, C::kOffZero - C::kOffK, bar_merge);
+    if (threadIdx.x == 0) p.counters[seg] = 0;  // ready for the next launch
   }
-  out[static_cast<int64_t>(s) * p.hq * HD + head * HD + d] = __float2bfloat16_rn(acc / l);
 }
 
 // ============================================================ cache store

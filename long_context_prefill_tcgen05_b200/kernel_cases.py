@@ -5,6 +5,8 @@ for ncu captures of a single kernel on a small case).
     python -m long_context_prefill_tcgen05_b200.kernel_cases linear --M 4096 --N 37888 --K 3584
     python -m long_context_prefill_tcgen05_b200.kernel_cases layer --T 4096
     python -m long_context_prefill_tcgen05_b200.kernel_cases select --T 32768
+    python -m long_context_prefill_tcgen05_b200.kernel_cases decode --T 32768 --M 1
+    python -m long_context_prefill_tcgen05_b200.kernel_cases decode_attention --T 32768 --M 1
 
 Shapes default to the Qwen2.5-7B-shaped stack (28 q / 4 kv heads, hd 128,
 d 3584, FFN 18944).  Prints one JSON line with the mean CUDA-event time.
@@ -32,7 +34,8 @@ def _time(fn, iters, warmup):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attention", "linear", "layer", "select", "score", "gather"])
+    ap.add_argument("case", choices=["attention", "linear", "layer", "select", "score", "gather", "decode",
+                                     "decode_attention"])
     ap.add_argument("--T", type=int, default=8192)
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=37888)
@@ -84,6 +87,34 @@ def main():
         idx = torch.sort(torch.randperm(args.T, generator=g, device=dev)[:args.T // 2]).values.int()
         ms = _time(lambda: dash.compact(X, idx), args.iters, args.warmup)
         out.update(T=args.T, ms=ms, gbs=2 * (args.T // 2) * dims.d_model * 2 / ms / 1e6)
+    elif args.case in ("decode", "decode_attention"):
+        # one generation step of a one-layer stack (or its attention alone) for
+        # M sequences, each with a cache of T random rows
+        n, T = args.M, args.T
+        hq, hkv, hd = dims.n_heads, dims.n_kv_heads, dims.head_dim
+        stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev, n_layers=1))
+        cap = T + args.iters + args.warmup + 1
+        cache = dash.KVCache(stack, n, cap, device=dev)
+        for i in range(n):
+            cache.k[i][:T] = rnd(T, hkv * hd)
+            cache.v[i][:T] = rnd(T, hkv * hd)
+            cache.desc[i].len = T
+        if args.case == "decode":
+            X = rnd(n, dims.d_model)
+            step = [T]
+
+            def run():
+                dash.decode_step(stack, X, [step[0]] * n, cache)
+                step[0] += 1
+            ms = _time(run, args.iters, args.warmup)
+            by = costs.layer_weight_bytes(dims) + n * (T + 1) * hkv * hd * 2 * 2
+        else:
+            Q = rnd(n, hq * hd)
+            O = torch.empty_like(Q)
+            kv = [(cache.k[i][:T], cache.v[i][:T]) for i in range(n)]
+            ms = _time(lambda: dash.decode_attention(Q, kv, hq, hkv, hd, out=O), args.iters, args.warmup)
+            by = n * T * hkv * hd * 2 * 2
+        out.update(T=T, n=n, ms=ms, gbs=by / ms / 1e6)
     dash.check_device()
     print(json.dumps(out), flush=True)
 
