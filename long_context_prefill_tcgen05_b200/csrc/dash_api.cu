@@ -1,6 +1,7 @@
 // C ABI of libdash (declared in include/dash.h and include/dash_ops.h):
 // argument checks, workspace carving, tensor-map encoding, kernel launches,
 // and the host-side layer loop of the single-shot DASH prefill.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -839,7 +840,8 @@ dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kin
 // tiles_per_cta key tiles of one (sequence, kv head) segment.
 template <int HD>
 dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n, const int64_t* len,
-                                const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st) {
+                                const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st,
+                                const dec::Prefetch* next = nullptr) {
   using C = dec::ACfg<HD>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -896,6 +898,7 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   ap.group = D.n_heads / hkv;
   ap.tiles_per_cta = static_cast<int>(per);
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
+  if (next) ap.next = *next;
   TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, nctas, st);
   if (launch_pdl(dec::decode_attn_kernel<HD>, static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st,
                  maps, ap) != cudaSuccess)
@@ -966,10 +969,21 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     qkv.hkv = hkv;
     qkv.hd = hd;
     qkv.theta = D.rope_theta;
+    for (int q = 0; q < n; ++q) {  // the attention streams this layer's cache next
+      const uint64_t bytes = static_cast<uint64_t>(lc[q]->len) * hkv * hd * 2;
+      qkv.next.ptr[qkv.next.count] = reinterpret_cast<const uint8_t*>(lc[q]->k);
+      qkv.next.bytes[qkv.next.count++] = bytes;
+      qkv.next.ptr[qkv.next.count] = reinterpret_cast<const uint8_t*>(lc[q]->v);
+      qkv.next.bytes[qkv.next.count++] = bytes;
+    }
     if ((s = launch_gemv<dec::kGvQkv>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
     // attention over each sequence's cache (including the new row)
-    s = hd == 128 ? decode_attention_hd<128>(*di, D, n, len, lc, w, st)
-                  : decode_attention_hd<64>(*di, D, n, len, lc, w, st);
+    dec::Prefetch wo{};  // o_proj streams W_o next
+    wo.ptr[0] = reinterpret_cast<const uint8_t*>(lw.w_o);
+    wo.bytes[0] = static_cast<uint64_t>(d) * qd * 2;
+    wo.count = 1;
+    s = hd == 128 ? decode_attention_hd<128>(*di, D, n, len, lc, w, st, &wo)
+                  : decode_attention_hd<64>(*di, D, n, len, lc, w, st, &wo);
     if (s != DASH_OK) break;
     // o_proj + residual
     dec::GemvParams o;
@@ -981,6 +995,14 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     o.tasks = d / 2;
     o.out = x;
     o.ldo = d;
+    {  // gate/up's first round of rows (every warp of the grid takes one task)
+      const int64_t first = std::min<int64_t>(F, static_cast<int64_t>(di->num_sms) * dec::kGemvWarps);
+      o.next.ptr[0] = reinterpret_cast<const uint8_t*>(lw.w_gate);
+      o.next.bytes[0] = static_cast<uint64_t>(first) * d * 2;
+      o.next.ptr[1] = reinterpret_cast<const uint8_t*>(lw.w_up);
+      o.next.bytes[1] = static_cast<uint64_t>(first) * d * 2;
+      o.next.count = 2;
+    }
     if ((s = launch_gemv<dec::kGvResid>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
     // RMSNorm (fused) -> gate/up with SwiGLU
     dec::GemvParams gu;
@@ -1006,6 +1028,11 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     dn.tasks = d / 2;
     dn.out = x;
     dn.ldo = d;
+    if (l + 1 < D.n_layers) {  // the next layer's QKV weights
+      dn.next.ptr[0] = reinterpret_cast<const uint8_t*>(layers[l + 1].w_qkv);
+      dn.next.bytes[0] = static_cast<uint64_t>(qd + 2 * hkv * hd) * d * 2;
+      dn.next.count = 1;
+    }
     if ((s = launch_gemv<dec::kGvResid>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
     for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
   }

@@ -45,6 +45,37 @@ constexpr int kStages = 3;
 constexpr int kAttnThreads = 192;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units, as in the prefill softmax
 
+// ========================================================= L2 prefetch
+// Regions the NEXT kernel of the step will stream (its weights or the
+// cache), fetched into L2 by the TMA engine while this kernel runs: the
+// kernels of a decode step alternate between latency-bound phases (launch,
+// prologue, merge) and bandwidth-bound streaming, so the prefetch fills the
+// former with the latter's bytes.
+constexpr int kMaxPrefetch = 2 * kMaxSeq;
+struct Prefetch {
+  const uint8_t* ptr[kMaxPrefetch];
+  uint64_t bytes[kMaxPrefetch];
+  int count;
+};
+
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(ptr)), "r"(bytes)
+               : "memory");
+}
+
+// Thread 0 of every CTA prefetches its share of each region (16-byte
+// aligned starts and sizes; a region's last partial 16 bytes are skipped).
+__device__ __forceinline__ void prefetch_share(const Prefetch& pf) {
+  if (threadIdx.x != 0) return;
+  for (int r = 0; r < pf.count; ++r) {
+    const uint64_t total = pf.bytes[r] & ~15ull;
+    const uint64_t per = ((total + gridDim.x - 1) / gridDim.x + 15) & ~15ull;
+    uint64_t a = per * blockIdx.x;
+    const uint64_t e = a + per < total ? a + per : total;
+    for (; a < e; a += 65536) prefetch_l2(pf.ptr[r] + a, static_cast<uint32_t>(e - a < 65536 ? e - a : 65536));
+  }
+}
+
 // =================================================================== GEMV
 enum GemvEpi : int { kGvQkv = 0, kGvResid = 1, kGvSwiglu = 2 };
 
@@ -70,6 +101,7 @@ struct GemvParams {
   int hq, hkv, hd;
   double theta;
   SeqSlots seq;
+  Prefetch next;  // what the next kernel streams
 };
 
 constexpr int kGemvWarps = 16;  // one CTA per SM; warps take tasks strided over the grid
@@ -133,6 +165,7 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
   __shared__ float red[kGemvWarps][kMaxSeq];
   __shared__ float rs_s[kMaxSeq];
   pdl_trigger();
+  prefetch_share(p.next);  // independent of the previous kernel
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = p.K, nv = K >> 3;
@@ -174,14 +207,11 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
   const bool from_smem = kNorm || p.stage_x;
   constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
   const int stride = gridDim.x * kGemvWarps;
-  for (int task = blockIdx.x + gridDim.x * warp; task < p.tasks; task += stride) {
-    int head = 0, i = 0;
-    const __nv_bfloat16* w0;
-    const __nv_bfloat16* w1;
+  // the two weight rows of a task
+  auto rows = [&](int task, const __nv_bfloat16*& w0, const __nv_bfloat16*& w1) {
     if constexpr (EPI == kGvQkv) {
       const int half = p.hd >> 1;
-      head = task / half;
-      i = task - head * half;
+      const int head = task / half, i = task - head * half;
       w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
       w1 = w0 + static_cast<int64_t>(half) * K;
     } else if constexpr (EPI == kGvSwiglu) {
@@ -190,6 +220,28 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
     } else {
       w0 = p.W + static_cast<int64_t>(2 * task) * K;
       w1 = w0 + K;
+    }
+  };
+  for (int task = blockIdx.x + gridDim.x * warp; task < p.tasks; task += stride) {
+    int head = 0, i = 0;
+    if constexpr (EPI == kGvQkv) {
+      head = task / (p.hd >> 1);
+      i = task - head * (p.hd >> 1);
+    }
+    const __nv_bfloat16* w0;
+    const __nv_bfloat16* w1;
+    rows(task, w0, w1);
+    // The next task's rows go to L2 while this one streams.  (Prefetching the
+    // current task's rows as well measured slower: the demand loads race
+    // their own prefetch.)
+    if (lane == 0) {
+      if (task + stride < p.tasks) {
+        const __nv_bfloat16* n0;
+        const __nv_bfloat16* n1;
+        rows(task + stride, n0, n1);
+        prefetch_l2(n0, K * 2);
+        prefetch_l2(n1, K * 2);
+      }
     }
     const uint4* wa = reinterpret_cast<const uint4*>(w0);
     const uint4* wb = reinterpret_cast<const uint4*>(w1);
@@ -281,6 +333,7 @@ struct AttnParams {
   int len[kMaxSeq];                // keys of each sequence (cache rows incl. the new one)
   int seg_cta0[kMaxSegs + 1];      // first CTA of segment s * hkv + h; [nseg] = CTA count
   float scale_log2;                // log2(e) / sqrt(HD)
+  Prefetch next;                   // what the next kernel streams
 };
 
 struct AttnMaps {
@@ -450,6 +503,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   pdl_trigger();
+  prefetch_share(p.next);
   pdl_wait();  // q and the appended cache row come from the previous kernel
   const int b = blockIdx.x;
   const int nseg = p.n * p.hkv;
