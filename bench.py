@@ -233,15 +233,18 @@ def run_reference(args, world, rank):
 
 
 # --------------------------------------------------------------- decode
-def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, steps=16, warmup=3):
+def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, block=8, rounds=5, warmup=3):
     """Generation after the prefill: ms per step (one new token per sequence)
     on the cache a DASH prefill leaves (prune mode: later layers hold the
-    active tokens only) against the dense prefill's cache."""
+    active tokens only) against the dense prefill's cache.  Both caches are
+    resident; timed blocks of `block` steps alternate between them and the
+    median block is reported."""
     nseq = len(cu) - 1 if cu else 1
     T_max = max(b - a for a, b in zip(cu[:-1], cu[1:])) if cu else h0.shape[0]
-    total = warmup + 2 * steps  # warm-up, a plain timed run, a run with per-kernel events
+    total = warmup + rounds * block + block  # + one block with per-kernel events
     g = torch.Generator(device=dev).manual_seed(99)
-    out = {}
+    starts = [cu[s + 1] - cu[s] for s in range(nseq)] if cu else [h0.shape[0]]
+    legs = {}
     for name, c in (("dash_cache", cfg_cache), ("dense_cache", cfg_dense)):
         cache = dash.KVCache(stack, nseq, T_max + total, device=dev)
         H = h0.clone()
@@ -250,24 +253,34 @@ def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, 
         else:
             dash.prefill_kv(stack, H, c, cache)
         del H
-        starts = [cu[s + 1] - cu[s] for s in range(nseq)] if cu else [h0.shape[0]]
         xs = torch.randn(total, nseq, dims.d_model, generator=g, device=dev).to(torch.bfloat16)
-        for j in range(warmup):
-            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
-        torch.cuda.synchronize()
-        base = [cache.lens(s) for s in range(nseq)]  # rows per layer before the timed steps
-        step_bytes = sum(costs.decode_step_bytes(dims, [[b + 1 + j for b in base[s]] for s in range(nseq)])
-                         for j in range(steps)) / steps
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for j in range(warmup, warmup + steps):
-            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / steps
+        legs[name] = {"cache": cache, "xs": xs, "j": 0, "ms": [], "rows": cache.lens(0)}
+
+    def run(leg, k):
+        for _ in range(k):
+            j = leg["j"]
+            dash.decode_step(stack, leg["xs"][j], [p + j for p in starts], leg["cache"])
+            leg["j"] += 1
+
+    for leg in legs.values():
+        run(leg, warmup)
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for leg in legs.values():
+            base = [leg["cache"].lens(s) for s in range(nseq)]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run(leg, block)
+            e1.record()
+            torch.cuda.synchronize()
+            leg["ms"].append(e0.elapsed_time(e1) / block)
+            leg.setdefault("bytes", []).append(sum(
+                costs.decode_step_bytes(dims, [[b + 1 + j for b in base[s]] for s in range(nseq)])
+                for j in range(block)) / block)
+    out = {}
+    for name, leg in legs.items():
         dash.timing_start()
-        for j in range(warmup + steps, total):
-            dash.decode_step(stack, xs[j], [p + j for p in starts], cache)
+        run(leg, block)
         torch.cuda.synchronize()
         recs = dash.timing_stop()
         per = {}
@@ -279,22 +292,24 @@ def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, 
             q["launches"] += 1
         dom = max(per, key=lambda k: per[k]["ms"])
         gbs = per[dom]["bytes"] / (per[dom]["ms"] / 1e3) / 1e9
-        out[name] = {"ms_per_step": ms, "tokens_per_s": nseq / (ms / 1e3),
-                     "cached_rows_per_layer": cache.lens(0),
+        ms = statistics.median(leg["ms"])
+        step_bytes = statistics.median(leg["bytes"])
+        out[name] = {"ms_per_step": ms, "ms_blocks": leg["ms"], "tokens_per_s": nseq / (ms / 1e3),
+                     "cached_rows_per_layer": leg["rows"],
                      "step_gb": step_bytes / 1e9, "step_gbs": step_bytes / (ms / 1e3) / 1e9,
                      "step_frac_of_hbm": step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                     "gpu_launches_per_step": len(recs) // steps,
-                     "kernels": {k: {"ms_per_step": v["ms"] / steps, "launches_per_step": v["launches"] // steps,
+                     "gpu_launches_per_step": len(recs) // block,
+                     "kernels": {k: {"ms_per_step": v["ms"] / block, "launches_per_step": v["launches"] // block,
                                      "gbs": v["bytes"] / (v["ms"] / 1e3) / 1e9 if v["ms"] else 0.0}
                                  for k, v in sorted(per.items(), key=lambda kv: -kv[1]["ms"])},
                      "roofline": {"bound": "hbm", "kernel": dom, "achieved": gbs, "peak": peaks["hbm_gbs"],
-                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}}
-        del cache, xs
-        torch.cuda.empty_cache()
+                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                  "note": "per-kernel times from CUDA events around each launch"}}
+    del legs
+    torch.cuda.empty_cache()
     out["speedup_vs_dense_cache"] = out["dense_cache"]["ms_per_step"] / out["dash_cache"]["ms_per_step"]
     out["sequences"] = nseq
-    out["steps"] = steps
-    out["warmup"] = warmup
+    out["timing"] = f"median of {rounds} blocks of {block} steps per cache, blocks alternating, after {warmup} warm-up steps"
     return out
 
 
