@@ -224,19 +224,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- MMA
     const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
     const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
-    const uint32_t sq = smem_u32(smem + C::kOffQ);
+    // Descriptors are built once and advanced by adding (byte offset >> 4) to
+    // the start-address field: building them inline per instruction left the
+    // tensor pipe waiting on this thread.
+    const uint64_t qdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+    const uint64_t kdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+    const uint64_t vdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffV), BKV * 128, 1024);
+    // a wait with an inline first try (the barrier is usually ready)
+    auto wait = [](uint32_t bar, uint32_t par) { return mbar_try_wait(bar, par) || mbar_wait(bar, par); };
     auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
       const int ks = (j - j0) % kKStages;
-      if (!mbar_wait(bar_kfull + 8 * ks, ((j - j0) / kKStages) & 1)) return false;
+      if (!wait(bar_kfull + 8 * ks, ((j - j0) / kKStages) & 1)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
-        const uint32_t qa = sq + t * C::kTileBytes;
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>((ks * C::kTileBytes) >> 4);
+        const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_bf16_ss(tmem_base + t * BKV, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(sk + off, 16, 1024),
-                       idesc_s, kk != 0 ? 1u : 0u);
+          constexpr int kPanelStep = (BQ * 128) >> 4;
+          const int off = (kk >> 2) * kPanelStep + (kk & 3) * 2;  // (panel, 32-byte column step) >> 4
+          umma_bf16_ss(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(bar_sfull + 8 * t);
       }
@@ -245,16 +252,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j  (P from TMEM)
       const int vs = (j - j0) % kVStages;
-      if (!mbar_wait(bar_pfull + 8 * t, (j - jb_t[t]) & 1)) return false;
-      if (!mbar_wait(bar_vfull + 8 * vs, ((j - j0) / kVStages) & 1)) return false;
+      if (!wait(bar_pfull + 8 * t, (j - jb_t[t]) & 1)) return false;
+      if (!wait(bar_vfull + 8 * vs, ((j - j0) / kVStages) & 1)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t sv = smem_u32(smem + C::kOffV + vs * C::kTileBytes);
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * C::kTileBytes) >> 4);
         const uint32_t pa = tmem_base + t * BKV + BKV / 2;
+        const uint32_t acc0 = j != jb_t[t] ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, umma_desc_sw128(sv + kk * 16 * 128, BKV * 128, 1024),
-                       idesc_o, (j != jb_t[t] || kk != 0) ? 1u : 0u);
+        for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
+          umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, vd + kk * ((16 * 128) >> 4), idesc_o,
+                       kk != 0 ? 1u : acc0);
         umma_commit(bar_odone + 8 * t);
       }
       __syncwarp();

@@ -304,6 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     const uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
+    // Descriptors differ only in their start-address field (bytes >> 4), so
+    // they are advanced by integer adds: building each one inline in the
+    // issue loop left the tensor pipe waiting on the issuing thread.
+    const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
+    const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
     int stage = 0, local = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -317,20 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(full0 + 8 * stage, phase)) {
+        if (!mbar_try_wait(full0 + 8 * stage, phase) && !mbar_wait(full0 + 8 * stage, phase)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-          const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+          const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = umma_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)  // 16 columns = 32 bytes along the 128-byte swizzle row
+            umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(empty0 + 8 * stage);
         }
         __syncwarp();
