@@ -9,6 +9,9 @@ import csv
 import sys
 
 SHORT = [
+    ("decode_attn_kernel", "decode_attention"),
+    ("gemv_kernel<0", "gemv_qkv_rope_append"), ("gemv_kernel<1", "gemv_resid (o_proj / down)"),
+    ("gemv_kernel<2", "gemv_gate_up_swiglu"), ("kv_store_kernel", "kv_store"),
     ("attn_kernel", "attention"),
     ("gemm_kernel<256, 4>", "gemm_qkv_rope"), ("gemm_kernel<128, 4>", "gemm_qkv_rope"),
     ("gemm_kernel<256, 2>", "gemm_o_resid_delta"), ("gemm_kernel<128, 2>", "gemm_o_resid_delta"),
