@@ -356,6 +356,11 @@ def main():
     H = torch.empty_like(h0)
     idx = torch.empty(T, dtype=torch.int32, device=dev)
     delta = torch.empty(T, dtype=torch.float32, device=dev)
+    def run(c):
+        if varlen:
+            return dash.prefill_varlen(stack, H, cu, c, idx_out=idx, delta_out=delta)[0]
+        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
+
     threshold = 0.0
     if wl.get("calibrate"):
         cal = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select="topk", keep=wl["keep"],
@@ -367,11 +372,6 @@ def main():
     cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select=wl["select"], keep=wl["keep"],
                            threshold=threshold, relative=wl["relative"])
     cfg_dense = dash.make_config(mode="dense")
-
-    def run(c):
-        if varlen:
-            return dash.prefill_varlen(stack, H, cu, c, idx_out=idx, delta_out=delta)[0]
-        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
 
     def step(c):
         H.copy_(h0)

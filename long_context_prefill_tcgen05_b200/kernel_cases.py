@@ -42,6 +42,7 @@ def main():
     ap.add_argument("--K", type=int, default=3584)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--layers", type=int, default=1, help="decode: layers of the stack")
     args = ap.parse_args()
     build.build()
     dims = inputs.QWEN7B
@@ -88,14 +89,14 @@ def main():
         ms = _time(lambda: dash.compact(X, idx), args.iters, args.warmup)
         out.update(T=args.T, ms=ms, gbs=2 * (args.T // 2) * dims.d_model * 2 / ms / 1e6)
     elif args.case in ("decode", "decode_attention"):
-        # one generation step of a one-layer stack (or its attention alone) for
-        # M sequences, each with a cache of T random rows
-        n, T = args.M, args.T
+        # one generation step of a stack of --layers layers (or one layer's
+        # attention alone) for M sequences, each with a cache of T random rows
+        n, T, nl = args.M, args.T, args.layers
         hq, hkv, hd = dims.n_heads, dims.n_kv_heads, dims.head_dim
-        stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev, n_layers=1))
+        stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev, n_layers=nl))
         cap = T + args.iters + args.warmup + 1
         cache = dash.KVCache(stack, n, cap, device=dev)
-        for i in range(n):
+        for i in range(n * nl):
             cache.k[i][:T] = rnd(T, hkv * hd)
             cache.v[i][:T] = rnd(T, hkv * hd)
             cache.desc[i].len = T
@@ -107,11 +108,11 @@ def main():
                 dash.decode_step(stack, X, [step[0]] * n, cache)
                 step[0] += 1
             ms = _time(run, args.iters, args.warmup)
-            by = costs.layer_weight_bytes(dims) + n * (T + 1) * hkv * hd * 2 * 2
+            by = nl * (costs.layer_weight_bytes(dims) + n * (T + 1) * hkv * hd * 2 * 2)
         else:
             Q = rnd(n, hq * hd)
             O = torch.empty_like(Q)
-            kv = [(cache.k[i][:T], cache.v[i][:T]) for i in range(n)]
+            kv = [(cache.k[i * nl][:T], cache.v[i * nl][:T]) for i in range(n)]
             ms = _time(lambda: dash.decode_attention(Q, kv, hq, hkv, hd, out=O), args.iters, args.warmup)
             by = n * T * hkv * hd * 2 * 2
         out.update(T=T, n=n, ms=ms, gbs=by / ms / 1e6)
