@@ -77,16 +77,25 @@ def load_peaks():
 
 
 # ------------------------------------------------------------ distributed
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+def dist_env():
+    """(world, rank, local rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(backend=None, timeout_s=600):
+    """One process per GPU: NCCL when CUDA is present, else gloo (CPU tests of the
+    multi-rank host logic).  The replicas exchange only timing results."""
+    world, rank, local = dist_env()
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, **kw)
     return world, rank, local
 
 
@@ -97,10 +106,12 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of x over the ranks (multi-GPU times are the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -326,10 +337,12 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the dense / other-mode / e2e legs")
     ap.add_argument("--no-decode", action="store_true", help="skip the generation leg")
     args = ap.parse_args()
-    world, rank, local = dist_setup()
     if args.impl == "reference":
+        # rank 0 alone times the oracle on the host cores; the other ranks exit at once
+        world, rank, _ = dist_env()
         run_reference(args, world, rank)
         return
+    world, rank, local = dist_setup()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
