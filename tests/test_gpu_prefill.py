@@ -396,3 +396,41 @@ def test_prefill_monitor_window_matches_oracle(tiny, mode, select, W):
     assert np.array_equal(idx, free["idx"])
     got = to_np(Hg[:K]) if mode == "prune" else to_np(Hg)
     assert row_rel_err(got, free["hidden"]) < HIDDEN_TOL
+
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129, 300])
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+def test_prefill_ragged_lengths_match_oracle(tiny, T, mode):
+    # degenerate and ragged prompts: a single token (K = 0), one tile +/- 1 row
+    dims, h0, stack, L = tiny
+    h = h0[:T]
+    Hg, idx, delta, K = _prefill(stack, h, halt_layer=1, mode=mode, keep=0.5)
+    free = O.dash_prefill(to_np(h), L, dims.as_dict(), 1, mode, keep=0.5)
+    assert K == len(free["idx"]) == math.floor(0.5 * T)
+    assert np.array_equal(idx, free["idx"])
+    assert _rel(delta, free["delta"]) < DELTA_TOL
+    got = to_np(Hg[:K]) if mode == "prune" else to_np(Hg)
+    if len(got):
+        assert row_rel_err(got, free["hidden"]) < HIDDEN_TOL
+
+
+@pytest.mark.slow
+def test_qwen_prefill_128k_threshold_halt_properties(gpu_lib):
+    """The 128K workload's configuration (halt mode, relative Δ, threshold): the
+    kept set is exactly {t : Δ_t >= thr} on the GPU's own Δ, halted rows equal
+    the halting layer's output, and every output row is finite."""
+    dims = inputs.QWEN7B
+    T = 131072
+    stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=DEV, n_layers=3))
+    h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=DEV, span_rows=6528, span_len=128)
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=1, mode="halt", select="threshold", threshold=0.05,
+                                 relative=True)
+    assert np.array_equal(idx, O.select_threshold(delta.astype(np.float64), np.float32(0.05)))
+    assert 0 < K < T
+    first2 = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=DEV, n_layers=2))
+    Hs, _, _, _ = _prefill(first2, h0, mode="dense")
+    halted = np.setdiff1d(np.arange(T), idx)
+    assert torch.equal(Hg[halted], Hs[halted])
+    assert torch.isfinite(Hg.float()).all()
+    del stack, first2
+    torch.cuda.empty_cache()
