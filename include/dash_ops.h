@@ -27,6 +27,17 @@ dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf
 dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf16* W, int32_t N,
                         dash_bf16* Y, void* stream);
 
+/* Selects the tile schedule of every tensor-core GEMM launched afterwards by
+ * this process (dash_linear and the projections inside the layer and prefill
+ * calls).  enable != 0 (the default): GEMMs whose output width splits into
+ * 256-column tiles and with more than 128 rows run as 256 x 256 tiles on SM
+ * pairs (2-CTA clusters sharing one tcgen05 MMA), when the device can
+ * co-schedule them; enable == 0: 128 x 256 / 128 x 128 tiles on single SMs.
+ * Both accumulate each output element in fp32 over k in the same order.
+ * Returns the previous setting.  Not synchronised with launches in flight on
+ * other host threads. */
+int32_t dash_set_gemm_pairs(int32_t enable);
+
 /* Causal grouped-query attention (the attention module of §2.1):
  *   Q: [M, hq*hd], K, V: [T_kv, hkv*hd], O: [M, hq*hd] bf16.
  *   Query i sees key j iff kstart(i) <= j <= qpos(i) and j < T_kv, where

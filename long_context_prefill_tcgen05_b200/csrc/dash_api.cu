@@ -2,6 +2,7 @@
 // argument checks, workspace carving, tensor-map encoding, kernel launches,
 // and the host-side layer loop of the single-shot DASH prefill.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -168,6 +169,78 @@ dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_
   return launch_status();
 }
 
+// 256 x 256 tiles on SM pairs (2-CTA clusters).
+std::atomic<int> g_gemm_pairs{1};
+
+// How many pairs of this kernel the device runs at once (0: none, e.g. the
+// attribute or the occupancy query failed; the single-SM kernel is used).
+template <int EPI>
+int gemm_pair_capacity(const DeviceInfo& di) {
+  using C = dash::gemm::PairCfg;
+  auto kernel = dash::gemm::gemm_pair_kernel<EPI>;
+  static std::once_flag once;
+  static int max_pairs = 0;
+  std::call_once(once, [&] {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(di.num_sms & ~1));
+    cfg.blockDim = dim3(dash::gemm::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess) max_pairs = n;
+    cudaGetLastError();
+  });
+  return max_pairs;
+}
+
+template <int EPI>
+dash_status launch_gemm_pair(int max_pairs, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
+                             const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
+  using C = dash::gemm::PairCfg;
+  auto kernel = dash::gemm::gemm_pair_kernel<EPI>;
+  if (M == 0) return DASH_OK;
+  CUtensorMap ma, mb, mb2;
+  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM)) return DASH_ERR_INVALID_ARG;
+  if (EPI == dash::gemm::kEpiSwiglu) {
+    if (!make_map(&mb, B, N / 2, K, K, C::BN / 2) || !make_map(&mb2, B2, N / 2, K, K, C::BN / 2))
+      return DASH_ERR_INVALID_ARG;
+  } else {
+    if (!make_map(&mb, B, N, K, K, C::BN / 2)) return DASH_ERR_INVALID_ARG;
+    mb2 = mb;
+  }
+  dash::gemm::Shape sh;
+  sh.M = static_cast<int>(M);
+  sh.N = N;
+  sh.K = K;
+  sh.tiles_m = static_cast<int>((M + C::kRows - 1) / C::kRows);
+  sh.tiles_n = N / C::BN;
+  sh.num_tiles = sh.tiles_m * sh.tiles_n;
+  const int pairs = sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(dash::gemm::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TimedLaunch tl(kind, M, N, K, st);
+  if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, mb2, sh, ep) != cudaSuccess) return DASH_ERR_CUDA;
+  return launch_status();
+}
+
 template <int EPI>
 dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
                  const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind, int* bn_used = nullptr) {
@@ -178,6 +251,10 @@ dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, in
   const bool can128 = EPI == dash::gemm::kEpiSwiglu ? (N / 2) % 64 == 0 : N % 128 == 0;
   if (can256) {
     if (bn_used) *bn_used = 256;
+    if (M > dash::gemm::BM && g_gemm_pairs.load(std::memory_order_relaxed)) {
+      const int pairs = gemm_pair_capacity<EPI>(di);
+      if (pairs > 0) return launch_gemm_pair<EPI>(pairs, A, lda, M, K, B, B2, N, ep, st, kind);
+    }
     return launch_gemm<256, EPI>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
   if (can128) {
@@ -1138,6 +1215,8 @@ dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf
   return rmsnorm(reinterpret_cast<const bf16*>(X), M, nullptr, M, d, reinterpret_cast<const bf16*>(g), eps,
                  reinterpret_cast<bf16*>(Y), as_stream(stream));
 }
+
+int32_t dash_set_gemm_pairs(int32_t enable) { return g_gemm_pairs.exchange(enable != 0 ? 1 : 0); }
 
 dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf16* W, int32_t N, dash_bf16* Y,
                         void* stream) {

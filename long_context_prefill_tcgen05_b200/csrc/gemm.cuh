@@ -66,11 +66,12 @@ struct Cfg {
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarBytes;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
-  const int per_group = kGroupM * tiles_n;
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn,
+                                            int group_m = kGroupM) {
+  const int per_group = group_m * tiles_n;
   const int g = t / per_group;
-  const int first_m = g * kGroupM;
-  const int gsize = min(tiles_m - first_m, kGroupM);
+  const int first_m = g * group_m;
+  const int gsize = min(tiles_m - first_m, group_m);
   const int r = t - g * per_group;
   tm = first_m + r % gsize;
   tn = r / gsize;
@@ -372,6 +373,211 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+}
+
+
+// ------------------------------------------------------- CTA-pair kernel
+// The same contraction and epilogues on a pair of SMs (a 2-CTA cluster) that
+// share one 256 x 256 tile.  The even CTA issues tcgen05.mma.cta_group::2
+// with M = 256: each CTA holds 128 rows of A and 128 rows of B (for SwiGLU:
+// CTA 0 the gate rows, CTA 1 the up rows) in its own shared memory and gets
+// its 128 x 256 fp32 half of the accumulator in its own TMEM, so its
+// epilogue is the single-CTA BN = 256 epilogue on rows tm*256 + rank*128.
+// Per SM a k-block stages 32 KB (A 16 KB + half of B 16 KB) instead of 48 KB
+// at the same MMA rate, a third less L2 -> SMEM traffic and a third fewer
+// shared-memory operand reads by the tensor core.
+//
+// Barriers: full[s] lives in the even CTA; both CTAs' loads count their bytes
+// on it (.cta_group::2) and the even CTA's producer arms it for both.  The
+// MMA commits arrive on empty[s] and tfull[a] of both CTAs; all 8 epilogue
+// warps of the pair arrive on the even CTA's tempty[a].
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int kRows = 2 * BM;  // rows of A per pair tile
+  static constexpr int kStages = 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = (BN / 2) * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kGroupM = 8;  // pair tiles per raster group (2048 rows of A)
+  static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 8;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarBytes;
+};
+
+// sh.tiles_m counts 256-row pair tiles; gridDim.x = 2 * number of pairs.
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_b2, const Shape sh, const EpiArgs ep) {
+  using C = PairCfg;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain[1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t drain = smem_u32(bars + 2 * S + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 8);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(leader || EPI != kEpiSwiglu ? &tmap_b : &tmap_b2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  // The peer's barriers must be initialised before any load or commit
+  // reaches them.
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nk = sh.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full_pair0 = mapa_shared(full0, 0);
+      const CUtensorMap* map_b = EPI == kEpiSwiglu && !leader ? &tmap_b2 : &tmap_b;
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = pair; t < sh.num_tiles && ok; t += npairs) {
+        int tm, tn;
+        tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn, C::kGroupM);
+        // A rows past M are loaded from row 0 instead of as an all-out-of-range
+        // box: their products land in accumulator rows the epilogue never stores.
+        int a_row = tm * C::kRows + static_cast<int>(rank) * BM;
+        if (a_row >= sh.M) a_row = 0;
+        const int b_row = EPI == kEpiSwiglu ? tn * (C::BN / 2) : tn * C::BN + static_cast<int>(rank) * (C::BN / 2);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
+          const uint32_t fb = full_pair0 + 8 * stage;
+          tma_load_2d_pair(&tmap_a, smem_u32(sA + stage * C::kABytes), fb, kb * BK, a_row);
+          tma_load_2d_pair(map_b, smem_u32(sB + stage * C::kBBytes), fb, kb * BK, b_row);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Before the CTA may exit: the even CTA waits for every armed stage to
+      // land (its full barriers count both CTAs' bytes); both wait for the
+      // last commit on each of their empty barriers, which may come from
+      // the other SM.
+      for (int s = 0; s < S; ++s) {
+        if (!((armed >> s) & 1u)) continue;
+        if (leader) mbar_wait_drain(full0 + 8 * s, (armed_par >> s) & 1u);
+        mbar_wait(empty0 + 8 * s, (armed_par >> s) & 1u);
+      }
+      if (!ok && !leader) {
+        // After an error the even CTA may not arm the phase this CTA's last
+        // loads count on; give those copies time to land.
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 100000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader) {
+      const uint32_t idesc = umma_idesc_bf16(C::kRows, C::BN, false, false);
+      const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
+      int stage = 0, local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < sh.num_tiles && ok; t += npairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_par = (local >> 1) & 1;
+        if (!mbar_wait(tempty0 + 8 * acc, acc_par ^ 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_try_wait(full0 + 8 * stage, phase) && !mbar_wait(full0 + 8 * stage, phase)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
+            const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_commit_pair(empty0 + 8 * stage, 3);
+          }
+          __syncwarp();
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair(tfull0 + 8 * acc, 3);
+        __syncwarp();
+      }
+      // Every MMA must finish before either CTA releases its TMEM.
+      if (lane == 0) umma_commit_pair(drain, 1);
+      __syncwarp();
+      mbar_wait_drain(drain, 0);
+    }
+  } else {
+    const int wq = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t tempty_pair0 = mapa_shared(tempty0, 0);
+    int local = 0;
+    for (int t = pair; t < sh.num_tiles; t += npairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_par)) break;
+      tc_fence_after();
+      int tm, tn;
+      tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn, C::kGroupM);
+      const int m = tm * C::kRows + static_cast<int>(rank) * BM + wq * 32 + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + acc * C::BN;
+      epilogue_tile<C::BN, EPI>(tbase, m, tn, sh, ep);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_pair0 + 8 * acc);
+    }
+  }
+  // barrier.cluster is .aligned: the producer lane rejoins its warp first.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+  cluster_sync();
 }
 
 }  // namespace gemm

@@ -73,6 +73,7 @@ _SIGS = {
                              c_vp, ctypes.POINTER(c_i64), c_vp, c_vp, c_sz, c_vp]),
     "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
     "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
+    "dash_set_gemm_pairs": (c_i32, [c_i32]),
     "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "dash_prefill_varlen_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i64, c_i32, ctypes.POINTER(Config)]),
     "dash_prefill_varlen": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp,
@@ -237,6 +238,12 @@ def linear(A, W, out=None, stream=None):
     out = torch.empty(M, N, dtype=A.dtype, device=A.device) if out is None else out
     _check(lib().dash_linear(_p(A), M, K, _p(W), N, _p(out), _stream(stream)), "dash_linear")
     return out
+
+
+def set_gemm_pairs(enable):
+    """Runs later GEMMs as 256x256 tiles on SM pairs (True, the default) or as
+    single-SM tiles (False); returns the previous setting."""
+    return bool(lib().dash_set_gemm_pairs(1 if enable else 0))
 
 
 def exp2_fma(x, stream=None):

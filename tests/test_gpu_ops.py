@@ -134,6 +134,30 @@ def test_linear_matches_fp64(gpu_lib, M, K, N):
     _no_device_error()
 
 
+@pytest.mark.parametrize("M,K,N", [(129, 64, 256), (300, 3584, 4608), (1000, 18944, 512), (4096, 3584, 4608),
+                                   (8192, 3584, 3584)])
+def test_linear_pair_tiles_match_fp64_and_single_sm_tiles(gpu_lib, M, K, N):
+    """256x256 tiles on SM pairs (ragged last pair tile, a pair whose odd CTA
+    has no live rows, more tiles than pairs, long K) against fp64 and against
+    the single-SM kernel on the same inputs."""
+    g = torch.Generator().manual_seed(M * 13 + N)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    prev = dash.set_gemm_pairs(True)
+    try:
+        pair = dash.linear(A, W).cpu()
+        dash.set_gemm_pairs(False)
+        single = dash.linear(A, W).cpu()
+    finally:
+        dash.set_gemm_pairs(prev)
+    ref = to_np(A.cpu()) @ to_np(W.cpu()).T
+    for got in (pair, single):
+        assert elem_rel_err(to_np(got), ref) < 1e-2
+        assert row_rel_err(to_np(got), ref) < 5e-3
+    assert row_rel_err(to_np(pair), to_np(single).astype(np.float64)) < 1e-3
+    _no_device_error()
+
+
 # -------------------------------------------------------------- attention
 def _attn_case(M, T_kv, hq, hkv, hd, qpos, seed):
     g = torch.Generator().manual_seed(seed)

@@ -257,6 +257,48 @@ def test_qwen_layer_halt_shape(qwen_layer):
     _sampled_check(dims, W, h_in.cpu(), H.cpu(), rows, idx[rows], hfull.cpu(), np.arange(T))
 
 
+@pytest.mark.parametrize("mode", ["dense", "halt"])
+def test_qwen_layer_pair_tiles_match_single_sm_tiles(qwen_layer, mode):
+    """Every fused GEMM epilogue (RoPE/QKV split, halted K/V at original rows,
+    residual + Δ partial sums, SwiGLU, residual) on SM-pair tiles against the
+    single-SM kernel at Qwen2.5-7B widths, ragged row count."""
+    dims, stack, W = qwen_layer
+    T, K = 4096, 1500
+    hfull, _ = inputs.make_hidden(T, dims.d_model, seed=24, device=DEV)
+    rng = np.random.default_rng(3)
+    idx = np.sort(rng.choice(T, K, replace=False))
+    halted = np.setdiff1d(np.arange(T), idx)
+    ti = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    th = torch.tensor(halted, dtype=torch.int32, device=DEV)
+
+    def run(pairs):
+        prev = dash.set_gemm_pairs(pairs)
+        try:
+            if mode == "dense":
+                H = hfull.clone()
+                delta = torch.empty(T, device=DEV)
+                dash.layer_forward(stack, 0, H, delta=delta)
+            else:
+                H = hfull[ti.long()].contiguous()
+                delta = torch.empty(K, device=DEV)
+                dash.layer_forward(stack, 0, H, halt=(ti, th, hfull), delta=delta)
+        finally:
+            dash.set_gemm_pairs(prev)
+        assert dash.device_error() == 0
+        return to_np(H.cpu()), delta.cpu().numpy()
+
+    Hp, dp = run(True)
+    Hs, ds = run(False)
+    assert row_rel_err(Hp, Hs.astype(np.float64)) < 1e-3
+    assert _rel(dp, ds.astype(np.float64)) < 1e-4
+    rows = np.sort(np.concatenate([[0, len(dp) - 1], rng.choice(len(dp), 14, replace=False)]))
+    if mode == "dense":
+        _sampled_check(dims, W, hfull.cpu(), torch.from_numpy(Hp), rows, rows, hfull.cpu(), np.arange(T), dp)
+    else:
+        _sampled_check(dims, W, hfull[ti.long()].cpu(), torch.from_numpy(Hp), rows, idx[rows], hfull.cpu(),
+                       np.arange(T), dp)
+
+
 # ----------------------------------------- full-size prefill properties
 @pytest.mark.slow
 @pytest.mark.parametrize("mode", ["prune", "halt"])
