@@ -13,9 +13,10 @@
 //
 // One CTA = two 128-row query tiles (Q0, Q1) of one query head, sharing every
 // K/V tile.  Warp roles (320 threads):
-//   warp 0      TMA producer: Q0/Q1 once, then K_j (3-stage ring) and V_j
-//               (2-stage ring)
-//   warp 1      TMEM allocator and MMA issuer, in the order
+//   warp 0      TMA producer: Q0/Q1 once, then load groups (2-stage ring):
+//               group 0 = K_0, group g = V_(g-1) and K_g, the operands the
+//               MMAs of one key step consume
+//   warp 1      TMEM allocator; one of its threads issues the MMAs, in the order
 //                 S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 ...
 //               so each softmax warpgroup overlaps two MMAs of the other tile.
 //   warps 2..5  softmax of Q0, warps 6..9 softmax of Q1: one query row per
@@ -29,6 +30,11 @@
 // MMAs issued by one thread complete in order, so the commit that signals
 // S_i(j+1) also proves that P_i(j) V_j is finished: the softmax may then
 // overwrite P_i and rescale O_i without another barrier.
+// A tcgen05.mma holds its issuing thread for about its execution time, so
+// the issuing thread's other work (barrier waits, commits, fences, warp
+// votes) idles the tensor pipe: one thread issues, waits once per load group
+// and once per P, fences only before P*V (the softmax threads' TMEM writes),
+// and commits three times per key step.
 #pragma once
 
 #include "common.cuh"
@@ -38,8 +44,7 @@ namespace attn {
 
 constexpr int BQ = 128;   // query rows per tile (two tiles per CTA)
 constexpr int BKV = 128;  // keys per tile
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
+constexpr int kStages = 2;  // load groups in flight
 constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // One exponential in every 2 * kEmuPeriod columns is computed on the FMA pipe
@@ -63,11 +68,11 @@ struct Cfg {
   static constexpr int kPanels = HD / 64;  // 128-byte swizzle panels per row
   static constexpr int kTileBytes = 128 * HD * 2;
   static constexpr int kOffQ = 0;  // Q0, Q1
-  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;  // K of group g in stage g % 2
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  // q_full, g_full[2], g_empty[2], s_full[2], p_full[2], o_done[2] (last P*V of a tile), drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
 };
@@ -117,11 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   const uint32_t bar_q = smem_u32(bars);
-  const uint32_t bar_kfull = smem_u32(bars + 1);
-  const uint32_t bar_kempty = smem_u32(bars + 1 + kKStages);
-  const uint32_t bar_vfull = smem_u32(bars + 1 + 2 * kKStages);
-  const uint32_t bar_vempty = smem_u32(bars + 1 + 2 * kKStages + kVStages);
-  const uint32_t bar_sfull = smem_u32(bars + 1 + 2 * kKStages + 2 * kVStages);
+  const uint32_t bar_gfull = smem_u32(bars + 1);
+  const uint32_t bar_gempty = smem_u32(bars + 1 + kStages);
+  const uint32_t bar_sfull = smem_u32(bars + 1 + 2 * kStages);
   const uint32_t bar_pfull = bar_sfull + 16;
   const uint32_t bar_odone = bar_sfull + 32;
   const uint32_t bar_drain = bar_sfull + 48;
@@ -156,13 +159,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(bar_kfull + 8 * s, 1);
-      mbar_init(bar_kempty + 8 * s, 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(bar_vfull + 8 * s, 1);
-      mbar_init(bar_vempty + 8 * s, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_gfull + 8 * s, 1);
+      mbar_init(bar_gempty + 8 * s, 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_sfull + 8 * t, 1);
@@ -194,50 +193,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < (has1 ? 2 : 1); ++t)
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_2d(&tmap_q, sq + t * C::kTileBytes + pn * (BQ * 128), bar_q, head * HD + pn * 64, q0 + t * BQ);
-      uint32_t karmed = 0, kpar = 0, varmed = 0, vpar = 0;
-      for (int j = j0; j < n_kv; ++j) {
-        const int jl = j - j0;  // ring index
-        const int ks = jl % kKStages, vs = jl % kVStages;
-        const uint32_t kph = (jl / kKStages) & 1, vph = (jl / kVStages) & 1;
-        if (!mbar_wait(bar_kempty + 8 * ks, kph ^ 1u)) break;
-        const uint32_t sk = smem_u32(smem + C::kOffK + ks * C::kTileBytes);
-        mbar_arrive_expect_tx(bar_kfull + 8 * ks, C::kTileBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(&tmap_k, sk + pn * (BKV * 128), bar_kfull + 8 * ks, kvh * HD + pn * 64, j * BKV);
-        karmed |= 1u << ks;
-        kpar = (kpar & ~(1u << ks)) | (kph << ks);
-        if (!mbar_wait(bar_vempty + 8 * vs, vph ^ 1u)) break;
-        const uint32_t sv = smem_u32(smem + C::kOffV + vs * C::kTileBytes);
-        mbar_arrive_expect_tx(bar_vfull + 8 * vs, C::kTileBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(&tmap_v, sv + pn * (BKV * 128), bar_vfull + 8 * vs, kvh * HD + pn * 64, j * BKV);
-        varmed |= 1u << vs;
-        vpar = (vpar & ~(1u << vs)) | (vph << vs);
+      uint32_t armed = 0, apar = 0;
+      for (int g = 0; g <= n_kv - j0; ++g) {
+        const bool has_k = j0 + g < n_kv, has_v = g >= 1;
+        const int st = g % kStages;
+        const uint32_t ph = (g / kStages) & 1;
+        if (!mbar_wait(bar_gempty + 8 * st, ph ^ 1u)) break;
+        const uint32_t fb = bar_gfull + 8 * st;
+        mbar_arrive_expect_tx(fb, ((has_k ? 1 : 0) + (has_v ? 1 : 0)) * C::kTileBytes);
+        const uint32_t sk = smem_u32(smem + C::kOffK + st * C::kTileBytes);
+        const uint32_t sv = smem_u32(smem + C::kOffV + st * C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          if (has_k) tma_load_2d(&tmap_k, sk + pn * (BKV * 128), fb, kvh * HD + pn * 64, (j0 + g) * BKV);
+          if (has_v) tma_load_2d(&tmap_v, sv + pn * (BKV * 128), fb, kvh * HD + pn * 64, (j0 + g - 1) * BKV);
+        }
+        armed |= 1u << st;
+        apar = (apar & ~(1u << st)) | (ph << st);
       }
       mbar_wait_drain(bar_q, 0);
-      for (int s = 0; s < kKStages; ++s)
-        if ((karmed >> s) & 1u) mbar_wait_drain(bar_kfull + 8 * s, (kpar >> s) & 1u);
-      for (int s = 0; s < kVStages; ++s)
-        if ((varmed >> s) & 1u) mbar_wait_drain(bar_vfull + 8 * s, (vpar >> s) & 1u);
+      for (int st = 0; st < kStages; ++st)
+        if ((armed >> st) & 1u) mbar_wait_drain(bar_gfull + 8 * st, (apar >> st) & 1u);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
-    const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
-    // Descriptors are built once and advanced by adding (byte offset >> 4) to
-    // the start-address field: building them inline per instruction left the
-    // tensor pipe waiting on this thread.
-    const uint64_t qdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
-    const uint64_t kdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
-    const uint64_t vdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffV), BKV * 128, 1024);
-    // a wait with an inline first try (the barrier is usually ready)
-    auto wait = [](uint32_t bar, uint32_t par) { return mbar_try_wait(bar, par) || mbar_wait(bar, par); };
-    auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
-      const int ks = (j - j0) % kKStages;
-      if (!wait(bar_kfull + 8 * ks, ((j - j0) / kKStages) & 1)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t kd = kdesc0 + static_cast<uint64_t>((ks * C::kTileBytes) >> 4);
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
+      const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
+      // Descriptors are built once and advanced by adding (byte offset >> 4)
+      // to the start-address field.
+      const uint64_t qdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffV), BKV * 128, 1024);
+      // a wait with an inline first try (the barrier is usually ready)
+      auto wait = [](uint32_t bar, uint32_t par) { return mbar_try_wait(bar, par) || mbar_wait(bar, par); };
+      auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T, K in stage st
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
         const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -246,45 +236,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16_ss(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(bar_sfull + 8 * t);
+      };
+      // group 0 holds K_j0 only
+      bool ok = wait(bar_q, 0) && wait(bar_gfull, 0);
+      if (ok) {
+        for (int t = 0; t < 2; ++t)
+          if (jb_t[t] == j0 && j0 < n_t[t]) issue_s(t, 0);
+        umma_commit(bar_gempty);
       }
-      __syncwarp();
-      return true;
-    };
-    auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j  (P from TMEM)
-      const int vs = (j - j0) % kVStages;
-      if (!wait(bar_pfull + 8 * t, (j - jb_t[t]) & 1)) return false;
-      if (!wait(bar_vfull + 8 * vs, ((j - j0) / kVStages) & 1)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * C::kTileBytes) >> 4);
-        const uint32_t pa = tmem_base + t * BKV + BKV / 2;
-        const uint32_t acc0 = j != jb_t[t] ? 1u : 0u;
+      for (int j = j0; ok && j < n_kv; ++j) {
+        const int g = j - j0 + 1, st = g % kStages;  // group g: V_j and K_(j+1)
+        if (!wait(bar_gfull + 8 * st, (g / kStages) & 1)) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < 2; ++t) {
+          if (jb_t[t] <= j && j < n_t[t]) {  // O_t += P_t V_j  (P from TMEM)
+            if (!wait(bar_pfull + 8 * t, (j - jb_t[t]) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();  // P_t and any O_t rescale by the softmax threads precede P*V
+            const uint64_t vd = vdesc0 + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
+            const uint32_t pa = tmem_base + t * BKV + BKV / 2;
+            const uint32_t acc0 = j != jb_t[t] ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
-          umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, vd + kk * ((16 * 128) >> 4), idesc_o,
-                       kk != 0 ? 1u : acc0);
-        umma_commit(bar_odone + 8 * t);
+            for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
+              umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, vd + kk * ((16 * 128) >> 4), idesc_o,
+                           kk != 0 ? 1u : acc0);
+            if (j == n_t[t] - 1) umma_commit(bar_odone + 8 * t);
+          }
+          if (jb_t[t] <= j + 1 && j + 1 < n_t[t]) issue_s(t, st);
+        }
+        if (!ok) break;
+        umma_commit(bar_gempty + 8 * st);
       }
-      __syncwarp();
-      return true;
-    };
-    bool ok = mbar_wait(bar_q, 0);
-    for (int t = 0; t < 2; ++t)
-      if (ok && jb_t[t] == j0 && j0 < n_t[t]) ok = issue_s(t, j0);
-    for (int j = j0; ok && j < n_kv; ++j) {
-      for (int t = 0; ok && t < 2; ++t) {
-        if (jb_t[t] <= j && j < n_t[t]) ok = issue_pv(t, j);
-        if (ok && jb_t[t] <= j + 1 && j + 1 < n_t[t]) ok = issue_s(t, j + 1);
-      }
-      if (ok && lane == 0) {
-        umma_commit(bar_kempty + 8 * ((j - j0) % kKStages));
-        umma_commit(bar_vempty + 8 * ((j - j0) % kVStages));
-      }
-      __syncwarp();
+      umma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0);
     }
-    if (lane == 0) umma_commit(bar_drain);
     __syncwarp();
-    mbar_wait_drain(bar_drain, 0);
   } else {
     // ------------------------------------------------------------ softmax
     const int t = (warp - 2) >> 2;   // query tile of this warpgroup
@@ -302,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = jb; j < n; ++j) {
-      if (!mbar_wait(bar_sfull + 8 * t, (j - jb) & 1)) {
+      // warp-uniform outcomes keep the warp converged for __any_sync and tcgen05.ld
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull + 8 * t, (j - jb) & 1))) {
         ok = false;
         break;
       }
@@ -380,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar_pfull + 8 * t);
     }
-    if (ok && n > jb && mbar_wait(bar_odone + 8 * t, (n - 1 - jb) & 1)) {
+    // o_done[t] completes once, after the last P*V of this tile
+    if (__all_sync(0xffffffffu, ok && n > jb && mbar_wait(bar_odone + 8 * t, 0))) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       __nv_bfloat16* dst = p.out + static_cast<int64_t>(mrow) * p.ldo + head * HD;

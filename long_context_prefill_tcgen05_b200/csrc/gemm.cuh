@@ -304,52 +304,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((armed >> s) & 1u) mbar_wait_drain(full0 + 8 * s, (armed_par >> s) & 1u);
     }
   } else if (warp == 1) {
-    const uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
-    // Descriptors differ only in their start-address field (bytes >> 4), so
-    // they are advanced by integer adds: building each one inline in the
-    // issue loop left the tensor pipe waiting on the issuing thread.
-    const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
-    const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
-    int stage = 0, local = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < sh.num_tiles && ok; t += gridDim.x, ++local) {
-      const int acc = local & 1;
-      const uint32_t acc_par = (local >> 1) & 1;
-      if (!mbar_wait(tempty0 + 8 * acc, acc_par ^ 1u)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_try_wait(full0 + 8 * stage, phase) && !mbar_wait(full0 + 8 * stage, phase)) {
+    // One thread issues: a tcgen05.mma holds its issuing thread for about its
+    // execution time, so time spent on warp syncs or fences here idles the
+    // tensor pipe.  The TMA-loaded stages are ordered by the full-barrier wait
+    // alone; a tcgen05 fence is taken only after the epilogue's release of an
+    // accumulator (other threads' tcgen05.ld before this thread's MMAs).
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
+      // Descriptors differ only in their start-address field (bytes >> 4), so
+      // they are advanced by integer adds.
+      const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
+      int stage = 0, local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < sh.num_tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_par = (local >> 1) & 1;
+        if (!mbar_wait(tempty0 + 8 * acc, acc_par ^ 1u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_try_wait(full0 + 8 * stage, phase) && !mbar_wait(full0 + 8 * stage, phase)) {
+            ok = false;
+            break;
+          }
           const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
           const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // 16 columns = 32 bytes along the 128-byte swizzle row
             umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(empty0 + 8 * stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * acc);
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(tfull0 + 8 * acc);
-      __syncwarp();
+      // Every MMA this thread issued must finish before TMEM is released.
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
     }
-    // Every MMA this warp issued must finish before TMEM is released.
-    if (lane == 0) umma_commit(drain);
     __syncwarp();
-    mbar_wait_drain(drain, 0);
   } else {
     const int wq = warp & 3;  // TMEM lane quarter this warp may access
     int local = 0;
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (leader) {
+    if (leader && lane == 0) {  // one issuing thread, as in gemm_kernel
       const uint32_t idesc = umma_idesc_bf16(C::kRows, C::BN, false, false);
       const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
       const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
@@ -526,30 +527,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
-            const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
+          const uint64_t ad = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-            umma_commit_pair(empty0 + 8 * stage, 3);
-          }
-          __syncwarp();
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(empty0 + 8 * stage, 3);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        if (lane == 0) umma_commit_pair(tfull0 + 8 * acc, 3);
-        __syncwarp();
+        umma_commit_pair(tfull0 + 8 * acc, 3);
       }
       // Every MMA must finish before either CTA releases its TMEM.
-      if (lane == 0) umma_commit_pair(drain, 1);
-      __syncwarp();
+      umma_commit_pair(drain, 1);
       mbar_wait_drain(drain, 0);
     }
+    __syncwarp();
   } else {
     const int wq = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t tempty_pair0 = mapa_shared(tempty0, 0);
