@@ -18,6 +18,9 @@ SHORT = [
     ("gemm_kernel<256, 3>", "gemm_gate_up_swiglu"), ("gemm_kernel<128, 3>", "gemm_gate_up_swiglu"),
     ("gemm_kernel<256, 1>", "gemm_resid (o_proj / down)"), ("gemm_kernel<128, 1>", "gemm_resid (o_proj / down)"),
     ("gemm_kernel<256, 0>", "gemm_store"), ("gemm_kernel<128, 0>", "gemm_store"),
+    ("gemm_pair_kernel<4>", "gemm_qkv_rope"), ("gemm_pair_kernel<2>", "gemm_o_resid_delta"),
+    ("gemm_pair_kernel<3>", "gemm_gate_up_swiglu"), ("gemm_pair_kernel<1>", "gemm_resid (o_proj / down)"),
+    ("gemm_pair_kernel<0>", "gemm_store"),
     ("rmsnorm_kernel", "rmsnorm"), ("score_from_ssq", "score"), ("score_kernel", "score"),
     ("select_kernel", "select"), ("move_rows_kernel<false>", "gather"), ("move_rows_kernel<true>", "scatter"),
     ("move_rows_kernel<0>", "gather"), ("move_rows_kernel<1>", "scatter"),
