@@ -89,6 +89,8 @@ __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_ro
 
 // -------------------------------------------------------------------- score
 // Δ_t = ||U_t||_2, or ||U_t||_2 / ||H_t||_2 (one warp per row).
+constexpr int kRowChunks = 16;  // 16-byte chunks per lane in flight (a 4096-wide bf16 row)
+
 __global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ h,
                              int64_t T, int d, int relative, float* __restrict__ delta) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,13 +99,22 @@ __global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfl
   const int nv = d >> 3;
   const uint4* ur = reinterpret_cast<const uint4*>(u + r * d);
   float su = 0.f, sh = 0.f;
-#pragma unroll 4
-  for (int c = lane; c < nv; c += 32) su += sumsq8(__ldcs(ur + c));
-  if (relative) {
-    const uint4* hr = reinterpret_cast<const uint4*>(h + r * d);
-#pragma unroll 4
-    for (int c = lane; c < nv; c += 32) sh += sumsq8(__ldcs(hr + c));
-  }
+  // all of a lane's chunks of the row in flight before the reduction
+  auto sumsq_row = [&](const uint4* row) {
+    float acc = 0.f;
+    for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunks) {
+      uint4 v[kRowChunks];
+#pragma unroll
+      for (int u = 0; u < kRowChunks; ++u)
+        if (c0 + 32 * u < nv) v[u] = __ldcs(row + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < kRowChunks; ++u)
+        if (c0 + 32 * u < nv) acc += sumsq8(v[u]);
+    }
+    return acc;
+  };
+  su = sumsq_row(ur);
+  if (relative) sh = sumsq_row(reinterpret_cast<const uint4*>(h + r * d));
   su = warp_sum(su);
   if (relative) sh = warp_sum(sh);
   if (lane == 0) {
@@ -377,8 +388,16 @@ __global__ void move_rows_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfl
     }
     const uint4* s = reinterpret_cast<const uint4*>(src + (kScatter ? i : t) * d);
     uint4* o = reinterpret_cast<uint4*>(dst + (kScatter ? t : i) * d);
-#pragma unroll 4
-    for (int c = lane; c < nv; c += 32) o[c] = __ldcs(s + c);
+    // all of a lane's chunks of the row in flight before the first store
+    for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunks) {
+      uint4 v[kRowChunks];
+#pragma unroll
+      for (int u = 0; u < kRowChunks; ++u)
+        if (c0 + 32 * u < nv) v[u] = __ldcs(s + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < kRowChunks; ++u)
+        if (c0 + 32 * u < nv) o[c0 + 32 * u] = v[u];
+    }
   }
 }
 

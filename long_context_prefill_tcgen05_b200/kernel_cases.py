@@ -7,6 +7,7 @@ for ncu captures of a single kernel on a small case).
     python -m long_context_prefill_tcgen05_b200.kernel_cases select --T 32768
     python -m long_context_prefill_tcgen05_b200.kernel_cases decode --T 32768 --M 1
     python -m long_context_prefill_tcgen05_b200.kernel_cases decode_attention --T 32768 --M 1
+    python -m long_context_prefill_tcgen05_b200.kernel_cases rows --T 32768
 
 Shapes default to the Qwen2.5-7B-shaped stack (28 q / 4 kv heads, hd 128,
 d 3584, FFN 18944).  Prints one JSON line with the mean CUDA-event time.
@@ -35,7 +36,7 @@ def _time(fn, iters, warmup):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["attention", "linear", "layer", "select", "score", "gather", "decode",
-                                     "decode_attention"])
+                                     "decode_attention", "rows"])
     ap.add_argument("--T", type=int, default=8192)
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=37888)
@@ -88,6 +89,46 @@ def main():
         idx = torch.sort(torch.randperm(args.T, generator=g, device=dev)[:args.T // 2]).values.int()
         ms = _time(lambda: dash.compact(X, idx), args.iters, args.warmup)
         out.update(T=args.T, ms=ms, gbs=2 * (args.T // 2) * dims.d_model * 2 / ms / 1e6)
+    elif args.case == "rows":
+        # score (absolute and relative), gather and scatter of T/2 rows, and top-k
+        # select, each launch timed alone with L2 flushed before it (cold HBM)
+        T, d = args.T, dims.d_model
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+        def cold(fn, n=20):
+            ts = []
+            for i in range(n + 3):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= 3:
+                    ts.append(e0.elapsed_time(e1))
+            return sorted(ts)[len(ts) // 2]
+        U, H = rnd(T, d), rnd(T, d)
+        delta = torch.empty(T, device=dev)
+        K = T // 2
+        idx = torch.sort(torch.randperm(T, generator=g, device=dev)[:K]).values.int()
+        Y = dash.compact(U, idx)
+        s = torch.rand(T, generator=g, device=dev)
+        sel_idx = torch.empty(T, dtype=torch.int32, device=dev)
+        count = torch.empty(1, dtype=torch.int32, device=dev)
+        L = dash.lib()
+        ms = {
+            "score": cold(lambda: dash.score(U, out=delta)),
+            "score_relative": cold(lambda: dash.score(U, H, relative=True, out=delta)),
+            "gather": cold(lambda: dash.compact(U, idx)),
+            "scatter": cold(lambda: dash.scatter(Y, idx, H)),
+            "select": cold(lambda: L.dash_select(dash._p(s), T, dash.SELECTS["topk"], 0.5, 0.0, 0, 0,
+                                                 dash._p(sel_idx), None, dash._p(count), None, 0, None)),
+        }
+        nbytes = {"score": T * d * 2, "score_relative": 2 * T * d * 2, "gather": 2 * K * d * 2,
+                  "scatter": 2 * K * d * 2, "select": T * 4 + K * 4}
+        out.update(T=T, d=d, K=K, us={k: round(v * 1e3, 1) for k, v in ms.items()},
+                   gbs={k: round(nbytes[k] / ms[k] / 1e6) for k in ms})
+        dash.check_device()
     elif args.case in ("decode", "decode_attention"):
         # one generation step of a stack of --layers layers (or one layer's
         # attention alone) for M sequences, each with a cache of T random rows
