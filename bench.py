@@ -483,25 +483,51 @@ def main():
             "speedup_vs_dense": ms_d / ms,
             "flop_bound": dense_flops / halted_flops,
         }
-        # end to end through the C ABI from pinned host memory: H2D of the
-        # input, the prefill, D2H of the K active rows' final states
+        # End to end through the C ABI from pinned host memory, as a serving
+        # loop runs it: the residual stream is double-buffered, so step i+1's
+        # input goes up and step i's result (the K active rows) comes back on
+        # a copy stream while step i computes.  Every step's copies are inside
+        # the timed region; only the first upload and the last read-back are
+        # not hidden behind a prefill.
         h_host = h0.cpu().pin_memory()
         out_host = torch.empty(T, dims.d_model, dtype=torch.bfloat16).pin_memory()
-        def e2e_step():
-            H.copy_(h_host, non_blocking=True)
-            k = run(cfg)
-            rows = k if args.mode == "prune" else T
-            out_host[:rows].copy_(H[:rows], non_blocking=True)
+        comp, copy = torch.cuda.Stream(), torch.cuda.Stream()
+        bufs = [H, torch.empty_like(H)]
+        ready = [torch.cuda.Event(), torch.cuda.Event()]
+        done = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def run_on(buf, c):
+            if varlen:
+                return dash.prefill_varlen(stack, buf, cu, c, idx_out=idx, delta_out=delta, stream=comp)[0]
+            return dash.prefill(stack, buf, c, idx_out=idx, delta_out=delta, stream=comp)
+
+        def e2e_run(n):
+            rows = T
+            with torch.cuda.stream(copy):
+                bufs[0].copy_(h_host, non_blocking=True)
+                ready[0].record(copy)
+            for i in range(n):
+                cur, nxt = bufs[i % 2], bufs[(i + 1) % 2]
+                if i + 1 < n:  # nxt's last read-back is already queued ahead on this stream
+                    with torch.cuda.stream(copy):
+                        nxt.copy_(h_host, non_blocking=True)
+                        ready[(i + 1) % 2].record(copy)
+                comp.wait_event(ready[i % 2])
+                k = run_on(cur, cfg)
+                done[i % 2].record(comp)
+                rows = k if args.mode == "prune" else T
+                copy.wait_event(done[i % 2])
+                with torch.cuda.stream(copy):
+                    out_host[:rows].copy_(cur[:rows], non_blocking=True)
             return rows
-        e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        n_e2e = max(2, args.steps // 2)
-        for _ in range(n_e2e):
-            rows = e2e_step()
-        e1.record()
+        n_e2e = max(2, args.steps)
+        e0.record(copy)
+        rows = e2e_run(n_e2e)
+        e1.record(copy)
         torch.cuda.synchronize()
         ms_e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
         extra["e2e"] = {"value": world * T / (ms_e / 1e3), "unit": "tokens/s",
