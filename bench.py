@@ -460,14 +460,21 @@ def main():
 
     extra = {}
     if not args.no_extra:
-        step(cfg_dense)
-        ms_d, _, _ = timed(cfg_dense, max(2, args.steps // 2))
         dense_flops = costs.varlen_prefill_flops(dims, cu) if varlen else costs.prefill_flops(dims, T)
         other = "halt" if args.mode == "prune" else "prune"
         cfg_o = dash.make_config(halt_layer=wl["halt_layer"], mode=other, select=wl["select"], keep=wl["keep"],
                                  threshold=threshold, relative=wl["relative"])
+        # Dense, this mode and the other mode are timed in alternating single
+        # steps (medians over the rounds), so a drift of the power-capped clock
+        # during the run does not bias their ratios.
+        step(cfg_dense)
         step(cfg_o)
-        ms_o, K_o, _ = timed(cfg_o, max(2, args.steps // 2))
+        legs = [(cfg_dense, []), (cfg, []), (cfg_o, [])]
+        for r in range(max(3, args.steps)):
+            for c, times in legs[r % 3:] + legs[:r % 3]:
+                times.append(timed(c, 1)[0])
+        ms_d, ms_m, ms_o = (statistics.median(t) for _, t in legs)
+        _, K_o, _ = timed(cfg_o, 1)  # the other mode's active set, for its FLOP count
         act_o = idx[:K_o].cpu().numpy()
         if varlen:
             cnt_o = [int(((act_o >= a) & (act_o < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
@@ -480,8 +487,10 @@ def main():
             other + "_mode": {"tokens_per_s": world * T / (ms_o / 1e3), "ms_per_step": ms_o, "K": K_o,
                               "speedup_vs_dense": ms_d / ms_o,
                               "flop_bound": dense_flops / flops_o},
-            "speedup_vs_dense": ms_d / ms,
+            "speedup_vs_dense": ms_d / ms_m,
             "flop_bound": dense_flops / halted_flops,
+            "interleaved": {"rounds": len(legs[0][1]), "ms_per_step": {"dense": ms_d, args.mode: ms_m, other: ms_o},
+                            "note": "median of single steps alternating dense / this mode / the other mode"},
         }
         # End to end through the C ABI from pinned host memory, as a serving
         # loop runs it: the residual stream is double-buffered, so step i+1's
