@@ -316,11 +316,12 @@ dash_status attention(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, 
 dash_status rmsnorm(const bf16* X, int64_t x_rows, const int32_t* rowmap, int64_t rows, int d, const bf16* g,
                     double eps, bf16* Y, cudaStream_t st, float* row_scale = nullptr) {
   if (rows == 0) return DASH_OK;
-  const int warps = 8;
-  const int64_t blocks = (rows + warps - 1) / warps;
+  // 4-warp blocks, one row per warp
+  constexpr int kWarps = 4;
+  const int64_t blocks = (rows + kWarps - 1) / kWarps;
   TimedLaunch tl(DASH_K_RMSNORM, rows, d, 0, st);
-  dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
-      X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y, row_scale);
+  dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * kWarps, static_cast<size_t>(d) * sizeof(bf16),
+                               st>>>(X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y, row_scale);
   return launch_status();
 }
 

@@ -36,46 +36,54 @@ __device__ __forceinline__ float sumsq8(const uint4& v) {
 // row_scale[r] = rsqrt(mean(x^2) + eps) instead: the GEMM that consumes y
 // applies the scale to its fp32 accumulator, so the normalised activation is
 // never rounded to bf16 (x * g is exact in bf16 when g = 1).
+// Each warp issues its row's loads first; the block then stages g (d bf16,
+// dynamic shared memory) while they are in flight, so the scaling after the
+// row's reduction waits on no second global load.
 __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_rows,
                                const int32_t* __restrict__ rowmap, int64_t rows, int d,
                                const __nv_bfloat16* __restrict__ g, float eps,
                                __nv_bfloat16* __restrict__ y, float* __restrict__ row_scale) {
+  extern __shared__ uint4 g_s[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-  if (r >= rows) return;
+  const int nv = d >> 3;
+  bool live = r < rows;
   int64_t src = r;
-  if (rowmap) {
+  if (live && rowmap) {
     src = rowmap[r];
-    if (src < 0 || src >= x_rows) {
+    if (src < 0 || src >= x_rows) {  // warp-uniform
       if (lane == 0) flag_error(kDevErrIndex);
-      return;
+      live = false;
     }
   }
-  const int nv = d >> 3;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + src * d);
   uint4 v[kMaxVec];
+  if (live) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + src * d);
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+      const int c = lane + 32 * i;
+      if (c < nv) v[i] = xr[c];
+    }
+  }
+  for (int c = threadIdx.x; c < nv; c += blockDim.x) g_s[c] = reinterpret_cast<const uint4*>(g)[c];
+  __syncthreads();
+  if (!live) return;
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    const int c = lane + 32 * i;
-    if (c < nv) {
-      v[i] = xr[c];
-      ss += sumsq8(v[i]);
-    }
-  }
+  for (int i = 0; i < kMaxVec; ++i)
+    if (lane + 32 * i < nv) ss += sumsq8(v[i]);
   ss = warp_sum(ss);
   float rs = rsqrtf(ss / static_cast<float>(d) + eps);
   if (row_scale) {
     if (lane == 0) row_scale[r] = rs;
     rs = 1.f;
   }
-  const uint4* gr = reinterpret_cast<const uint4*>(g);
   uint4* yr = reinterpret_cast<uint4*>(y + r * d);
 #pragma unroll
   for (int i = 0; i < kMaxVec; ++i) {
     const int c = lane + 32 * i;
     if (c < nv) {
-      const uint4 gv = gr[c];
+      const uint4 gv = g_s[c];
       const uint32_t xw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
       uint32_t o[4];

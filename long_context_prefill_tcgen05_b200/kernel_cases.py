@@ -90,8 +90,8 @@ def main():
         ms = _time(lambda: dash.compact(X, idx), args.iters, args.warmup)
         out.update(T=args.T, ms=ms, gbs=2 * (args.T // 2) * dims.d_model * 2 / ms / 1e6)
     elif args.case == "rows":
-        # score (absolute and relative), gather and scatter of T/2 rows, and top-k
-        # select, each launch timed alone with L2 flushed before it (cold HBM)
+        # RMSNorm, score (absolute and relative), gather and scatter of T/2 rows, and
+        # top-k select, each launch timed alone with L2 flushed before it (cold HBM)
         T, d = args.T, dims.d_model
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -116,7 +116,11 @@ def main():
         sel_idx = torch.empty(T, dtype=torch.int32, device=dev)
         count = torch.empty(1, dtype=torch.int32, device=dev)
         L = dash.lib()
+        gain = (1 + 0.1 * torch.randn(d, generator=g, device=dev)).bfloat16()
+        Yn = torch.empty_like(H)
         ms = {
+            "rmsnorm": cold(lambda: dash._check(L.dash_rmsnorm(dash._p(H), T, d, dash._p(gain), 1e-6, dash._p(Yn), None),
+                                                "dash_rmsnorm")),
             "score": cold(lambda: dash.score(U, out=delta)),
             "score_relative": cold(lambda: dash.score(U, H, relative=True, out=delta)),
             "gather": cold(lambda: dash.compact(U, idx)),
@@ -124,7 +128,7 @@ def main():
             "select": cold(lambda: L.dash_select(dash._p(s), T, dash.SELECTS["topk"], 0.5, 0.0, 0, 0,
                                                  dash._p(sel_idx), None, dash._p(count), None, 0, None)),
         }
-        nbytes = {"score": T * d * 2, "score_relative": 2 * T * d * 2, "gather": 2 * K * d * 2,
+        nbytes = {"rmsnorm": 2 * T * d * 2, "score": T * d * 2, "score_relative": 2 * T * d * 2, "gather": 2 * K * d * 2,
                   "scatter": 2 * K * d * 2, "select": T * 4 + K * 4}
         out.update(T=T, d=d, K=K, us={k: round(v * 1e3, 1) for k, v in ms.items()},
                    gbs={k: round(nbytes[k] / ms[k] / 1e6) for k in ms})
