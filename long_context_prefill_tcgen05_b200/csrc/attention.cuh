@@ -16,9 +16,11 @@
 //   warp 0      TMA producer: Q0/Q1 once, then load groups (2-stage ring):
 //               group 0 = K_0, group g = V_(g-1) and K_g, the operands the
 //               MMAs of one key step consume
-//   warp 1      TMEM allocator; one of its threads issues the MMAs, in the order
+//   warp 1      TMEM allocator and MMA issue, in the order
 //                 S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 ...
 //               so each softmax warpgroup overlaps two MMAs of the other tile.
+//               The warp runs the issue loop converged; elect.sync picks the
+//               lane that issues each MMA and commit.
 //   warps 2..5  softmax of Q0, warps 6..9 softmax of Q1: one query row per
 //               thread (TMEM lane = row); S_j is read from TMEM, the running
 //               max / sum kept in registers, O rescaled in TMEM only when the
@@ -30,11 +32,12 @@
 // MMAs issued by one thread complete in order, so the commit that signals
 // S_i(j+1) also proves that P_i(j) V_j is finished: the softmax may then
 // overwrite P_i and rescale O_i without another barrier.
-// A tcgen05.mma holds its issuing thread for about its execution time, so
-// the issuing thread's other work (barrier waits, commits, fences, warp
-// votes) idles the tensor pipe: one thread issues, waits once per load group
-// and once per P, fences only before P*V (the softmax threads' TMEM writes),
-// and commits three times per key step.
+// A tcgen05.mma holds its issuing warp for about its execution time, so the
+// warp's other work (barrier waits, commits, fences) idles the tensor pipe:
+// it waits once per load group and once per P, fences only before P*V (the
+// softmax threads' TMEM writes), and commits three times per key step.
+// Issuing from the converged warp measured faster than from a lone lane-0
+// thread in a divergent branch.
 #pragma once
 
 #include "common.cuh"
@@ -109,6 +112,36 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Issue forms for a converged warp: elect.sync picks one lane, which alone
+// issues the MMA / commit (every lane of the warp must execute them).
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
 }
 
@@ -216,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
+    {  // converged warp; elected lanes issue
       const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
       const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
       // Descriptors are built once and advanced by adding (byte offset >> 4)
@@ -225,7 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t kdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
       const uint64_t vdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffV), BKV * 128, 1024);
       // a wait with an inline first try (the barrier is usually ready)
-      auto wait = [](uint32_t bar, uint32_t par) { return mbar_try_wait(bar, par) || mbar_wait(bar, par); };
+      // lane 0's outcome, broadcast: every decision stays warp-uniform, so
+      // elect.sync always sees the whole warp
+      auto wait = [](uint32_t bar, uint32_t par) {
+        const bool r = mbar_try_wait(bar, par) || mbar_wait(bar, par);
+        return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      };
       auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T, K in stage st
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
         const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
@@ -233,16 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < HD / 16; ++kk) {
           constexpr int kPanelStep = (BQ * 128) >> 4;
           const int off = (kk >> 2) * kPanelStep + (kk & 3) * 2;  // (panel, 32-byte column step) >> 4
-          umma_bf16_ss(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+          umma_ss_elect(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
-        umma_commit(bar_sfull + 8 * t);
+        umma_commit_elect(bar_sfull + 8 * t);
       };
       // group 0 holds K_j0 only
       bool ok = wait(bar_q, 0) && wait(bar_gfull, 0);
       if (ok) {
         for (int t = 0; t < 2; ++t)
           if (jb_t[t] == j0 && j0 < n_t[t]) issue_s(t, 0);
-        umma_commit(bar_gempty);
+        umma_commit_elect(bar_gempty);
       }
       for (int j = j0; ok && j < n_kv; ++j) {
         const int g = j - j0 + 1, st = g % kStages;  // group g: V_j and K_(j+1)
@@ -262,16 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t acc0 = j != jb_t[t] ? 1u : 0u;
 #pragma unroll
             for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 16 rows of 128 bytes
-              umma_bf16_ts(tmem_base + 256 + t * 128, pa + kk * 8, vd + kk * ((16 * 128) >> 4), idesc_o,
+              umma_ts_elect(tmem_base + 256 + t * 128, pa + kk * 8, vd + kk * ((16 * 128) >> 4), idesc_o,
                            kk != 0 ? 1u : acc0);
-            if (j == n_t[t] - 1) umma_commit(bar_odone + 8 * t);
+            if (j == n_t[t] - 1) umma_commit_elect(bar_odone + 8 * t);
           }
           if (jb_t[t] <= j + 1 && j + 1 < n_t[t]) issue_s(t, st);
         }
         if (!ok) break;
-        umma_commit(bar_gempty + 8 * st);
+        umma_commit_elect(bar_gempty + 8 * st);
       }
-      umma_commit(bar_drain);
+      umma_commit_elect(bar_drain);
       mbar_wait_drain(bar_drain, 0);
     }
     __syncwarp();
