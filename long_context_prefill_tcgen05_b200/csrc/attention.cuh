@@ -115,18 +115,7 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-// Issue forms for a converged warp: elect.sync picks one lane, which alone
-// issues the MMA / commit (every lane of the warp must execute them).
-__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
+// P*V with A = P from TMEM, issued by one elected lane of a converged warp.
 __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate) {
   asm volatile(
@@ -137,14 +126,6 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
-      : "memory");
-}
-
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -260,10 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // a wait with an inline first try (the barrier is usually ready)
       // lane 0's outcome, broadcast: every decision stays warp-uniform, so
       // elect.sync always sees the whole warp
-      auto wait = [](uint32_t bar, uint32_t par) {
-        const bool r = mbar_try_wait(bar, par) || mbar_wait(bar, par);
-        return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
-      };
+      auto wait = [](uint32_t bar, uint32_t par) { return warp_wait(bar, par); };
       auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T, K in stage st
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
         const uint64_t qd = qdesc0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
@@ -271,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < HD / 16; ++kk) {
           constexpr int kPanelStep = (BQ * 128) >> 4;
           const int off = (kk >> 2) * kPanelStep + (kk & 3) * 2;  // (panel, 32-byte column step) >> 4
-          umma_ss_elect(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+          umma_bf16_ss_elect(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit_elect(bar_sfull + 8 * t);
       };
