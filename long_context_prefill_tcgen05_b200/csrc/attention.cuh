@@ -314,25 +314,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // S in two halves: the max of the first runs while the second loads
       uint32_t u[BKV];
       tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(u + 0));
       tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+      tmem_ld_wait();
       tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(u + 64));
       tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(u + 96));
-      tmem_ld_wait();
       float* s = reinterpret_cast<float*>(u);
       const int kv0 = j * BKV;
-      if (kv0 + BKV - 1 > pos_first[t] || kv0 + BKV > p.T_kv || kv0 < ks_last[t]) {
-        const int hi = min(row_pos, p.T_kv - 1) - kv0;  // visible columns of this row: [lo, hi]
-        const int lo = row_ks - kv0;
-#pragma unroll
-        for (int c = 0; c < BKV; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
-      }
+      const bool edge = kv0 + BKV - 1 > pos_first[t] || kv0 + BKV > p.T_kv || kv0 < ks_last[t];
+      const int hi = min(row_pos, p.T_kv - 1) - kv0;  // visible columns of this row: [lo, hi]
+      const int lo = row_ks - kv0;
       float mx[8];
+      if (edge) {
+#pragma unroll
+        for (int c = 0; c < BKV / 2; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx[k] = s[k];
 #pragma unroll
-      for (int c = 8; c < BKV; c += 8)
+      for (int c = 8; c < BKV / 2; c += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
+      tmem_ld_wait();
+      if (edge) {
+#pragma unroll
+        for (int c = BKV / 2; c < BKV; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
+      }
+#pragma unroll
+      for (int c = BKV / 2; c < BKV; c += 8)
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
       const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
