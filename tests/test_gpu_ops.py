@@ -191,6 +191,34 @@ def test_attention_indexed_queries_match_oracle(gpu_lib, M, T_kv, hq, hkv, hd):
     _no_device_error()
 
 
+@pytest.mark.parametrize("M,hq,hkv,hd,growth", [(700, 8, 2, 128, 0.002), (1030, 4, 2, 64, 0.003),
+                                                 (600, 4, 1, 128, 0.02)])
+def test_attention_growing_scores_rescale_matches_oracle(gpu_lib, M, hq, hkv, hd, growth):
+    """Scores that grow along the keys (k_j = noise + growth * j * u, q_i = noise + u for one fixed
+    direction u of norm sqrt(hd)) make a row's maximum climb tile after tile, so the online softmax
+    has to move its reference and rescale O and l, the path that random N(0,1) inputs never reach.
+    The case checks that the climb really passes the kernel's lazy-rescale margin of 2^8."""
+    g = torch.Generator().manual_seed(M + hd)
+    u = torch.randn(hd, generator=g)
+    u = u / u.norm() * hd ** 0.5
+    pos = torch.arange(M, dtype=torch.float32)
+    Q = (torch.randn(M, hq, hd, generator=g) + u).reshape(M, hq * hd).to(torch.bfloat16)
+    K = (torch.randn(M, hkv, hd, generator=g) + growth * pos[:, None, None] * u).reshape(M, hkv * hd)
+    K = K.to(torch.bfloat16)
+    V = torch.randn(M, hkv * hd, generator=g).to(torch.bfloat16)
+    q, k = to_np(Q).reshape(M, hq, hd), to_np(K).reshape(M, hkv, hd)
+    # some row's causal maximum (log2 units) rises by more than 8 from one 128-key tile to a later one
+    s = np.einsum("ihd,jhd->hij", q[:, ::hq // hkv], k) / np.sqrt(hd) * np.log2(np.e)  # head h*G <-> kv head h
+    s = np.where(np.arange(M)[None, :, None] >= np.arange(M)[None, None, :], s, -np.inf)
+    first = s[:, :, :128].max(-1)
+    assert np.nanmax(s.max(-1) - first) > 8.0
+    got = to_np(dash.attention(Q.to(DEV), K.to(DEV), V.to(DEV), hq, hkv, hd).cpu())
+    ref = O.causal_gqa_attention(q, k, to_np(V).reshape(M, hkv, hd), np.arange(M), np.arange(M)).reshape(M, -1)
+    assert row_rel_err(got.reshape(M * hq, hd), ref.reshape(M * hq, hd)) < 2e-2
+    assert elem_rel_err(got, ref) < 2e-2
+    _no_device_error()
+
+
 def test_exp2_fma_within_its_error_bound(gpu_lib):
     x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.999])])
     y = dash.exp2_fma(x.to(DEV)).cpu().double().numpy()
