@@ -348,16 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
       const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
-      bool rescale = false;
+      // Each row moves its own reference (rarely); the warp-wide vote on
+      // whether O needs rescaling waits until after the exponentials.
       float alpha = 1.f;
       if (j == jb) {
         m_run = rmax;  // -inf if this row's keys start in a later tile
-      } else if (__any_sync(0xffffffffu, rmax > m_run + kRescaleThreshold)) {
-        const float m_new = fmaxf(m_run, rmax);
-        // a row still fully masked (-inf - -inf) or unchanged keeps alpha = 1
-        alpha = m_new == m_run ? 1.f : ex2_approx(m_run - m_new);
-        m_run = m_new;
-        rescale = true;
+      } else if (rmax > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - rmax);  // 0 for a row fully masked so far (m_run = -inf)
+        m_run = rmax;
       }
       const float neg = m_run == -INFINITY ? 0.f : -m_run;  // fully masked so far: p = 0
       float ls[8];
@@ -382,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       l_run = fmaf(l_run, alpha, lsum);
-      if (rescale) {
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
         // P_t(j-1) V_(j-1) is complete (in-order MMAs): O_t may be rescaled.
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
