@@ -25,8 +25,10 @@ def prefill_flops(dims, T, halt_layer=None, K=None, mode="dense", active_idx=Non
 
     dense: every layer on T tokens.  prune: layers 0..halt_layer on T, later
     layers on K tokens with causal attention among them.  halt: later layers
-    run K queries against all visible keys (sum of active positions + 1) and
-    recompute the K/V projections of the T-K halted rows.
+    run K queries against all visible keys (sum of active positions + 1; K/T
+    of the causal pairs when the positions are not given, as for evenly
+    spread active rows) and recompute the K/V projections of the T-K halted
+    rows.
     """
     lin = linear_flops_per_token(dims)
     full = T * lin + attn_flops(dims, causal_pairs(T))
@@ -38,7 +40,7 @@ def prefill_flops(dims, T, halt_layer=None, K=None, mode="dense", active_idx=Non
     if mode == "prune":
         late = K * lin + attn_flops(dims, causal_pairs(K))
     else:
-        pairs = int(sum(int(i) + 1 for i in active_idx)) if active_idx is not None else causal_pairs(T) // 2
+        pairs = int(sum(int(i) + 1 for i in active_idx)) if active_idx is not None else causal_pairs(T) * K // T
         kvd = dims.n_kv_heads * dims.head_dim
         late = K * lin + attn_flops(dims, pairs) + (T - K) * 2 * dims.d_model * 2 * kvd
     return n_full * full + n_late * late
