@@ -139,6 +139,33 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _t(t, dtype, name, shape=None):
+    """Pointer to a contiguous CUDA tensor of `dtype` (None passes through).
+    The library takes row-major buffers whose sizes follow from the shape
+    arguments, so a strided view, another dtype or a host tensor is refused
+    here rather than read as something else.  `shape` entries that are None
+    are not checked."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        what = f"{tuple(t.shape)} {t.dtype} {t.device}{'' if t.is_contiguous() else ' strided'}" \
+            if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {what}")
+    if shape is not None and (t.dim() != len(shape) or any(w is not None and g != w for g, w in zip(t.shape, shape))):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _out(t, dtype, name, n):
+    """Pointer to an output buffer of at least n elements (None passes through)."""
+    if isinstance(t, torch.Tensor) and t.numel() < n:
+        raise ValueError(f"{name}: needs at least {n} elements, has {t.numel()}")
+    return _t(t, dtype, name)
+
+
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -189,7 +216,8 @@ def release_workspaces():
 def score(U, H=None, relative=False, out=None, stream=None):
     T, d = U.shape
     out = torch.empty(T, dtype=torch.float32, device=U.device) if out is None else out
-    _check(lib().dash_score(_p(U), _p(H), T, d, int(relative), _p(out), _stream(stream)), "dash_score")
+    _check(lib().dash_score(_t(U, BF16, "U"), _t(H, BF16, "H", (T, d)), T, d, int(relative),
+                            _t(out, F32, "out", (T,)), _stream(stream)), "dash_score")
     return out
 
 
@@ -205,7 +233,7 @@ def select(scores, kind="topk", keep=0.5, threshold=0.0, keep_first=0, keep_last
     idx = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
     halted = torch.empty(max(T, 1), dtype=torch.int32, device=dev) if want_halted else None
     count = torch.empty(1, dtype=torch.int32, device=dev)
-    _check(lib().dash_select(_p(scores), T, SELECTS[kind], keep, threshold, keep_first, keep_last, _p(idx),
+    _check(lib().dash_select(_t(scores, F32, "scores"), T, SELECTS[kind], keep, threshold, keep_first, keep_last, _p(idx),
                              _p(halted), _p(count), None, 0, _stream(stream)), "dash_select")
     n = int(count.item())
     if n < 0:
@@ -216,19 +244,21 @@ def select(scores, kind="topk", keep=0.5, threshold=0.0, keep_first=0, keep_last
 def compact(X, idx, stream=None):
     K = idx.numel()
     Y = torch.empty(K, X.shape[1], dtype=X.dtype, device=X.device)
-    _check(lib().dash_compact(_p(X), X.shape[0], _p(idx), K, X.shape[1], _p(Y), _stream(stream)), "dash_compact")
+    _check(lib().dash_compact(_t(X, BF16, "X"), X.shape[0], _t(idx, I32, "idx"), K, X.shape[1], _p(Y),
+                              _stream(stream)), "dash_compact")
     return Y
 
 
 def scatter(Y, idx, X, stream=None):
-    _check(lib().dash_scatter(_p(Y), _p(idx), idx.numel(), X.shape[1], _p(X), X.shape[0], _stream(stream)),
-           "dash_scatter")
+    _check(lib().dash_scatter(_t(Y, BF16, "Y", (idx.numel(), X.shape[1])), _t(idx, I32, "idx"), idx.numel(),
+                              X.shape[1], _t(X, BF16, "X"), X.shape[0], _stream(stream)), "dash_scatter")
     return X
 
 
 def rmsnorm(X, g, eps, stream=None):
     Y = torch.empty_like(X)
-    _check(lib().dash_rmsnorm(_p(X), X.shape[0], X.shape[1], _p(g), eps, _p(Y), _stream(stream)), "dash_rmsnorm")
+    _check(lib().dash_rmsnorm(_t(X, BF16, "X"), X.shape[0], X.shape[1], _t(g, BF16, "g", (X.shape[1],)), eps, _p(Y),
+                              _stream(stream)), "dash_rmsnorm")
     return Y
 
 
@@ -236,7 +266,8 @@ def linear(A, W, out=None, stream=None):
     M, K = A.shape
     N = W.shape[0]
     out = torch.empty(M, N, dtype=A.dtype, device=A.device) if out is None else out
-    _check(lib().dash_linear(_p(A), M, K, _p(W), N, _p(out), _stream(stream)), "dash_linear")
+    _check(lib().dash_linear(_t(A, BF16, "A"), M, K, _t(W, BF16, "W", (N, K)), N, _t(out, BF16, "out", (M, N)),
+                             _stream(stream)), "dash_linear")
     return out
 
 
@@ -248,14 +279,17 @@ def set_gemm_pairs(enable):
 
 def exp2_fma(x, stream=None):
     y = torch.empty_like(x)
-    _check(lib().dash_exp2_fma(_p(x), x.numel(), _p(y), _stream(stream)), "dash_exp2_fma")
+    _check(lib().dash_exp2_fma(_t(x, F32, "x"), x.numel(), _p(y), _stream(stream)), "dash_exp2_fma")
     return y
 
 
 def attention(Q, K, V, hq, hkv, hd, qpos=None, kstart=None, out=None, stream=None):
     M = Q.shape[0]
     out = torch.empty(M, hq * hd, dtype=Q.dtype, device=Q.device) if out is None else out
-    _check(lib().dash_attention(_p(Q), _p(K), _p(V), M, K.shape[0], hq, hkv, hd, _p(qpos), _p(kstart), _p(out),
+    T_kv = K.shape[0]
+    _check(lib().dash_attention(_t(Q, BF16, "Q", (M, hq * hd)), _t(K, BF16, "K", (T_kv, hkv * hd)),
+                                _t(V, BF16, "V", (T_kv, hkv * hd)), M, T_kv, hq, hkv, hd, _t(qpos, I32, "qpos", (M,)),
+                                _t(kstart, I32, "kstart", (M,)), _t(out, BF16, "out", (M, hq * hd)),
                                 _stream(stream)), "dash_attention")
     return out
 
@@ -290,6 +324,10 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
     if halt is not None:
         active, halted, h_full = halt
         T_kv = h_full.shape[0]
+        _t(active, I32, "active_idx", (M,))
+        _t(h_full, BF16, "h_full", (T_kv, H.shape[1]))
+        if halted.numel():
+            _t(halted, I32, "halted_idx", (T_kv - M,))
         hctx = HaltCtx(active.data_ptr(), halted.data_ptr() if halted.numel() else None, h_full.data_ptr(), T_kv)
         pos = active
     if max_pos is None:
@@ -297,8 +335,10 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
     need = lib().dash_layer_workspace_size(ctypes.byref(stack.dims), M, T_kv, max_pos)
     ws = workspace(need, H.device)
     w = ctypes.pointer(stack.layers[l])
-    _check(lib().dash_layer_forward(ctypes.byref(stack.dims), w, _p(H), M, _p(pos), max_pos,
-                                    ctypes.byref(hctx) if hctx is not None else None, _p(delta), int(relative),
+    _check(lib().dash_layer_forward(ctypes.byref(stack.dims), w, _t(H, BF16, "H", (M, stack.dims.d_model)),
+                                    M, _t(pos, I32, "pos", (M,)), max_pos,
+                                    ctypes.byref(hctx) if hctx is not None else None, _out(delta, F32, "delta", M),
+                                    int(relative),
                                     _p(ws), ws.numel(), _stream(stream)), "dash_layer_forward")
     return H
 
@@ -320,8 +360,9 @@ def prefill_varlen(stack, H, cu_seqlens, cfg, idx_out=None, delta_out=None, stre
     cu_arr = (c_i32 * (nseq + 1))(*cu)
     counts = (c_i32 * nseq)()
     K = c_i64(0)
-    _check(lib().dash_prefill_varlen(ctypes.byref(stack.dims), stack.layers, _p(H), cu_arr, nseq, ctypes.byref(cfg),
-                                     _p(idx_out), ctypes.byref(K), counts, _p(delta_out), _p(ws), ws.numel(),
+    _check(lib().dash_prefill_varlen(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)),
+                                     cu_arr, nseq, ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T),
+                                     ctypes.byref(K), counts, _out(delta_out, F32, "delta_out", T), _p(ws), ws.numel(),
                                      _stream(stream)), "dash_prefill_varlen")
     return K.value, list(counts)
 
@@ -332,8 +373,10 @@ def prefill(stack, H, cfg, idx_out=None, delta_out=None, stream=None):
     need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
     ws = workspace(need, H.device)
     K = c_i64(0)
-    _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _p(H), T, ctypes.byref(cfg), _p(idx_out),
-                              ctypes.byref(K), _p(delta_out), _p(ws), ws.numel(), _stream(stream)), "dash_prefill")
+    _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)), T,
+                              ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T), ctypes.byref(K),
+                              _out(delta_out, F32, "delta_out", T), _p(ws), ws.numel(), _stream(stream)),
+           "dash_prefill")
     return K.value
 
 
@@ -380,9 +423,10 @@ def prefill_kv(stack, H, cfg, cache, idx_out=None, delta_out=None, stream=None):
     need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
     ws = workspace(need, H.device)
     K = c_i64(0)
-    _check(lib().dash_prefill_kv(ctypes.byref(stack.dims), stack.layers, _p(H), T, ctypes.byref(cfg), _p(idx_out),
-                                 ctypes.byref(K), _p(delta_out), cache.desc, _p(ws), ws.numel(), _stream(stream)),
-           "dash_prefill_kv")
+    _check(lib().dash_prefill_kv(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)), T,
+                                 ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T), ctypes.byref(K),
+                                 _out(delta_out, F32, "delta_out", T), cache.desc, _p(ws), ws.numel(),
+                                 _stream(stream)), "dash_prefill_kv")
     return K.value
 
 
@@ -396,9 +440,11 @@ def prefill_varlen_kv(stack, H, cu_seqlens, cfg, cache, idx_out=None, delta_out=
     cu_arr = (c_i32 * (nseq + 1))(*cu)
     counts = (c_i32 * nseq)()
     K = c_i64(0)
-    _check(lib().dash_prefill_varlen_kv(ctypes.byref(stack.dims), stack.layers, _p(H), cu_arr, nseq,
-                                        ctypes.byref(cfg), _p(idx_out), ctypes.byref(K), counts, _p(delta_out),
-                                        cache.desc, _p(ws), ws.numel(), _stream(stream)), "dash_prefill_varlen_kv")
+    _check(lib().dash_prefill_varlen_kv(ctypes.byref(stack.dims), stack.layers,
+                                        _t(H, BF16, "H", (T, stack.dims.d_model)), cu_arr, nseq, ctypes.byref(cfg),
+                                        _out(idx_out, I32, "idx_out", T), ctypes.byref(K), counts,
+                                        _out(delta_out, F32, "delta_out", T), cache.desc, _p(ws), ws.numel(),
+                                        _stream(stream)), "dash_prefill_varlen_kv")
     return K.value, list(counts)
 
 
@@ -409,8 +455,8 @@ def decode_step(stack, X, pos, cache, stream=None):
     need = lib().dash_decode_workspace_size(ctypes.byref(stack.dims), n)
     ws = workspace(need, X.device)
     pos_arr = (c_i32 * n)(*[int(p) for p in pos])
-    _check(lib().dash_decode_step(ctypes.byref(stack.dims), stack.layers, _p(X), n, pos_arr, cache.desc, _p(ws),
-                                  ws.numel(), _stream(stream)), "dash_decode_step")
+    _check(lib().dash_decode_step(ctypes.byref(stack.dims), stack.layers, _t(X, BF16, "X", (n, stack.dims.d_model)),
+                                  n, pos_arr, cache.desc, _p(ws), ws.numel(), _stream(stream)), "dash_decode_step")
     return X
 
 
@@ -420,9 +466,12 @@ def decode_attention(Q, kv, hq, hkv, hd, out=None, stream=None):
     out = torch.empty_like(Q) if out is None else out
     desc = (KVCacheDesc * n)()
     for s, (k, v) in enumerate(kv):
+        _t(k, BF16, f"K[{s}]", (None, hkv * hd))
+        _t(v, BF16, f"V[{s}]", tuple(k.shape))
         desc[s] = KVCacheDesc(k.data_ptr(), v.data_ptr(), None, k.shape[0], k.shape[0])
     need = lib().dash_decode_attention_workspace_size(hd)
     ws = workspace(need, Q.device)
-    _check(lib().dash_decode_attention(_p(Q), n, desc, hq, hkv, hd, _p(out), _p(ws), ws.numel(), _stream(stream)),
+    _check(lib().dash_decode_attention(_t(Q, BF16, "Q", (n, hq * hd)), n, desc, hq, hkv, hd,
+                                       _t(out, BF16, "out", (n, hq * hd)), _p(ws), ws.numel(), _stream(stream)),
            "dash_decode_attention")
     return out

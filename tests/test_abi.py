@@ -172,3 +172,28 @@ def test_kv_cache_and_decode_argument_errors(L):
     assert att(2, 4, 2, 64, caches=_cache_arr(2, ln=0)) == 2               # an empty cache
     assert att(2, 4, 2, 64) == 4                                           # no workspace
     assert L.dash_decode_attention_workspace_size(64) > 0 and L.dash_decode_attention_workspace_size(80) == 0
+
+
+def test_binding_refuses_tensors_the_library_would_misread(L):
+    """The binding passes raw pointers, so it checks each tensor first: a host
+    tensor, another dtype, a strided view or a wrong shape raises ValueError
+    before any library call (no GPU needed for these refusals)."""
+    import torch
+    bf = torch.zeros(8, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        dash.score(bf)                                   # host memory
+    with pytest.raises(ValueError, match="CUDA"):
+        dash.linear(bf, torch.zeros(16, 256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        dash.compact(bf, torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        dash.attention(bf, bf, bf, 2, 1, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        dash.select(torch.zeros(10))
+    # dtype, stride and shape are checked the same way (shown on the helper itself)
+    for bad, why in [(torch.zeros(4, 6), "float32"), (bf.t(), "strided"), (bf, "CUDA")]:
+        with pytest.raises(ValueError, match=why):
+            dash._t(bad, torch.bfloat16, "x")
+    assert dash._t(None, torch.bfloat16, "x") is None
+    with pytest.raises(ValueError, match="at least 9"):
+        dash._out(torch.zeros(8, dtype=torch.int32), torch.int32, "idx_out", 9)
