@@ -2,6 +2,7 @@
 exports every symbol the headers declare, and its host-side arithmetic and
 argument checks behave (no kernel is launched by any call here)."""
 import ctypes
+import os
 import math
 
 import pytest
@@ -197,3 +198,30 @@ def test_binding_refuses_tensors_the_library_would_misread(L):
     assert dash._t(None, torch.bfloat16, "x") is None
     with pytest.raises(ValueError, match="at least 9"):
         dash._out(torch.zeros(8, dtype=torch.int32), torch.int32, "idx_out", 9)
+
+
+def test_headers_compile_and_link_as_plain_c(L, tmp_path):
+    """The ABI is usable from C: both headers compile as strict C99, and a C
+    program linked against libdash.so calls two host-only entry points."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi_user.c"
+    src.write_text(
+        '#include "dash.h"\n#include "dash_ops.h"\n#include <stdio.h>\n#include <string.h>\n'
+        "int main(void) {\n"
+        "  const char* s = dash_status_string(DASH_OK);\n"
+        "  long long k = (long long)dash_topk_count(1000, 0.5, 64, 32);\n"
+        '  printf("%s %lld\\n", s, k);\n'
+        "  return (s != NULL && strlen(s) > 0 && k == 64 + 32 + 452) ? 0 : 1;\n"
+        "}\n")
+    exe = tmp_path / "abi_user"
+    libdir = os.path.dirname(build.LIB)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", build.INCLUDE,
+                        str(src), "-o", str(exe), "-L", libdir, "-l:libdash.so", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
