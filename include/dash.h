@@ -224,9 +224,11 @@ dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* 
  * is a deployment convenience.
  *   - Shapes whose workspace (dash_layer_workspace_size) exceeds 32 MiB are
  *     rejected with DASH_ERR_NO_MEMORY before anything is launched.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing), so the address stays
+ *     right after a device reset.  The first call on a device may load the
+ *     library's device code there; make that first call before any stream
+ *     capture.
  *   - Every call shares the one array and leaves its contents behind; no
  *     part of it needs to start at zero (each call writes every byte it
  *     reads).  Calls whose executions overlap on the GPU (other streams,

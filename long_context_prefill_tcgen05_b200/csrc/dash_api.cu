@@ -374,6 +374,7 @@ struct LayerWs {
   float* ssq_u;  // [o_proj tiles, M]
   float* ssq_h;
   float* rs;     // [max(M, T_kv - M)] RMSNorm 1/rms per row, applied in the GEMM epilogues
+  int64_t rope_rows;  // positions held by the RoPE table
 };
 
 bool dims_ok(const dash_dims* D) {
@@ -391,6 +392,7 @@ void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, C
   const int64_t d = D.d_model, qd = static_cast<int64_t>(D.n_heads) * D.head_dim;
   const int64_t kvd = static_cast<int64_t>(D.n_kv_heads) * D.head_dim, F = D.ffn_dim;
   w.rope = c.take<float2>(static_cast<size_t>(max_pos) * (D.head_dim / 2));
+  w.rope_rows = max_pos;
   w.X = c.take<bf16>(static_cast<size_t>(M) * (d > qd ? d : qd));
   w.Q = c.take<bf16>(static_cast<size_t>(M) * qd);
   w.Kb = c.take<bf16>(static_cast<size_t>(T_kv) * kvd);
@@ -427,6 +429,8 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   qkv.hq = hq;
   qkv.hkv = hkv;
   qkv.hd = hd;
+  qkv.rope_rows = ws.rope_rows;
+  qkv.kv_rows = T_kv;
 
   // Keys / values of the halted rows, from their frozen states, at their
   // original positions ([DASH news] "选择性停止机制").
@@ -561,20 +565,14 @@ dash_status seq_layout(const int32_t* cu, int nseq, const int32_t* rows, int64_t
 // host-side stand-in; its device address comes from cudaGetSymbolAddress.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-void* g_noalloc_ptr[kMaxDevices];
 
-// Device address of g_noalloc_scratch for the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of g_noalloc_scratch on the current device, looked up on
+// every call (cheap; allocates nothing), so it stays valid across a device
+// reset or a re-created primary context.
 dash_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DASH_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DASH_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DASH_ERR_CUDA;
+  *out = p;
   return DASH_OK;
 }
 

@@ -48,6 +48,8 @@ struct EpiArgs {
   const float* row_scale;    // [M] or NULL: per-row factor on the accumulator (RMSNorm 1/rms)
   int col_offset;            // qkv column of this GEMM's column 0
   int hq, hkv, hd;
+  int64_t rope_rows;         // kEpiQkv: positions in the RoPE table (pos must lie in [0, rope_rows))
+  int64_t kv_rows;           // kEpiQkv: rows of the k / v buffers (kv rows must lie in [0, kv_rows))
 };
 
 struct Shape {
@@ -159,9 +161,17 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
     const int hd = ep.hd, half = hd >> 1;
     int p = 0, kvrow = 0;
     float sc = 1.f;
-    if (live) {
+    bool ok = live;
+    if (ok) {
       p = ep.pos ? ep.pos[m] : m;
       kvrow = ep.kv_rowmap ? ep.kv_rowmap[m] : m;
+      // Caller-supplied positions index the RoPE table and row maps pick the
+      // k / v row written: a row with either out of range is flagged and
+      // left unwritten.
+      if (p < 0 || p >= ep.rope_rows || kvrow < 0 || kvrow >= ep.kv_rows) {
+        flag_error(kDevErrIndex);
+        ok = false;
+      }
       if (ep.row_scale) sc = ep.row_scale[m];
     }
 #pragma unroll 1
@@ -185,7 +195,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
           tmem_ld32(tb + c, x1);
           tmem_ld32(tb + half + c, x2);
           tmem_ld_wait();
-          if (live) {
+          if (ok) {
             const float4* cs = ep.rope + ((static_cast<int64_t>(p) * half + c) >> 1);
             float y1[32], y2[32];
 #pragma unroll
@@ -208,7 +218,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
           uint32_t r[32];
           tmem_ld32(tb + c, r);
           tmem_ld_wait();
-          if (live) {
+          if (ok) {
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]) * sc;

@@ -113,6 +113,30 @@ def test_layer_halt_context(tiny):
     assert _rel(delta.cpu().numpy(), O.delta_scores(u)) < DELTA_TOL
 
 
+def test_layer_halt_context_bad_active_index_is_flagged(tiny):
+    """An active index past the sequence would address the RoPE table and the
+    k / v rows out of range: the QKV epilogue leaves that row unwritten and
+    reports INDEX; the context stays usable."""
+    dims, h0, stack, L = tiny
+    T = 512
+    idx = np.arange(0, T, 4)
+    halted = np.setdiff1d(np.arange(T), idx)
+    bad = idx.copy()
+    bad[-1] = T + 5  # ascending, but out of range
+    ti = torch.tensor(bad, dtype=torch.int32, device=DEV)
+    th = torch.tensor(halted, dtype=torch.int32, device=DEV)
+    hf = h0.to(DEV)
+    H = hf[torch.tensor(idx, device=DEV).long()].contiguous()
+    dash.layer_forward(stack, 3, H, halt=(ti, th, hf))
+    assert dash.device_error() == 7  # reported and cleared
+    good = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    H = hf[good.long()].contiguous()
+    dash.layer_forward(stack, 3, H, halt=(good, th, hf))
+    assert dash.device_error() == 0
+    ref, _ = O.decoder_block(to_np(h0)[idx], idx, to_np(h0), np.arange(T), L[3], dims.as_dict())
+    assert row_rel_err(to_np(H), ref) < HIDDEN_TOL
+
+
 # ----------------------------------------------------------- tiny prefill
 @pytest.mark.parametrize("mode", ["prune", "halt"])
 @pytest.mark.parametrize("keep,nf,nl", [(0.5, 0, 0), (0.3, 64, 32)])
