@@ -24,8 +24,10 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; a call returns before the GPU finishes unless
  *     its comment says it synchronises.
- *   - Activations and weights are bf16 (raw bit patterns, dash_bf16),
- *     row-major; scores fp32; token indices int32.
+ *   - Activations, weights and K/V caches are 16-bit floats (raw bit
+ *     patterns, dash_bf16) in the model's format, dash_dims.dtype: bf16 (the
+ *     default) or fp16; row-major.  Entry points without a dash_dims
+ *     argument take bf16.  Scores are fp32, token indices int32.
  *   - Faults found on the device (a bounded wait that gave up, an index out
  *     of range, a non-finite score) set a sticky device error word instead of
  *     trapping; dash_device_error() reads and clears it.  While it is set,
@@ -41,7 +43,7 @@
 extern "C" {
 #endif
 
-typedef uint16_t dash_bf16; /* bf16 bit pattern */
+typedef uint16_t dash_bf16; /* 16-bit float bit pattern: bf16, or fp16 where dash_dims.dtype says so */
 
 typedef enum dash_status {
   DASH_OK = 0,
@@ -53,6 +55,18 @@ typedef enum dash_status {
   DASH_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
   DASH_ERR_INDEX = 7        /* an index list entry out of range */
 } dash_status;
+
+/* 16-bit float format of a model's activations, weights and K/V caches.
+ * Both run on the same tensor-core instructions at the same rate, with fp32
+ * accumulation.  bf16 keeps fp32's exponent range with 8 significant bits;
+ * fp16 has 11 significant bits (8x less rounding per stored value) but holds
+ * magnitudes up to 65504 only.  A value past that range stored as fp16
+ * becomes Inf; nothing checks for it, except that a non-finite Δ score is
+ * reported as DASH_ERR_NONFINITE. */
+typedef enum dash_dtype {
+  DASH_DTYPE_BF16 = 0,
+  DASH_DTYPE_F16 = 1
+} dash_dtype;
 
 /* Decoder-stack dimensions.  Supported: head_dim 64 or 128; d_model and
  * n_heads*head_dim multiples of 128 (d_model <= 4096); ffn_dim a multiple
@@ -66,11 +80,13 @@ typedef struct dash_dims {
   int32_t ffn_dim;    /* F */
   double rms_eps;     /* RMSNorm epsilon */
   double rope_theta;  /* RoPE base θ (rotate-half pairs (i, i + hd/2)) */
+  int32_t dtype;      /* dash_dtype of every 16-bit array the call passes (0 = bf16) */
 } dash_dims;
 
 /* Weights of one pre-norm decoder block ([DASH blog] §2.1: norm ->
  * attention -> U, H' = H + U; then norm -> SwiGLU FFN -> residual).
- * All bf16, row-major [out_features, in_features], no biases. */
+ * All in the model's 16-bit format, row-major [out_features, in_features],
+ * no biases. */
 typedef struct dash_layer_weights {
   const dash_bf16* attn_norm; /* [d] RMSNorm gain before attention */
   const dash_bf16* w_qkv;     /* [(hq + 2*hkv)*hd, d]: q heads, then k heads, then v heads */
@@ -165,7 +181,8 @@ dash_status dash_select(const float* scores, int64_t T, int32_t kind, double kee
 
 /* ------------------------------------------------------ compact/scatter --
  * Gather of the active rows ([DASH blog] §3.1 "复用活跃集合"):
- * Y[i, :] = X[idx[i], :] for i < K.  X: [T, d], Y: [K, d] bf16, d % 8 == 0.
+ * Y[i, :] = X[idx[i], :] for i < K.  X: [T, d], Y: [K, d] 16-bit elements
+ * (either format: rows are copied bit for bit), d % 8 == 0.
  * An idx entry outside [0, T) sets the INDEX device error; its row is not
  * written. */
 dash_status dash_compact(const dash_bf16* X, int64_t T, const int32_t* idx, int64_t K,
@@ -249,7 +266,7 @@ size_t dash_prefill_workspace_size(const dash_dims* dims, int64_t T, const dash_
  * update gives Δ (fused into its o_proj epilogue); the active set is
  * selected once and reused by every later layer.
  *   layers:    [dims->n_layers] weights.
- *   H:         [T, d] bf16 in: input hidden states; out: prune -> rows
+ *   H:         [T, d] (model format) in: input hidden states; out: prune -> rows
  *              0..K-1 hold the active tokens' final states (rest undefined);
  *              halt / dense -> all T rows (halted rows frozen at the halting
  *              layer's output).
@@ -329,7 +346,7 @@ size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq);
 
 /* One generation step: one new token for each of nseq (<= DASH_DECODE_MAX_SEQ)
  * sequences runs through every layer.
- *   X      [nseq, d_model] bf16: the new tokens' input hidden states; on
+ *   X      [nseq, d_model] (model format): the new tokens' input hidden states; on
  *          return the hidden states after the last layer (no final norm).
  *   pos    HOST [nseq]: RoPE position of each new token; it must exceed
  *          every position already in that sequence's cache (the token

@@ -25,8 +25,8 @@
 //               thread (TMEM lane = row); S_j is read from TMEM, the running
 //               max / sum kept in registers, O rescaled in TMEM only when the
 //               max grows by more than 2^8 (exact: l and O share the stale
-//               reference), and P_j written back to TMEM as packed bf16 pairs
-//               over the upper half of S_j, where the P*V MMA reads it as its
+//               reference), and P_j written back to TMEM as packed 16-bit
+//               pairs (the model's format, DT) over the upper half of S_j, where the P*V MMA reads it as its
 //               A operand.
 // TMEM columns: S0/P0 [0,128) S1/P1 [128,256) O0 [256,384) O1 [384,512).
 // MMAs issued by one thread complete in order, so the commit that signals
@@ -58,7 +58,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kEmuPeriod = DASH_ATTN_EMU_PERIOD;
 
 struct Params {
-  __nv_bfloat16* out;  // [M, hq*hd]
+  s16* out;  // [M, hq*hd]
   int64_t ldo;
   const int32_t* qpos;    // [M] or NULL
   const int32_t* kstart;  // [M] or NULL (non-decreasing)
@@ -92,10 +92,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // bits) and f in [-0.5, 0.5]; 2^f by a cubic whose coefficients were fitted
 // here to minimise the relative error on [-0.5, 0.5] (iteratively reweighted
 // least squares on Chebyshev nodes; max relative error 7.5e-5 in fp32, far
-// below bf16's 3.9e-3); 2^j is added to the exponent field.  Inputs are
+// below the 16-bit P's rounding); 2^j is added to the exponent field.  Inputs are
 // clamped at -125 so the exponent add stays within normal numbers (j <= -127
 // would wrap into the sign bit); fully masked scores give ~2e-38 instead of 0,
-// negligible next to any bf16 weight.
+// negligible next to any stored weight.
 __device__ __forceinline__ float ex2_fma(float x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   x = fmaxf(x, -125.0f);
@@ -105,7 +105,7 @@ __device__ __forceinline__ float ex2_fma(float x) {
   return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -126,7 +126,7 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-template <int HD>
+template <int HD, int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const Params p) {
@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     {  // converged warp; elected lanes issue
-      const uint32_t idesc_s = umma_idesc_bf16(BQ, BKV, false, false);
-      const uint32_t idesc_o = umma_idesc_bf16(BQ, HD, false, true);
+      const uint32_t idesc_s = umma_idesc<DT>(BQ, BKV, false, false);
+      const uint32_t idesc_o = umma_idesc<DT>(BQ, HD, false, true);
       // Descriptors are built once and advanced by adding (byte offset >> 4)
       // to the start-address field.
       const uint64_t qdesc0 = umma_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < HD / 16; ++kk) {
           constexpr int kPanelStep = (BQ * 128) >> 4;
           const int off = (kk >> 2) * kPanelStep + (kk & 3) * 2;  // (panel, 32-byte column step) >> 4
-          umma_bf16_ss_elect(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+          umma_ss_elect(tmem_base + t * BKV, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit_elect(bar_sfull + 8 * t);
       };
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                ? ex2_fma(x1)  // FMA pipe
                                : ex2_approx(x1);
           ls[i & 7] += e0 + e1;
-          pk[i] = pack_bf16(e0, e1);
+          pk[i] = Num<DT>::pack(e0, e1);
         }
         tmem_st32(s_addr + BKV / 2 + 32 * half, pk);
       }
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__all_sync(0xffffffffu, ok && n > jb && mbar_wait(bar_odone + 8 * t, 0))) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      __nv_bfloat16* dst = p.out + static_cast<int64_t>(mrow) * p.ldo + head * HD;
+      s16* dst = p.out + static_cast<int64_t>(mrow) * p.ldo + head * HD;
 #pragma unroll 1
       for (int c = 0; c < HD; c += 32) {
         uint32_t o[32];
@@ -411,10 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
-            w.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-            w.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-            w.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-            w.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+            w.x = Num<DT>::pack(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+            w.y = Num<DT>::pack(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+            w.z = Num<DT>::pack(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+            w.w = Num<DT>::pack(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
             d4[i] = w;
           }
         }

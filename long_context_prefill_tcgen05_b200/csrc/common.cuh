@@ -1,5 +1,5 @@
-// Device helpers shared by the sm_100a kernels of libdash: bf16 packing,
-// bounded mbarrier waits, TMA tile loads, and tcgen05 (TMEM / UMMA) wrappers.
+// Device helpers shared by the sm_100a kernels of libdash: 16-bit float
+// formats, bounded mbarrier waits, TMA tile loads, and tcgen05 (TMEM / UMMA) wrappers.
 //
 // Every spin-wait here is bounded: after kWaitLimitNs of wall-clock time (or
 // as soon as another thread has flagged an error) it records an error bit in
@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,13 +40,49 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// ------------------------------------------------------------ bf16 helpers
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&b);
-}
+// ------------------------------------------------------ 16-bit float formats
+// Activations, weights and K/V caches are 16-bit floats of one format per
+// model: bf16 (8 significant bits, fp32's exponent range; the default) or
+// fp16 (11 significant bits, range +-65504).  Both feed the same tcgen05
+// kind::f16 MMA at the same rate.  Kernels move them as raw 16-bit storage
+// (s16) and take the format as the template parameter DT.
+using s16 = uint16_t;
+enum : int { kBf16 = 0, kF16 = 1 };
+
+template <int DT>
+struct Num;
+template <>
+struct Num<kBf16> {
+  static constexpr uint32_t kUmmaFmt = 1;  // A/B format code of a kind::f16 instruction descriptor
+  static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // low / high element of a packed pair, widened exactly
+  __device__ static __forceinline__ float lo(uint32_t v) { return __uint_as_float(v << 16); }
+  __device__ static __forceinline__ float hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+  __device__ static __forceinline__ float to_f(s16 v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
+  // round to nearest even
+  __device__ static __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+  }
+  __device__ static __forceinline__ s16 from_f(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+};
+template <>
+struct Num<kF16> {
+  static constexpr uint32_t kUmmaFmt = 0;
+  static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  __device__ static __forceinline__ float lo(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xffffu)));
+  }
+  __device__ static __forceinline__ float hi(uint32_t v) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+  }
+  __device__ static __forceinline__ float to_f(s16 v) { return __half2float(__ushort_as_half(v)); }
+  __device__ static __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ static __forceinline__ s16 from_f(float f) { return __half_as_ushort(__float2half_rn(f)); }
+};
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -155,18 +192,20 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulate.
-// a_mn / b_mn select MN-major (transposed) operands.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4)                                   // D format fp32
-         | (1u << 7)                                 // A format bf16
-         | (1u << 10)                                // B format bf16
+// Instruction descriptor for kind::f16 with A and B of format DT (both the
+// same: bf16 or fp16) and fp32 accumulate.  a_mn / b_mn select MN-major
+// (transposed) operands.
+template <int DT>
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                           // D format fp32
+         | (Num<DT>::kUmmaFmt << 7)          // A format
+         | (Num<DT>::kUmmaFmt << 10)         // B format
          | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -177,7 +216,7 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, ui
 }
 // Forms for a converged warp: elect.sync picks one lane, which alone issues
 // the MMA / commit (every lane of the warp must execute them).
-__device__ __forceinline__ void umma_bf16_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                    uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
@@ -253,7 +292,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-__device__ __forceinline__ void umma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                   uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"

@@ -20,7 +20,10 @@
 
 namespace {
 
-using bf16 = __nv_bfloat16;
+using dash::kBf16;
+using dash::kF16;
+using dash::Num;
+using dash::s16;
 using dash::attn::attn_kernel;
 using dash::gemm::EpiArgs;
 using dash::gemm::gemm_kernel;
@@ -62,7 +65,7 @@ dash_status device_info(DeviceInfo** out) {
 }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
-inline const bf16* cb(const dash_bf16* p) { return reinterpret_cast<const bf16*>(p); }
+inline const s16* cb(const dash_bf16* p) { return reinterpret_cast<const s16*>(p); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline dash_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
@@ -121,39 +124,41 @@ class TimedLaunch {
   int idx_ = -1;
 };
 
-// 2D bf16 tensor map with a 64-element (128-byte) inner box and 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
-              uint32_t box_rows) {
+// 2D tensor map of 16-bit elements (format dt) with a 64-element (128-byte)
+// inner box and 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
+              CUtensorMapDataType dt) {
   if (!aligned16(base) || (ld * 2) % 16 != 0 || rows == 0 || cols % 64 != 0) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {ld * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t es[2] = {1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------- GEMM
-template <int BN, int EPI>
-dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
-                        const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
+template <int BN, int EPI, int DT>
+dash_status launch_gemm(const DeviceInfo& di, const s16* A, int64_t lda, int64_t M, int K, const s16* B,
+                        const s16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
   using C = dash::gemm::Cfg<BN>;
   if (M == 0) return DASH_OK;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(gemm_kernel<BN, EPI, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  constexpr CUtensorMapDataType kMt = Num<DT>::kMapType;
   CUtensorMap ma, mb, mb2;
-  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM)) return DASH_ERR_INVALID_ARG;
+  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM, kMt)) return DASH_ERR_INVALID_ARG;
   if (EPI == dash::gemm::kEpiSwiglu) {
-    if (!make_map(&mb, B, N / 2, K, K, BN / 2) || !make_map(&mb2, B2, N / 2, K, K, BN / 2))
+    if (!make_map(&mb, B, N / 2, K, K, BN / 2, kMt) || !make_map(&mb2, B2, N / 2, K, K, BN / 2, kMt))
       return DASH_ERR_INVALID_ARG;
   } else {
-    if (!make_map(&mb, B, N, K, K, BN)) return DASH_ERR_INVALID_ARG;
+    if (!make_map(&mb, B, N, K, K, BN, kMt)) return DASH_ERR_INVALID_ARG;
     mb2 = mb;
   }
   dash::gemm::Shape sh;
@@ -165,7 +170,7 @@ dash_status launch_gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_
   sh.num_tiles = sh.tiles_m * sh.tiles_n;
   const int grid = sh.num_tiles < di.num_sms ? sh.num_tiles : di.num_sms;
   TimedLaunch tl(kind, M, N, K, st);
-  gemm_kernel<BN, EPI><<<grid, dash::gemm::kThreads, C::kSmemBytes, st>>>(ma, mb, mb2, sh, ep);
+  gemm_kernel<BN, EPI, DT><<<grid, dash::gemm::kThreads, C::kSmemBytes, st>>>(ma, mb, mb2, sh, ep);
   return launch_status();
 }
 
@@ -174,10 +179,10 @@ std::atomic<int> g_gemm_pairs{1};
 
 // How many pairs of this kernel the device runs at once (0: none, e.g. the
 // attribute or the occupancy query failed; the single-SM kernel is used).
-template <int EPI>
+template <int EPI, int DT>
 int gemm_pair_capacity(const DeviceInfo& di) {
   using C = dash::gemm::PairCfg;
-  auto kernel = dash::gemm::gemm_pair_kernel<EPI>;
+  auto kernel = dash::gemm::gemm_pair_kernel<EPI, DT>;
   static std::once_flag once;
   static int max_pairs = 0;
   std::call_once(once, [&] {
@@ -201,19 +206,20 @@ int gemm_pair_capacity(const DeviceInfo& di) {
   return max_pairs;
 }
 
-template <int EPI>
-dash_status launch_gemm_pair(int max_pairs, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
-                             const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
+template <int EPI, int DT>
+dash_status launch_gemm_pair(int max_pairs, const s16* A, int64_t lda, int64_t M, int K, const s16* B,
+                             const s16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
   using C = dash::gemm::PairCfg;
-  auto kernel = dash::gemm::gemm_pair_kernel<EPI>;
+  auto kernel = dash::gemm::gemm_pair_kernel<EPI, DT>;
   if (M == 0) return DASH_OK;
+  constexpr CUtensorMapDataType kMt = Num<DT>::kMapType;
   CUtensorMap ma, mb, mb2;
-  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM)) return DASH_ERR_INVALID_ARG;
+  if (!make_map(&ma, A, M, K, lda, dash::gemm::BM, kMt)) return DASH_ERR_INVALID_ARG;
   if (EPI == dash::gemm::kEpiSwiglu) {
-    if (!make_map(&mb, B, N / 2, K, K, C::BN / 2) || !make_map(&mb2, B2, N / 2, K, K, C::BN / 2))
+    if (!make_map(&mb, B, N / 2, K, K, C::BN / 2, kMt) || !make_map(&mb2, B2, N / 2, K, K, C::BN / 2, kMt))
       return DASH_ERR_INVALID_ARG;
   } else {
-    if (!make_map(&mb, B, N, K, K, C::BN / 2)) return DASH_ERR_INVALID_ARG;
+    if (!make_map(&mb, B, N, K, K, C::BN / 2, kMt)) return DASH_ERR_INVALID_ARG;
     mb2 = mb;
   }
   dash::gemm::Shape sh;
@@ -241,9 +247,9 @@ dash_status launch_gemm_pair(int max_pairs, const bf16* A, int64_t lda, int64_t 
   return launch_status();
 }
 
-template <int EPI>
-dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, int K, const bf16* B,
-                 const bf16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind, int* bn_used = nullptr) {
+template <int EPI, int DT>
+dash_status gemm(const DeviceInfo& di, const s16* A, int64_t lda, int64_t M, int K, const s16* B,
+                 const s16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind, int* bn_used = nullptr) {
   if (K % dash::gemm::BK != 0 || M > INT32_MAX) return DASH_ERR_SHAPE;
   // SwiGLU tiles hold BN/2 gate + BN/2 up columns, so N = 2F must split into
   // whole tiles on both halves.
@@ -252,14 +258,14 @@ dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, in
   if (can256) {
     if (bn_used) *bn_used = 256;
     if (M > dash::gemm::BM && g_gemm_pairs.load(std::memory_order_relaxed)) {
-      const int pairs = gemm_pair_capacity<EPI>(di);
-      if (pairs > 0) return launch_gemm_pair<EPI>(pairs, A, lda, M, K, B, B2, N, ep, st, kind);
+      const int pairs = gemm_pair_capacity<EPI, DT>(di);
+      if (pairs > 0) return launch_gemm_pair<EPI, DT>(pairs, A, lda, M, K, B, B2, N, ep, st, kind);
     }
-    return launch_gemm<256, EPI>(di, A, lda, M, K, B, B2, N, ep, st, kind);
+    return launch_gemm<256, EPI, DT>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
   if (can128) {
     if (bn_used) *bn_used = 128;
-    return launch_gemm<128, EPI>(di, A, lda, M, K, B, B2, N, ep, st, kind);
+    return launch_gemm<128, EPI, DT>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
   return DASH_ERR_SHAPE;
 }
@@ -267,22 +273,23 @@ dash_status gemm(const DeviceInfo& di, const bf16* A, int64_t lda, int64_t M, in
 inline int o_proj_tiles(int d) { return d % 256 == 0 ? d / 256 : d / 128; }
 
 // -------------------------------------------------------------- attention
-template <int HD>
-dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
-                           int64_t T_kv, int hq, int hkv, const int32_t* qpos, const int32_t* kstart, bf16* O,
+template <int HD, int DT>
+dash_status launch_attn_hd(const s16* Q, int64_t ldq, const s16* K, const s16* V, int64_t ldkv, int64_t M,
+                           int64_t T_kv, int hq, int hkv, const int32_t* qpos, const int32_t* kstart, s16* O,
                            int64_t ldo, cudaStream_t st) {
   using C = dash::attn::Cfg<HD>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(attn_kernel<HD, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, M, static_cast<uint64_t>(hq) * HD, ldq, dash::attn::BQ) ||
-      !make_map(&mk, K, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV) ||
-      !make_map(&mv, V, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV))
+  constexpr CUtensorMapDataType kMt = Num<DT>::kMapType;
+  if (!make_map(&mq, Q, M, static_cast<uint64_t>(hq) * HD, ldq, dash::attn::BQ, kMt) ||
+      !make_map(&mk, K, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV, kMt) ||
+      !make_map(&mv, V, T_kv, static_cast<uint64_t>(hkv) * HD, ldkv, dash::attn::BKV, kMt))
     return DASH_ERR_INVALID_ARG;
   dash::attn::Params p;
   p.out = O;
@@ -298,34 +305,36 @@ dash_status launch_attn_hd(const bf16* Q, int64_t ldq, const bf16* K, const bf16
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
   const int64_t grid = static_cast<int64_t>(p.n_qblocks) * hq;
   TimedLaunch tl(DASH_K_ATTENTION, M, T_kv, (qpos || kstart) ? -1 : M * (M + 1) / 2, st);
-  attn_kernel<HD><<<static_cast<unsigned>(grid), dash::attn::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+  attn_kernel<HD, DT><<<static_cast<unsigned>(grid), dash::attn::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
   return launch_status();
 }
 
-dash_status attention(const bf16* Q, int64_t ldq, const bf16* K, const bf16* V, int64_t ldkv, int64_t M,
-                      int64_t T_kv, int hq, int hkv, int hd, const int32_t* qpos, const int32_t* kstart, bf16* O,
+template <int DT>
+dash_status attention(const s16* Q, int64_t ldq, const s16* K, const s16* V, int64_t ldkv, int64_t M,
+                      int64_t T_kv, int hq, int hkv, int hd, const int32_t* qpos, const int32_t* kstart, s16* O,
                       int64_t ldo, cudaStream_t st) {
   if (M == 0) return DASH_OK;
   if (T_kv <= 0 || M > INT32_MAX || T_kv > INT32_MAX || hkv <= 0 || hq % hkv != 0) return DASH_ERR_SHAPE;
-  if (hd == 128) return launch_attn_hd<128>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
-  if (hd == 64) return launch_attn_hd<64>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
+  if (hd == 128) return launch_attn_hd<128, DT>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
+  if (hd == 64) return launch_attn_hd<64, DT>(Q, ldq, K, V, ldkv, M, T_kv, hq, hkv, qpos, kstart, O, ldo, st);
   return DASH_ERR_SHAPE;
 }
 
 // ---------------------------------------------------------------- row ops
-dash_status rmsnorm(const bf16* X, int64_t x_rows, const int32_t* rowmap, int64_t rows, int d, const bf16* g,
-                    double eps, bf16* Y, cudaStream_t st, float* row_scale = nullptr) {
+template <int DT>
+dash_status rmsnorm(const s16* X, int64_t x_rows, const int32_t* rowmap, int64_t rows, int d, const s16* g,
+                    double eps, s16* Y, cudaStream_t st, float* row_scale = nullptr) {
   if (rows == 0) return DASH_OK;
   // 4-warp blocks, one row per warp
   constexpr int kWarps = 4;
   const int64_t blocks = (rows + kWarps - 1) / kWarps;
   TimedLaunch tl(DASH_K_RMSNORM, rows, d, 0, st);
-  dash::rows::rmsnorm_kernel<<<static_cast<unsigned>(blocks), 32 * kWarps, static_cast<size_t>(d) * sizeof(bf16),
+  dash::rows::rmsnorm_kernel<DT><<<static_cast<unsigned>(blocks), 32 * kWarps, static_cast<size_t>(d) * sizeof(s16),
                                st>>>(X, x_rows, rowmap, rows, d, g, static_cast<float>(eps), Y, row_scale);
   return launch_status();
 }
 
-dash_status move_rows(bool scatter, const bf16* src, bf16* dst, const int32_t* idx, int64_t K, int64_t T, int d,
+dash_status move_rows(bool scatter, const s16* src, s16* dst, const int32_t* idx, int64_t K, int64_t T, int d,
                       const DeviceInfo& di, cudaStream_t st) {
   if (K == 0) return DASH_OK;
   const int warps = 8;
@@ -366,11 +375,11 @@ struct Carver {
 
 struct LayerWs {
   float2* rope;  // [max_pos, hd/2]
-  bf16* X;       // [M, max(d, hq*hd)]: norm output, then attention output
-  bf16* Q;       // [M, hq*hd]
-  bf16* Kb;      // [T_kv, hkv*hd]
-  bf16* Vb;      // [T_kv, hkv*hd]
-  bf16* Act;     // [max(M*F, (T_kv-M)*d)]: SwiGLU output; halt-mode frozen-row norms
+  s16* X;       // [M, max(d, hq*hd)]: norm output, then attention output
+  s16* Q;       // [M, hq*hd]
+  s16* Kb;      // [T_kv, hkv*hd]
+  s16* Vb;      // [T_kv, hkv*hd]
+  s16* Act;     // [max(M*F, (T_kv-M)*d)]: SwiGLU output; halt-mode frozen-row norms
   float* ssq_u;  // [o_proj tiles, M]
   float* ssq_h;
   float* rs;     // [max(M, T_kv - M)] RMSNorm 1/rms per row, applied in the GEMM epilogues
@@ -385,6 +394,7 @@ bool dims_ok(const dash_dims* D) {
   if (hq % hkv != 0) return false;
   if (d % 128 != 0 || d > 4096 || F % 64 != 0 || (hq * hd) % 128 != 0) return false;
   if (!(D->rms_eps >= 0.0) || !(D->rope_theta > 0.0)) return false;
+  if (D->dtype != DASH_DTYPE_BF16 && D->dtype != DASH_DTYPE_F16) return false;
   return true;
 }
 
@@ -393,12 +403,12 @@ void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, C
   const int64_t kvd = static_cast<int64_t>(D.n_kv_heads) * D.head_dim, F = D.ffn_dim;
   w.rope = c.take<float2>(static_cast<size_t>(max_pos) * (D.head_dim / 2));
   w.rope_rows = max_pos;
-  w.X = c.take<bf16>(static_cast<size_t>(M) * (d > qd ? d : qd));
-  w.Q = c.take<bf16>(static_cast<size_t>(M) * qd);
-  w.Kb = c.take<bf16>(static_cast<size_t>(T_kv) * kvd);
-  w.Vb = c.take<bf16>(static_cast<size_t>(T_kv) * kvd);
+  w.X = c.take<s16>(static_cast<size_t>(M) * (d > qd ? d : qd));
+  w.Q = c.take<s16>(static_cast<size_t>(M) * qd);
+  w.Kb = c.take<s16>(static_cast<size_t>(T_kv) * kvd);
+  w.Vb = c.take<s16>(static_cast<size_t>(T_kv) * kvd);
   const int64_t act = M * F > (T_kv - M) * d ? M * F : (T_kv - M) * d;
-  w.Act = c.take<bf16>(static_cast<size_t>(act));
+  w.Act = c.take<s16>(static_cast<size_t>(act));
   const int nt = o_proj_tiles(D.d_model);
   w.ssq_u = c.take<float>(static_cast<size_t>(nt) * M);
   w.ssq_h = c.take<float>(static_cast<size_t>(nt) * M);
@@ -409,7 +419,8 @@ void carve_layer(const dash_dims& D, int64_t M, int64_t T_kv, int64_t max_pos, C
 // pos: RoPE position of each row (NULL: row index); kstart: first key each
 // row may attend to (NULL: 0; varlen batches); halted_pos: RoPE positions of
 // the halted rows (NULL: their original index).
-dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_layer_weights& w, bf16* H, int64_t M,
+template <int DT>
+dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_layer_weights& w, s16* H, int64_t M,
                        const int32_t* pos, const dash_halt_ctx* halt, float* delta, int relative,
                        const LayerWs& ws, cudaStream_t st, const int32_t* kstart = nullptr,
                        const int32_t* halted_pos = nullptr, int delta_accumulate = 0) {
@@ -436,7 +447,7 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   // original positions ([DASH news] "选择性停止机制").
   if (halt && T_kv > M) {
     const int64_t nh = T_kv - M;
-    if ((s = rmsnorm(cb(halt->h_full), T_kv, halt->halted_idx, nh, d, cb(w.attn_norm), D.rms_eps, ws.Act, st,
+    if ((s = rmsnorm<DT>(cb(halt->h_full), T_kv, halt->halted_idx, nh, d, cb(w.attn_norm), D.rms_eps, ws.Act, st,
                      ws.rs)) != DASH_OK)
       return s;
     EpiArgs kv = qkv;
@@ -445,22 +456,22 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
     kv.pos = halted_pos ? halted_pos : halt->halted_idx;
     kv.kv_rowmap = halt->halted_idx;
     kv.col_offset = qd;
-    if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.Act, d, nh, d, cb(w.w_qkv) + static_cast<int64_t>(qd) * d, nullptr,
+    if ((s = gemm<dash::gemm::kEpiQkv, DT>(di, ws.Act, d, nh, d, cb(w.w_qkv) + static_cast<int64_t>(qd) * d, nullptr,
                                        2 * kvd, kv, st, DASH_K_GEMM_KV_HALTED)) != DASH_OK)
       return s;
   }
 
   // a1: input RMSNorm (its 1/rms is applied to the QKV accumulator)
-  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.attn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
+  if ((s = rmsnorm<DT>(H, M, nullptr, M, d, cb(w.attn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
   // a2: QKV projection + RoPE (k/v of active rows land at their original rows in halt mode)
   qkv.row_scale = ws.rs;
   qkv.pos = pos;
   qkv.kv_rowmap = halt ? halt->active_idx : nullptr;
   qkv.col_offset = 0;
-  if ((s = gemm<dash::gemm::kEpiQkv>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st, DASH_K_GEMM_QKV)) != DASH_OK)
+  if ((s = gemm<dash::gemm::kEpiQkv, DT>(di, ws.X, d, M, d, cb(w.w_qkv), nullptr, qd + 2 * kvd, qkv, st, DASH_K_GEMM_QKV)) != DASH_OK)
     return s;
   // a3: causal GQA attention -> O (into X)
-  if ((s = attention(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, kstart,
+  if ((s = attention<DT>(ws.Q, qd, ws.Kb, ws.Vb, kvd, M, T_kv, hq, hkv, hd, halt ? halt->active_idx : nullptr, kstart,
                      ws.X, qd, st)) != DASH_OK)
     return s;
   // a4: o_proj + residual (+ per-row sums of U^2 and H^2 for Δ)
@@ -471,9 +482,9 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
   o.ssq_h = ws.ssq_h;
   int bn = 0;
   if (delta)
-    s = gemm<dash::gemm::kEpiResidSsq>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
+    s = gemm<dash::gemm::kEpiResidSsq, DT>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
   else
-    s = gemm<dash::gemm::kEpiResid>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
+    s = gemm<dash::gemm::kEpiResid, DT>(di, ws.X, qd, M, qd, cb(w.w_o), nullptr, d, o, st, DASH_K_GEMM_O, &bn);
   if (s != DASH_OK) return s;
   if (delta) {
     const int64_t blocks = (M + 255) / 256;
@@ -484,17 +495,24 @@ dash_status layer_impl(const DeviceInfo& di, const dash_dims& D, const dash_laye
     if ((s = launch_status()) != DASH_OK) return s;
   }
   // a5: post-attention RMSNorm, gate/up GEMM with SwiGLU
-  if ((s = rmsnorm(H, M, nullptr, M, d, cb(w.ffn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
+  if ((s = rmsnorm<DT>(H, M, nullptr, M, d, cb(w.ffn_norm), D.rms_eps, ws.X, st, ws.rs)) != DASH_OK) return s;
   EpiArgs sw{};
   sw.out = ws.Act;
   sw.ldo = F;
   sw.row_scale = ws.rs;
-  if ((s = gemm<dash::gemm::kEpiSwiglu>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st, DASH_K_GEMM_GATE_UP)) != DASH_OK) return s;
+  if ((s = gemm<dash::gemm::kEpiSwiglu, DT>(di, ws.X, d, M, d, cb(w.w_gate), cb(w.w_up), 2 * F, sw, st, DASH_K_GEMM_GATE_UP)) != DASH_OK) return s;
   // a6: down projection + residual
   EpiArgs dn{};
   dn.out = H;
   dn.ldo = d;
-  return gemm<dash::gemm::kEpiResid>(di, ws.Act, F, M, F, cb(w.w_down), nullptr, d, dn, st, DASH_K_GEMM_DOWN);
+  return gemm<dash::gemm::kEpiResid, DT>(di, ws.Act, F, M, F, cb(w.w_down), nullptr, d, dn, st, DASH_K_GEMM_DOWN);
+}
+
+// The decoder block in the model's 16-bit format (dims.dtype).
+template <typename... A>
+dash_status layer_fmt(const DeviceInfo& di, const dash_dims& D, A&&... a) {
+  if (D.dtype == DASH_DTYPE_F16) return layer_impl<kF16>(di, D, std::forward<A>(a)...);
+  return layer_impl<kBf16>(di, D, std::forward<A>(a)...);
 }
 
 bool weights_ok(const dash_layer_weights* w) {
@@ -505,7 +523,7 @@ bool weights_ok(const dash_layer_weights* w) {
 
 struct PrefillWs {
   LayerWs L;
-  bf16* Hc;         // [T, d] compacted active rows
+  s16* Hc;         // [T, d] compacted active rows
   float* delta;     // [T]
   int32_t* idx;     // [T]
   int32_t* halted;  // [T]
@@ -522,7 +540,7 @@ struct PrefillWs {
 
 void carve_prefill(const dash_dims& D, int64_t T, int nseq, Carver& c, PrefillWs& w) {
   carve_layer(D, T, T, T, c, w.L);
-  w.Hc = c.take<bf16>(static_cast<size_t>(T) * D.d_model);
+  w.Hc = c.take<s16>(static_cast<size_t>(T) * D.d_model);
   w.delta = c.take<float>(static_cast<size_t>(T));
   w.idx = c.take<int32_t>(static_cast<size_t>(T));
   w.halted = c.take<int32_t>(static_cast<size_t>(T));
@@ -598,7 +616,7 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, int64_t n, float* _
 
 
 // ---------------------------------------------------------------- KV cache
-dash_status kv_store(const bf16* Kb, const bf16* Vb, int kvd, int64_t a, int64_t rows, const int32_t* pos_src,
+dash_status kv_store(const s16* Kb, const s16* Vb, int kvd, int64_t a, int64_t rows, const int32_t* pos_src,
                      const dash_kv_cache& c, const DeviceInfo& di, cudaStream_t st) {
   if (rows == 0) return DASH_OK;
   const int warps = 8;
@@ -607,7 +625,7 @@ dash_status kv_store(const bf16* Kb, const bf16* Vb, int kvd, int64_t a, int64_t
   if (blocks > cap) blocks = cap;
   TimedLaunch tl(DASH_K_KV_STORE, rows, kvd, 0, st);
   dash::decode::kv_store_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, st>>>(
-      Kb, Vb, kvd, a, rows, pos_src, reinterpret_cast<bf16*>(c.k), reinterpret_cast<bf16*>(c.v), c.pos);
+      Kb, Vb, kvd, a, rows, pos_src, reinterpret_cast<s16*>(c.k), reinterpret_cast<s16*>(c.v), c.pos);
   return launch_status();
 }
 
@@ -687,7 +705,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   PrefillWs P;
   carve_prefill(*dims, T, nseq, c, P);
   cudaStream_t st = as_stream(stream);
-  bf16* h = reinterpret_cast<bf16*>(H);
+  s16* h = reinterpret_cast<s16*>(H);
   const dash_dims& D = *dims;
   const bool varlen = nseq > 1;
   if ((s = rope_table(P.L.rope, T, D.head_dim, D.rope_theta, *di, st)) != DASH_OK) return s;
@@ -713,13 +731,13 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   const int32_t* kv_pos = nullptr;
 
   // Δ is taken at the layers [delta_first, delta_last] and combined by maximum.
-  auto run_layers = [&](int l0, int l1, bf16* rows, int64_t M, const int32_t* pos, const dash_halt_ctx* hc,
+  auto run_layers = [&](int l0, int l1, s16* rows, int64_t M, const int32_t* pos, const dash_halt_ctx* hc,
                         const int32_t* kst, const int32_t* hpos, int delta_first, int delta_last,
                         float* delta) -> dash_status {
     for (int l = l0; l < l1; ++l) {
       g_timing.layer = l;
       const bool take = l >= delta_first && l <= delta_last;
-      dash_status r = layer_impl(*di, D, layers[l], rows, M, pos, hc, take ? delta : nullptr,
+      dash_status r = layer_fmt(*di, D, layers[l], rows, M, pos, hc, take ? delta : nullptr,
                                  cfg->score == DASH_SCORE_REL, P.L, st, kst, hpos, l > delta_first ? 1 : 0);
       for (int q = 0; r == DASH_OK && caches && q < nseq; ++q) {
         dash_kv_cache& c = caches[static_cast<size_t>(q) * D.n_layers + l];
@@ -809,7 +827,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
     }
     if ((s = run_layers(Ls + 1, D.n_layers, P.Hc, K, pos_c, nullptr, kst_c, nullptr, -1, -1, nullptr)) != DASH_OK)
       return s;
-    if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(bf16),
+    if (K > 0 && cudaMemcpyAsync(h, P.Hc, static_cast<size_t>(K) * D.d_model * sizeof(s16),
                                  cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return DASH_ERR_CUDA;
     return DASH_OK;
@@ -839,9 +857,9 @@ namespace dec = dash::decode;
 
 struct DecodeWs {
   int* counters;   // [kMaxSegs] finished decode-attention CTAs per segment
-  bf16* Q;         // [n, hq*hd]
-  bf16* O;         // [n, hq*hd] attention output
-  bf16* Act;       // [n, F]
+  s16* Q;         // [n, hq*hd]
+  s16* O;         // [n, hq*hd] attention output
+  s16* Act;       // [n, F]
   float* part_o;   // [kMaxCtas, 16, hd]
   float* part_ml;  // [kMaxCtas, 16, 2]
 };
@@ -849,9 +867,9 @@ struct DecodeWs {
 void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
   w.counters = c.take<int>(dec::kMaxSegs);
-  w.Q = c.take<bf16>(n * qd);
-  w.O = c.take<bf16>(n * qd);
-  w.Act = c.take<bf16>(static_cast<size_t>(n) * D.ffn_dim);
+  w.Q = c.take<s16>(n * qd);
+  w.O = c.take<s16>(n * qd);
+  w.Act = c.take<s16>(static_cast<size_t>(n) * D.ffn_dim);
   w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * D.head_dim);
   w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
 }
@@ -877,7 +895,7 @@ cudaError_t launch_pdl(void (*kernel)(ExpTypes...), unsigned grid, unsigned bloc
 
 constexpr size_t kGemvSmemMax = 160 * 1024;  // x staged in shared memory up to this size
 
-template <int EPI, int NS>
+template <int EPI, int NS, int DT>
 dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out,
                            cudaStream_t st) {
   if (gp.tasks == 0) return DASH_OK;
@@ -891,30 +909,30 @@ dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int 
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(dec::gemv_kernel<EPI, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(dec::gemv_kernel<EPI, NS, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(kGemvSmemMax));
   });
   if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
   // one CTA per SM (tasks strided over the grid), so every SM streams weights
   const unsigned grid = static_cast<unsigned>(gp.tasks < di.num_sms ? gp.tasks : di.num_sms);
   TimedLaunch tl(kind, gp.n, n_out, gp.K, st);
-  if (launch_pdl(dec::gemv_kernel<EPI, NS>, grid, 32 * dec::kGemvWarps, smem, st, q) != cudaSuccess)
+  if (launch_pdl(dec::gemv_kernel<EPI, NS, DT>, grid, 32 * dec::kGemvWarps, smem, st, q) != cudaSuccess)
     return DASH_ERR_CUDA;
   return launch_status();
 }
 
-template <int EPI>
+template <int EPI, int DT>
 dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
-  if (gp.n <= 1) return launch_gemv_ns<EPI, 1>(di, gp, kind, n_out, st);
-  if (gp.n <= 2) return launch_gemv_ns<EPI, 2>(di, gp, kind, n_out, st);
-  if (gp.n <= 4) return launch_gemv_ns<EPI, 4>(di, gp, kind, n_out, st);
-  return launch_gemv_ns<EPI, 8>(di, gp, kind, n_out, st);
+  if (gp.n <= 1) return launch_gemv_ns<EPI, 1, DT>(di, gp, kind, n_out, st);
+  if (gp.n <= 2) return launch_gemv_ns<EPI, 2, DT>(di, gp, kind, n_out, st);
+  if (gp.n <= 4) return launch_gemv_ns<EPI, 4, DT>(di, gp, kind, n_out, st);
+  return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, st);
 }
 
 // Split-key decode attention of one layer: the CTA count is held to one
 // wave (at most one CTA per SM, at most kMaxCtas) by giving each CTA a run of
 // tiles_per_cta key tiles of one (sequence, kv head) segment.
-template <int HD>
+template <int HD, int DT>
 dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n, const int64_t* len,
                                 const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st,
                                 const dec::Prefetch* next = nullptr) {
@@ -922,7 +940,7 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(dec::decode_attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(dec::decode_attn_kernel<HD, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
@@ -934,8 +952,8 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   int64_t total_tiles = 0, max_tiles = 0, keys = 0;
   for (int q = 0; q < n; ++q) {
     const dash_kv_cache& c = *layer_caches[q];
-    if (!make_map(&maps.k[q], c.k, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV) ||
-        !make_map(&maps.v[q], c.v, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV))
+    if (!make_map(&maps.k[q], c.k, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV, Num<DT>::kMapType) ||
+        !make_map(&maps.v[q], c.v, static_cast<uint64_t>(len[q]), kvd, kvd, dec::BKV, Num<DT>::kMapType))
       return DASH_ERR_INVALID_ARG;
     ap.len[q] = static_cast<int>(len[q]);
     const int64_t t = (len[q] + dec::BKV - 1) / dec::BKV;
@@ -976,12 +994,13 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
   if (next) ap.next = *next;
   TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, nctas, st);
-  if (launch_pdl(dec::decode_attn_kernel<HD>, static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st,
+  if (launch_pdl(dec::decode_attn_kernel<HD, DT>, static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st,
                  maps, ap) != cudaSuccess)
     return DASH_ERR_CUDA;
   return launch_status();
 }
 
+template <int DT>
 dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X, int n,
                         const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes, void* stream) {
   if (!dims_ok(dims)) return DASH_ERR_SHAPE;
@@ -1011,7 +1030,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
   DecodeWs w;
   carve_decode(D, n, c, w);
   cudaStream_t st = as_stream(stream);
-  bf16* x = reinterpret_cast<bf16*>(X);
+  s16* x = reinterpret_cast<s16*>(X);
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd;
   if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
@@ -1025,8 +1044,8 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     std::memset(&qkv, 0, sizeof(qkv));
     for (int q = 0; q < n; ++q) {
       lc[q] = &caches[static_cast<size_t>(q) * D.n_layers + l];
-      qkv.seq.k[q] = reinterpret_cast<bf16*>(lc[q]->k);
-      qkv.seq.v[q] = reinterpret_cast<bf16*>(lc[q]->v);
+      qkv.seq.k[q] = reinterpret_cast<s16*>(lc[q]->k);
+      qkv.seq.v[q] = reinterpret_cast<s16*>(lc[q]->v);
       qkv.seq.pos[q] = lc[q]->pos;
       qkv.seq.row[q] = lc[q]->len;
       qkv.seq.p[q] = pos[q];
@@ -1052,14 +1071,14 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
       qkv.next.ptr[qkv.next.count] = reinterpret_cast<const uint8_t*>(lc[q]->v);
       qkv.next.bytes[qkv.next.count++] = bytes;
     }
-    if ((s = launch_gemv<dec::kGvQkv>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvQkv, DT>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
     // attention over each sequence's cache (including the new row)
     dec::Prefetch wo{};  // o_proj streams W_o next
     wo.ptr[0] = reinterpret_cast<const uint8_t*>(lw.w_o);
     wo.bytes[0] = static_cast<uint64_t>(d) * qd * 2;
     wo.count = 1;
-    s = hd == 128 ? decode_attention_hd<128>(*di, D, n, len, lc, w, st, &wo)
-                  : decode_attention_hd<64>(*di, D, n, len, lc, w, st, &wo);
+    s = hd == 128 ? decode_attention_hd<128, DT>(*di, D, n, len, lc, w, st, &wo)
+                  : decode_attention_hd<64, DT>(*di, D, n, len, lc, w, st, &wo);
     if (s != DASH_OK) break;
     // o_proj + residual
     dec::GemvParams o;
@@ -1079,7 +1098,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
       o.next.bytes[1] = static_cast<uint64_t>(first) * d * 2;
       o.next.count = 2;
     }
-    if ((s = launch_gemv<dec::kGvResid>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid, DT>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
     // RMSNorm (fused) -> gate/up with SwiGLU
     dec::GemvParams gu;
     std::memset(&gu, 0, sizeof(gu));
@@ -1093,7 +1112,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     gu.tasks = F;
     gu.out = w.Act;
     gu.ldo = F;
-    if ((s = launch_gemv<dec::kGvSwiglu>(*di, gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvSwiglu, DT>(*di, gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
     // down + residual
     dec::GemvParams dn;
     std::memset(&dn, 0, sizeof(dn));
@@ -1109,7 +1128,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
       dn.next.bytes[0] = static_cast<uint64_t>(qd + 2 * hkv * hd) * d * 2;
       dn.next.count = 1;
     }
-    if ((s = launch_gemv<dec::kGvResid>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid, DT>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
     for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
   }
   g_timing.layer = -1;
@@ -1153,8 +1172,8 @@ dash_status dash_score(const dash_bf16* U, const dash_bf16* H, int64_t T, int32_
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
   TimedLaunch tl(DASH_K_SCORE, T, d, relative ? 1 : 0, as_stream(stream));
-  dash::rows::score_kernel<<<static_cast<unsigned>(blocks), 32 * warps, 0, as_stream(stream)>>>(
-      reinterpret_cast<const bf16*>(U), reinterpret_cast<const bf16*>(H), T, d, relative ? 1 : 0, delta);
+  dash::rows::score_kernel<kBf16><<<static_cast<unsigned>(blocks), 32 * warps, 0, as_stream(stream)>>>(
+      reinterpret_cast<const s16*>(U), reinterpret_cast<const s16*>(H), T, d, relative ? 1 : 0, delta);
   return launch_status();
 }
 
@@ -1190,7 +1209,7 @@ dash_status dash_compact(const dash_bf16* X, int64_t T, const int32_t* idx, int6
   DeviceInfo* di;
   dash_status s = device_info(&di);
   if (s != DASH_OK) return s;
-  return move_rows(false, reinterpret_cast<const bf16*>(X), reinterpret_cast<bf16*>(Y), idx, K, T, d, *di,
+  return move_rows(false, reinterpret_cast<const s16*>(X), reinterpret_cast<s16*>(Y), idx, K, T, d, *di,
                    as_stream(stream));
 }
 
@@ -1202,7 +1221,7 @@ dash_status dash_scatter(const dash_bf16* Y, const int32_t* idx, int64_t K, int3
   DeviceInfo* di;
   dash_status s = device_info(&di);
   if (s != DASH_OK) return s;
-  return move_rows(true, reinterpret_cast<const bf16*>(Y), reinterpret_cast<bf16*>(X), idx, K, T, d, *di,
+  return move_rows(true, reinterpret_cast<const s16*>(Y), reinterpret_cast<s16*>(X), idx, K, T, d, *di,
                    as_stream(stream));
 }
 
@@ -1211,8 +1230,8 @@ dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf
   if (M < 0 || d <= 0 || d % 8 != 0 || d > 8 * 32 * dash::rows::kMaxVec) return DASH_ERR_SHAPE;
   if (M == 0) return DASH_OK;
   if (!X || !g || !Y || !aligned16(X) || !aligned16(g) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
-  return rmsnorm(reinterpret_cast<const bf16*>(X), M, nullptr, M, d, reinterpret_cast<const bf16*>(g), eps,
-                 reinterpret_cast<bf16*>(Y), as_stream(stream));
+  return rmsnorm<kBf16>(reinterpret_cast<const s16*>(X), M, nullptr, M, d, reinterpret_cast<const s16*>(g), eps,
+                 reinterpret_cast<s16*>(Y), as_stream(stream));
 }
 
 int32_t dash_set_gemm_pairs(int32_t enable) { return g_gemm_pairs.exchange(enable != 0 ? 1 : 0); }
@@ -1226,9 +1245,9 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
   dash_status s = device_info(&di);
   if (s != DASH_OK) return s;
   EpiArgs ep{};
-  ep.out = reinterpret_cast<bf16*>(Y);
+  ep.out = reinterpret_cast<s16*>(Y);
   ep.ldo = N;
-  return gemm<dash::gemm::kEpiStore>(*di, reinterpret_cast<const bf16*>(A), K, M, K, reinterpret_cast<const bf16*>(W),
+  return gemm<dash::gemm::kEpiStore, kBf16>(*di, reinterpret_cast<const s16*>(A), K, M, K, reinterpret_cast<const s16*>(W),
                                      nullptr, N, ep, as_stream(stream), DASH_K_GEMM);
 }
 
@@ -1262,9 +1281,9 @@ dash_status dash_attention(const dash_bf16* Q, const dash_bf16* K, const dash_bf
   dash_status s = device_info(&di);
   if (s != DASH_OK) return s;
   const int64_t qd = static_cast<int64_t>(hq) * hd, kvd = static_cast<int64_t>(hkv) * hd;
-  return attention(reinterpret_cast<const bf16*>(Q), qd, reinterpret_cast<const bf16*>(K),
-                   reinterpret_cast<const bf16*>(V), kvd, M, T_kv, hq, hkv, hd, qpos, kstart,
-                   reinterpret_cast<bf16*>(O), qd, as_stream(stream));
+  return attention<kBf16>(reinterpret_cast<const s16*>(Q), qd, reinterpret_cast<const s16*>(K),
+                   reinterpret_cast<const s16*>(V), kvd, M, T_kv, hq, hkv, hd, qpos, kstart,
+                   reinterpret_cast<s16*>(O), qd, as_stream(stream));
 }
 
 size_t dash_layer_workspace_size(const dash_dims* dims, int64_t M, int64_t T_kv, int64_t max_pos) {
@@ -1301,7 +1320,7 @@ dash_status dash_layer_forward(const dash_dims* dims, const dash_layer_weights* 
   carve_layer(*dims, M, T_kv, max_pos, c, L);
   cudaStream_t st = as_stream(stream);
   if ((s = rope_table(L.rope, max_pos, dims->head_dim, dims->rope_theta, *di, st)) != DASH_OK) return s;
-  return layer_impl(*di, *dims, *w, reinterpret_cast<bf16*>(H), M, pos, halt, delta, relative, L, st);
+  return layer_fmt(*di, *dims, *w, reinterpret_cast<s16*>(H), M, pos, halt, delta, relative, L, st);
 }
 
 dash_status dash_layer_forward_noalloc(const dash_dims* dims, const dash_layer_weights* w, dash_bf16* H,
@@ -1415,15 +1434,15 @@ dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_k
   D.head_dim = hd;
   Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
   DecodeWs w{};
-  w.Q = const_cast<bf16*>(reinterpret_cast<const bf16*>(Q));
-  w.O = reinterpret_cast<bf16*>(O);
+  w.Q = const_cast<s16*>(reinterpret_cast<const s16*>(Q));
+  w.O = reinterpret_cast<s16*>(O);
   w.counters = c.take<int>(dec::kMaxSegs);
   w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * hd);
   w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
   cudaStream_t st = as_stream(stream);
   if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
-  return hd == 128 ? decode_attention_hd<128>(*di, D, nseq, len, lc, w, st)
-                   : decode_attention_hd<64>(*di, D, nseq, len, lc, w, st);
+  return hd == 128 ? decode_attention_hd<128, kBf16>(*di, D, nseq, len, lc, w, st)
+                   : decode_attention_hd<64, kBf16>(*di, D, nseq, len, lc, w, st);
 }
 
 size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq) {
@@ -1437,7 +1456,9 @@ size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq) {
 dash_status dash_decode_step(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X,
                              int32_t nseq, const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes,
                              void* stream) {
-  return decode_impl(dims, layers, X, nseq, pos, caches, ws, ws_bytes, stream);
+  if (dims && dims->dtype == DASH_DTYPE_F16)
+    return decode_impl<kF16>(dims, layers, X, nseq, pos, caches, ws, ws_bytes, stream);
+  return decode_impl<kBf16>(dims, layers, X, nseq, pos, caches, ws, ws_bytes, stream);
 }
 
 dash_status dash_timing_start(int32_t capacity) {

@@ -80,24 +80,24 @@ __device__ __forceinline__ void prefetch_share(const Prefetch& pf) {
 enum GemvEpi : int { kGvQkv = 0, kGvResid = 1, kGvSwiglu = 2 };
 
 struct SeqSlots {
-  __nv_bfloat16* k[kMaxSeq];  // cache arrays of this layer
-  __nv_bfloat16* v[kMaxSeq];
+  s16* k[kMaxSeq];  // cache arrays of this layer
+  s16* v[kMaxSeq];
   int32_t* pos[kMaxSeq];      // may be NULL
   int64_t row[kMaxSeq];       // row the new token's k/v go to
   int32_t p[kMaxSeq];         // RoPE position of the new token
 };
 
 struct GemvParams {
-  const __nv_bfloat16* W;     // [rows, K] row-major
-  const __nv_bfloat16* W2;    // kGvSwiglu: up-projection [rows, K]
-  const __nv_bfloat16* x;     // [n, K]
-  const __nv_bfloat16* gain;  // kGvQkv / kGvSwiglu: RMSNorm gain [K] (the norm is fused)
+  const s16* W;     // [rows, K] row-major
+  const s16* W2;    // kGvSwiglu: up-projection [rows, K]
+  const s16* x;     // [n, K]
+  const s16* gain;  // kGvQkv / kGvSwiglu: RMSNorm gain [K] (the norm is fused)
   float eps;
   int n, K, tasks;
   int stage_x;                // kGvResid: copy x to shared memory first (it fits)
-  __nv_bfloat16* out;  // kGvResid: residual stream [n, ldo] (in/out); kGvSwiglu: act [n, ldo]
+  s16* out;  // kGvResid: residual stream [n, ldo] (in/out); kGvSwiglu: act [n, ldo]
   int64_t ldo;
-  __nv_bfloat16* q;  // kGvQkv: [n, hq*hd]
+  s16* q;  // kGvQkv: [n, hq*hd]
   int hq, hkv, hd;
   double theta;
   SeqSlots seq;
@@ -112,34 +112,38 @@ constexpr int kGemvWarps = 16;  // one CTA per SM; warps take tasks strided over
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+template <int DT>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
-  float a = bf16_lo(w.x) * bf16_lo(x.x);
-  float b = bf16_hi(w.x) * bf16_hi(x.x);
-  a = fmaf(bf16_lo(w.y), bf16_lo(x.y), a);
-  b = fmaf(bf16_hi(w.y), bf16_hi(x.y), b);
-  a = fmaf(bf16_lo(w.z), bf16_lo(x.z), a);
-  b = fmaf(bf16_hi(w.z), bf16_hi(x.z), b);
-  a = fmaf(bf16_lo(w.w), bf16_lo(x.w), a);
-  b = fmaf(bf16_hi(w.w), bf16_hi(x.w), b);
+  using N = Num<DT>;
+  float a = N::lo(w.x) * N::lo(x.x);
+  float b = N::hi(w.x) * N::hi(x.x);
+  a = fmaf(N::lo(w.y), N::lo(x.y), a);
+  b = fmaf(N::hi(w.y), N::hi(x.y), b);
+  a = fmaf(N::lo(w.z), N::lo(x.z), a);
+  b = fmaf(N::hi(w.z), N::hi(x.z), b);
+  a = fmaf(N::lo(w.w), N::lo(x.w), a);
+  b = fmaf(N::hi(w.w), N::hi(x.w), b);
   return a + b;
 }
 
+template <int DT>
 __device__ __forceinline__ float sumsq8(const uint4& v) {
+  using N = Num<DT>;
   float s = 0.f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int e = 0; e < 4; ++e) s = fmaf(bf16_lo(w[e]), bf16_lo(w[e]), fmaf(bf16_hi(w[e]), bf16_hi(w[e]), s));
+  for (int e = 0; e < 4; ++e) s = fmaf(N::lo(w[e]), N::lo(w[e]), fmaf(N::hi(w[e]), N::hi(w[e]), s));
   return s;
 }
 
+template <int DT>
 __device__ __forceinline__ uint4 mul8(const uint4& x, const uint4& g) {
-  return make_uint4(pack_bf16(bf16_lo(x.x) * bf16_lo(g.x), bf16_hi(x.x) * bf16_hi(g.x)),
-                    pack_bf16(bf16_lo(x.y) * bf16_lo(g.y), bf16_hi(x.y) * bf16_hi(g.y)),
-                    pack_bf16(bf16_lo(x.z) * bf16_lo(g.z), bf16_hi(x.z) * bf16_hi(g.z)),
-                    pack_bf16(bf16_lo(x.w) * bf16_lo(g.w), bf16_hi(x.w) * bf16_hi(g.w)));
+  using N = Num<DT>;
+  return make_uint4(N::pack(N::lo(x.x) * N::lo(g.x), N::hi(x.x) * N::hi(g.x)),
+                    N::pack(N::lo(x.y) * N::lo(g.y), N::hi(x.y) * N::hi(g.y)),
+                    N::pack(N::lo(x.z) * N::lo(g.z), N::hi(x.z) * N::hi(g.z)),
+                    N::pack(N::lo(x.w) * N::lo(g.w), N::hi(x.w) * N::hi(g.w)));
 }
-
-__device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // Streaming read of weights: not kept in L1, 256-byte L2 fetch granularity.
 __device__ __forceinline__ uint4 ldg_stream(const uint4* ptr) {
@@ -155,10 +159,10 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* ptr) {
 //   kGvSwiglu  row t of W (gate) and row t of W2 (up)
 //   kGvResid   rows (2t, 2t + 1)
 // With the norm fused (kGvQkv, kGvSwiglu) the CTA first computes each
-// input row's 1/rms and stages x * gain as bf16 in shared memory (exact for
-// unit gains); the 1/rms multiplies the finished dot products, as the
+// input row's 1/rms and stages x * gain in shared memory, in the model's
+// 16-bit format (exact for unit gains); the 1/rms multiplies the finished dot products, as the
 // prefill's GEMM epilogues do.  kGvResid stages x as is when it fits.
-template <int EPI, int NS>
+template <int EPI, int NS, int DT>
 __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvParams p) {
   constexpr bool kNorm = EPI != kGvResid;
   extern __shared__ uint4 xg_smem[];  // kNorm: [n][K/8]
@@ -181,8 +185,8 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
       for (int m = 0; m < NS; ++m)
         if (m < p.n) {
           const uint4 v = __ldg(xg + static_cast<int64_t>(m) * nv + c);
-          ss[m] += sumsq8(v);
-          xg_smem[m * nv + c] = mul8(v, g);
+          ss[m] += sumsq8<DT>(v);
+          xg_smem[m * nv + c] = mul8<DT>(v, g);
         }
     }
 #pragma unroll
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
   constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
   const int stride = gridDim.x * kGemvWarps;
   // the two weight rows of a task
-  auto rows = [&](int task, const __nv_bfloat16*& w0, const __nv_bfloat16*& w1) {
+  auto rows = [&](int task, const s16*& w0, const s16*& w1) {
     if constexpr (EPI == kGvQkv) {
       const int half = p.hd >> 1;
       const int head = task / half, i = task - head * half;
@@ -228,16 +232,16 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
       head = task / (p.hd >> 1);
       i = task - head * (p.hd >> 1);
     }
-    const __nv_bfloat16* w0;
-    const __nv_bfloat16* w1;
+    const s16* w0;
+    const s16* w1;
     rows(task, w0, w1);
     // The next task's rows go to L2 while this one streams.  (Prefetching the
     // current task's rows as well measured slower: the demand loads race
     // their own prefetch.)
     if (lane == 0) {
       if (task + stride < p.tasks) {
-        const __nv_bfloat16* n0;
-        const __nv_bfloat16* n1;
+        const s16* n0;
+        const s16* n1;
         rows(task + stride, n0, n1);
         prefetch_l2(n0, K * 2);
         prefetch_l2(n1, K * 2);
@@ -266,8 +270,8 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
           for (int m = 0; m < NS; ++m) {
             if (m < p.n) {
               const uint4 xm = from_smem ? xg[m * nv + c] : __ldg(xg + static_cast<int64_t>(m) * nv + c);
-              a0[m] += dot8(ra[u], xm);
-              a1[m] += dot8(rb[u], xm);
+              a0[m] += dot8<DT>(ra[u], xm);
+              a1[m] += dot8<DT>(rb[u], xm);
             }
           }
         }
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
           o0 = y0 * c - y1 * s;
           o1 = y1 * c + y0 * s;
         }
-        __nv_bfloat16* dst;
+        s16* dst;
         if (head < p.hq) {
           dst = p.q + static_cast<int64_t>(m) * p.hq * hd + head * hd;
         } else {
@@ -308,14 +312,14 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
           dst = (is_k ? p.seq.k[m] : p.seq.v[m]) + p.seq.row[m] * kvd + h * hd;
           if (head == p.hq && i == 0 && p.seq.pos[m]) p.seq.pos[m][p.seq.row[m]] = p.seq.p[m];
         }
-        dst[i] = __float2bfloat16_rn(o0);
-        dst[i + half] = __float2bfloat16_rn(o1);
+        dst[i] = Num<DT>::from_f(o0);
+        dst[i + half] = Num<DT>::from_f(o1);
       } else if constexpr (EPI == kGvSwiglu) {
-        p.out[static_cast<int64_t>(m) * p.ldo + task] = __float2bfloat16_rn(y0 / (1.f + __expf(-y0)) * y1);
+        p.out[static_cast<int64_t>(m) * p.ldo + task] = Num<DT>::from_f(y0 / (1.f + __expf(-y0)) * y1);
       } else {
-        __nv_bfloat16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
-        const float r0 = bf16_to_f(o[0]) + y0, r1 = bf16_to_f(o[1]) + y1;
-        *reinterpret_cast<uint32_t*>(o) = pack_bf16(r0, r1);
+        s16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
+        const float r0 = Num<DT>::to_f(o[0]) + y0, r1 = Num<DT>::to_f(o[1]) + y1;
+        *reinterpret_cast<uint32_t*>(o) = Num<DT>::pack(r0, r1);
       }
     }
   }
@@ -323,8 +327,8 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
 
 // ========================================================= decode attention
 struct AttnParams {
-  const __nv_bfloat16* q;  // [n, hq*HD], RoPE applied
-  __nv_bfloat16* out;      // [n, hq*HD]
+  const s16* q;  // [n, hq*HD], RoPE applied
+  s16* out;      // [n, hq*HD]
   float* part_o;           // [CTA c][g < group][HD]: unnormalised O of each CTA (a segment's CTAs adjacent)
   float* part_ml;          // [CTA c][16][2]: (running max in log2 units, sum); 128 bytes per CTA, so
                            // a segment's block starts 16-byte aligned for the bulk copy
@@ -337,7 +341,7 @@ struct AttnParams {
 };
 
 struct AttnMaps {
-  CUtensorMap k[kMaxSeq];  // [len, hkv*HD] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap k[kMaxSeq];  // [len, hkv*HD] 16-bit, box {64, 128}, 128B swizzle
   CUtensorMap v[kMaxSeq];
 };
 
@@ -404,7 +408,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 //   O_g = sum_c w_cg o_cg.
 // A segment's partial results are adjacent in memory, so they come into
 // shared memory by a few large bulk async copies (one L2 round trip each).
-template <int HD>
+template <int HD, int DT>
 __device__ void merge_segment(const AttnParams& p, int seg, int s, int kvh, uint8_t* scratch, int scratch_bytes,
                               uint32_t bar) {
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -478,14 +482,14 @@ __device__ void merge_segment(const AttnParams& p, int seg, int s, int kvh, uint
       }
     }
   }
-  __nv_bfloat16* dst = p.out + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
+  s16* dst = p.out + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
 #pragma unroll
   for (int j = 0; j < kMaxOut; ++j) {
     const int i = t + j * kAttnThreads;
     if (i < n4) {
       uint2 v;
-      v.x = pack_bf16(acc[j].x, acc[j].y);
-      v.y = pack_bf16(acc[j].z, acc[j].w);
+      v.x = Num<DT>::pack(acc[j].x, acc[j].y);
+      v.y = Num<DT>::pack(acc[j].z, acc[j].w);
       *reinterpret_cast<uint2*>(dst + 4 * i) = v;
     }
   }
@@ -495,7 +499,7 @@ __device__ void merge_segment(const AttnParams& p, int seg, int s, int kvh, uint
 // segment.  Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.
 // Warps 2..5: Q staging, softmax (lane r = key r of the tile), and the
 // epilogue (lane r = dimension r of O^T), writing the CTA's partial result.
-template <int HD>
+template <int HD, int DT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     decode_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using C = ACfg<HD>;
@@ -593,8 +597,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    const uint32_t idesc_s = umma_idesc_bf16(BKV, kGroupPad, false, false);
-    const uint32_t idesc_o = umma_idesc_bf16(BKV, kGroupPad, true, false);
+    const uint32_t idesc_s = umma_idesc<DT>(BKV, kGroupPad, false, false);
+    const uint32_t idesc_o = umma_idesc<DT>(BKV, kGroupPad, true, false);
     const uint32_t sq = smem_u32(smem + C::kOffQ);
     const uint32_t sp = smem_u32(smem + C::kOffP);
     const uint32_t sz = smem_u32(smem + C::kOffZero);
@@ -608,7 +612,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t oa = (kk >> 2) * (BKV * 128) + (kk & 3) * 32;
           const uint32_t ob = (kk >> 2) * 2048 + (kk & 3) * 32;
-          umma_bf16_ss(tmem_base + (i & 1) * kGroupPad, umma_desc_sw128(sk + oa, 16, 1024),
+          umma_ss(tmem_base + (i & 1) * kGroupPad, umma_desc_sw128(sk + oa, 16, 1024),
                        umma_desc_sw128(sq + ob, 16, 1024), idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(bar_sfull + 8 * (i & 1));
@@ -626,7 +630,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint32_t ob = (kk >> 2) * 2048 + (kk & 3) * 32;
-          umma_bf16_ss(tmem_base + 2 * kGroupPad, umma_desc_sw128(sv + kk * 16 * 128, lbo, 1024),
+          umma_ss(tmem_base + 2 * kGroupPad, umma_desc_sw128(sv + kk * 16 * 128, lbo, 1024),
                        umma_desc_sw128(sp + (i & 1) * 4096 + ob, 16, 1024), idesc_o,
                        (i != 0 || kk != 0) ? 1u : 0u);
         }
@@ -653,7 +657,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int G = p.group;
     // Q of this kv head's group, rows G..15 zero, K-major 128B-swizzled.
     {
-      const __nv_bfloat16* qs = p.q + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
+      const s16* qs = p.q + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
       constexpr int kChunks = kGroupPad * HD / 8;
       for (int ch = r; ch < kChunks; ch += 128) {
         const int g = ch / (HD / 8), c = ch - g * (HD / 8);
@@ -728,9 +732,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int g = 0; g < kGroupPad; ++g) {
         const float e = valid ? ex2f(sv[g] - m_run[g]) : 0.f;
-        const __nv_bfloat16 eb = __float2bfloat16_rn(e);
         l_part[g] += e;
-        pb[g] = *reinterpret_cast<const uint16_t*>(&eb);
+        pb[g] = Num<DT>::from_f(e);
       }
       // P^T buffer i & 1 is free once P_(i-2) V_(i-2) is done; a rescale of
       // O^T also needs P_(i-1) V_(i-1) done.  (Each pv_done barrier is at
@@ -821,7 +824,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
   if (*ticket == 1) {  // uniform: written before the barrier above
-    merge_segment<HD>(p, seg, s, kvh, smem + C::kOffK, C::kOffZero - C::kOffK, bar_merge);
+    merge_segment<HD, DT>(p, seg, s, kvh, smem + C::kOffK, C::kOffZero - C::kOffK, bar_merge);
     if (threadIdx.x == 0) p.counters[seg] = 0;  // ready for the next launch
   }
 }
@@ -829,10 +832,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // ============================================================ cache store
 // Rows [a, a + rows) of the prefill's per-layer K/V buffers -> cache rows
 // [0, rows); pos[r] = pos_src[a + r] (or r when pos_src is NULL).
-__global__ void kv_store_kernel(const __nv_bfloat16* __restrict__ Kb, const __nv_bfloat16* __restrict__ Vb,
-                                int kvd, int64_t a, int64_t rows, const int32_t* __restrict__ pos_src,
-                                __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
-                                int32_t* __restrict__ pos) {
+__global__ void kv_store_kernel(const s16* __restrict__ Kb, const s16* __restrict__ Vb, int kvd, int64_t a,
+                                int64_t rows, const int32_t* __restrict__ pos_src, s16* __restrict__ k,
+                                s16* __restrict__ v, int32_t* __restrict__ pos) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t wpb = blockDim.x >> 5;
   const int nv = kvd >> 3;

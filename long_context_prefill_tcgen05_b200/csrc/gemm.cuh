@@ -1,8 +1,9 @@
 // Persistent tcgen05 GEMM for sm_100a: D[M, N] = A[M, K] * B[N, K]^T with
-// bf16 operands, fp32 accumulation in tensor memory, and epilogues fused for
+// 16-bit operands (bf16 or fp16, template parameter DT; the outputs take the
+// same format), fp32 accumulation in tensor memory, and epilogues fused for
 // the decoder block of the DASH prefill path:
 //
-//   kEpiStore     out = D (bf16)
+//   kEpiStore     out = D
 //   kEpiResid     out = out + D             (residual add, in place)
 //   kEpiResidSsq  out = out + D, plus per-row partial sums of D^2 and out_in^2
 //                 over the tile's columns -> the attention-update norm
@@ -27,20 +28,20 @@ namespace dash {
 namespace gemm {
 
 constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int BK = 64;  // 64 16-bit elements = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kGroupM = 16;  // M tiles per raster group (L2 reuse of B)
 
 enum Epi : int { kEpiStore = 0, kEpiResid = 1, kEpiResidSsq = 2, kEpiSwiglu = 3, kEpiQkv = 4 };
 
 struct EpiArgs {
-  __nv_bfloat16* out;  // store / resid / swiglu destination
+  s16* out;  // store / resid / swiglu destination
   int64_t ldo;
   float* ssq_u;  // [tiles_n, M] partial sums of D^2 (kEpiResidSsq)
   float* ssq_h;  // [tiles_n, M] partial sums of out_in^2
-  __nv_bfloat16* q;
-  __nv_bfloat16* k;
-  __nv_bfloat16* v;
+  s16* q;
+  s16* k;
+  s16* v;
   int64_t ldq, ldkv;
   const int32_t* pos;        // RoPE position of row m (NULL: m)
   const int32_t* kv_rowmap;  // k/v destination row of row m (NULL: m)
@@ -79,21 +80,22 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   tn = r / gsize;
 }
 
-__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
+template <int DT>
+__device__ __forceinline__ void store32(s16* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint4 w;
-    w.x = pack_bf16(v[8 * i + 0], v[8 * i + 1]);
-    w.y = pack_bf16(v[8 * i + 2], v[8 * i + 3]);
-    w.z = pack_bf16(v[8 * i + 4], v[8 * i + 5]);
-    w.w = pack_bf16(v[8 * i + 6], v[8 * i + 7]);
+    w.x = Num<DT>::pack(v[8 * i + 0], v[8 * i + 1]);
+    w.y = Num<DT>::pack(v[8 * i + 2], v[8 * i + 3]);
+    w.z = Num<DT>::pack(v[8 * i + 4], v[8 * i + 5]);
+    w.w = Num<DT>::pack(v[8 * i + 6], v[8 * i + 7]);
     d[i] = w;
   }
 }
 
 // ----------------------------------------------------------------- epilogues
-template <int BN, int EPI>
+template <int BN, int EPI, int DT>
 __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, const Shape& sh,
                                               const EpiArgs& ep) {
   const bool live = m < sh.M;
@@ -105,7 +107,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
       tmem_ld32(tbase + c, r);
       tmem_ld_wait();
       if (live) {
-        __nv_bfloat16* p = ep.out + static_cast<int64_t>(m) * ep.ldo + tn * BN + c;
+        s16* p = ep.out + static_cast<int64_t>(m) * ep.ldo + tn * BN + c;
         float o[32];
         if constexpr (EPI == kEpiStore) {
 #pragma unroll
@@ -118,7 +120,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
             const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float h0 = bf16_lo(hw[e]), h1 = bf16_hi(hw[e]);
+              const float h0 = Num<DT>::lo(hw[e]), h1 = Num<DT>::hi(hw[e]);
               const float a0 = __uint_as_float(r[8 * j + 2 * e]);
               const float a1 = __uint_as_float(r[8 * j + 2 * e + 1]);
               o[8 * j + 2 * e] = h0 + a0;
@@ -130,7 +132,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
             }
           }
         }
-        store32_bf16(p, o);
+        store32<DT>(p, o);
       }
     }
     if constexpr (EPI == kEpiResidSsq) {
@@ -154,7 +156,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
           const float gf = __uint_as_float(g[i]) * sc;
           o[i] = gf / (1.f + __expf(-gf)) * (__uint_as_float(u[i]) * sc);
         }
-        store32_bf16(ep.out + static_cast<int64_t>(m) * ep.ldo + tn * (BN / 2) + c, o);
+        store32<DT>(ep.out + static_cast<int64_t>(m) * ep.ldo + tn * (BN / 2) + c, o);
       }
     }
   } else {  // kEpiQkv
@@ -177,7 +179,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
 #pragma unroll 1
     for (int hb = 0; hb < BN / hd; ++hb) {
       const int head = (ep.col_offset + tn * BN + hb * hd) / hd;  // warp-uniform
-      __nv_bfloat16* dst;
+      s16* dst;
       bool rope = true;
       if (head < ep.hq) {
         dst = ep.q + static_cast<int64_t>(m) * ep.ldq + head * hd;
@@ -208,8 +210,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
               y1[2 * i + 1] = a1 * t.z - b1 * t.w;
               y2[2 * i + 1] = b1 * t.z + a1 * t.w;
             }
-            store32_bf16(dst + c, y1);
-            store32_bf16(dst + half + c, y2);
+            store32<DT>(dst + c, y1);
+            store32<DT>(dst + half + c, y2);
           }
         }
       } else {
@@ -222,7 +224,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]) * sc;
-            store32_bf16(dst + c, o);
+            store32<DT>(dst + c, o);
           }
         }
       }
@@ -231,7 +233,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
 }
 
 // -------------------------------------------------------------------- kernel
-template <int BN, int EPI>
+template <int BN, int EPI, int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_b2, const Shape sh, const EpiArgs ep) {
@@ -320,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // alone; a tcgen05 fence is taken only after the epilogue's release of an
     // accumulator (other threads' tcgen05.ld before this thread's MMAs).
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
+      const uint32_t idesc = umma_idesc<DT>(BM, BN, false, false);
       // Descriptors differ only in their start-address field (bytes >> 4), so
       // they are advanced by integer adds.
       const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)  // 16 columns = 32 bytes along the 128-byte swizzle row
-            umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(empty0 + 8 * stage);
           if (++stage == S) {
             stage = 0;
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn);
       const int m = tm * BM + wq * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + acc * BN;
-      epilogue_tile<BN, EPI>(tbase, m, tn, sh, ep);
+      epilogue_tile<BN, EPI, DT>(tbase, m, tn, sh, ep);
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
     }
@@ -416,7 +418,7 @@ struct PairCfg {
 };
 
 // sh.tiles_m counts 256-row pair tiles; gridDim.x = 2 * number of pairs.
-template <int EPI>
+template <int EPI, int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_b2, const Shape sh, const EpiArgs ep) {
@@ -517,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {  // one issuing thread, as in gemm_kernel
-      const uint32_t idesc = umma_idesc_bf16(C::kRows, C::BN, false, false);
+      const uint32_t idesc = umma_idesc<DT>(C::kRows, C::BN, false, false);
       const uint64_t adesc0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
       const uint64_t bdesc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
       int stage = 0, local = 0;
@@ -541,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit_pair(empty0 + 8 * stage, 3);
           if (++stage == S) {
             stage = 0;
@@ -569,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_coords(t, sh.tiles_m, sh.tiles_n, tm, tn, C::kGroupM);
       const int m = tm * C::kRows + static_cast<int>(rank) * BM + wq * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + acc * C::BN;
-      epilogue_tile<C::BN, EPI>(tbase, m, tn, sh, ep);
+      epilogue_tile<C::BN, EPI, DT>(tbase, m, tn, sh, ep);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_pair0 + 8 * acc);

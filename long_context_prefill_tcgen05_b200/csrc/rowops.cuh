@@ -9,7 +9,7 @@
 namespace dash {
 namespace rows {
 
-constexpr int kMaxVec = 16;  // 16-byte vectors per lane: rows of up to 4096 bf16
+constexpr int kMaxVec = 16;  // 16-byte vectors per lane: rows of up to 4096 16-bit elements
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -17,12 +17,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+template <int DT>
 __device__ __forceinline__ float sumsq8(const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float s = 0.f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const float a = bf16_lo(w[e]), b = bf16_hi(w[e]);
+    const float a = Num<DT>::lo(w[e]), b = Num<DT>::hi(w[e]);
     s = fmaf(a, a, fmaf(b, b, s));
   }
   return s;
@@ -35,14 +36,14 @@ __device__ __forceinline__ float sumsq8(const uint4& v) {
 // With row_scale given, the kernel writes y[r] = x[src(r)] * g and
 // row_scale[r] = rsqrt(mean(x^2) + eps) instead: the GEMM that consumes y
 // applies the scale to its fp32 accumulator, so the normalised activation is
-// never rounded to bf16 (x * g is exact in bf16 when g = 1).
-// Each warp issues its row's loads first; the block then stages g (d bf16,
-// dynamic shared memory) while they are in flight, so the scaling after the
+// never rounded to 16 bits (x * g is exact when g = 1).
+// Each warp issues its row's loads first; the block then stages g (d
+// elements, dynamic shared memory) while they are in flight, so the scaling after the
 // row's reduction waits on no second global load.
-__global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_rows,
-                               const int32_t* __restrict__ rowmap, int64_t rows, int d,
-                               const __nv_bfloat16* __restrict__ g, float eps,
-                               __nv_bfloat16* __restrict__ y, float* __restrict__ row_scale) {
+template <int DT>
+__global__ void rmsnorm_kernel(const s16* __restrict__ x, int64_t x_rows, const int32_t* __restrict__ rowmap,
+                               int64_t rows, int d, const s16* __restrict__ g, float eps, s16* __restrict__ y,
+                               float* __restrict__ row_scale) {
   extern __shared__ uint4 g_s[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
@@ -71,7 +72,7 @@ __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_ro
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < kMaxVec; ++i)
-    if (lane + 32 * i < nv) ss += sumsq8(v[i]);
+    if (lane + 32 * i < nv) ss += sumsq8<DT>(v[i]);
   ss = warp_sum(ss);
   float rs = rsqrtf(ss / static_cast<float>(d) + eps);
   if (row_scale) {
@@ -89,7 +90,8 @@ __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_ro
       uint32_t o[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        o[e] = pack_bf16(bf16_lo(xw[e]) * rs * bf16_lo(gw[e]), bf16_hi(xw[e]) * rs * bf16_hi(gw[e]));
+        o[e] = Num<DT>::pack(Num<DT>::lo(xw[e]) * rs * Num<DT>::lo(gw[e]),
+                             Num<DT>::hi(xw[e]) * rs * Num<DT>::hi(gw[e]));
       yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -97,10 +99,11 @@ __global__ void rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, int64_t x_ro
 
 // -------------------------------------------------------------------- score
 // Δ_t = ||U_t||_2, or ||U_t||_2 / ||H_t||_2 (one warp per row).
-constexpr int kRowChunks = 16;  // 16-byte chunks per lane in flight (a 4096-wide bf16 row)
+constexpr int kRowChunks = 16;  // 16-byte chunks per lane in flight (a 4096-wide 16-bit row)
 
-__global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ h,
-                             int64_t T, int d, int relative, float* __restrict__ delta) {
+template <int DT>
+__global__ void score_kernel(const s16* __restrict__ u, const s16* __restrict__ h, int64_t T, int d,
+                             int relative, float* __restrict__ delta) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
   if (r >= T) return;
@@ -117,7 +120,7 @@ __global__ void score_kernel(const __nv_bfloat16* __restrict__ u, const __nv_bfl
         if (c0 + 32 * u < nv) v[u] = __ldcs(row + c0 + 32 * u);
 #pragma unroll
       for (int u = 0; u < kRowChunks; ++u)
-        if (c0 + 32 * u < nv) acc += sumsq8(v[u]);
+        if (c0 + 32 * u < nv) acc += sumsq8<DT>(v[u]);
     }
     return acc;
   };
@@ -383,7 +386,7 @@ __global__ void seq_layout_kernel(const int32_t* __restrict__ cu, int nseq, cons
 // -------------------------------------------------------- gather / scatter
 // Y[i] = X[idx[i]] (gather) or X[idx[i]] = Y[i] (scatter); one warp per row.
 template <bool kScatter>
-__global__ void move_rows_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+__global__ void move_rows_kernel(const s16* __restrict__ src, s16* __restrict__ dst,
                                  const int32_t* __restrict__ idx, int64_t K, int64_t T, int d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t wpb = blockDim.x >> 5;

@@ -31,7 +31,12 @@ class DashError(RuntimeError):
 
 class Dims(ctypes.Structure):
     _fields_ = [("n_layers", c_i32), ("d_model", c_i32), ("n_heads", c_i32), ("n_kv_heads", c_i32),
-                ("head_dim", c_i32), ("ffn_dim", c_i32), ("rms_eps", c_f64), ("rope_theta", c_f64)]
+                ("head_dim", c_i32), ("ffn_dim", c_i32), ("rms_eps", c_f64), ("rope_theta", c_f64),
+                ("dtype", c_i32)]
+
+
+# dash_dtype codes of the 16-bit float formats a model may use
+DTYPES = {torch.bfloat16: 0, torch.float16: 1}
 
 
 class LayerWeights(ctypes.Structure):
@@ -244,14 +249,16 @@ def select(scores, kind="topk", keep=0.5, threshold=0.0, keep_first=0, keep_last
 def compact(X, idx, stream=None):
     K = idx.numel()
     Y = torch.empty(K, X.shape[1], dtype=X.dtype, device=X.device)
-    _check(lib().dash_compact(_t(X, BF16, "X"), X.shape[0], _t(idx, I32, "idx"), K, X.shape[1], _p(Y),
+    x_dtype = X.dtype if X.dtype in DTYPES else BF16  # rows are copied bit for bit: either 16-bit format
+    _check(lib().dash_compact(_t(X, x_dtype, "X"), X.shape[0], _t(idx, I32, "idx"), K, X.shape[1], _p(Y),
                               _stream(stream)), "dash_compact")
     return Y
 
 
 def scatter(Y, idx, X, stream=None):
-    _check(lib().dash_scatter(_t(Y, BF16, "Y", (idx.numel(), X.shape[1])), _t(idx, I32, "idx"), idx.numel(),
-                              X.shape[1], _t(X, BF16, "X"), X.shape[0], _stream(stream)), "dash_scatter")
+    x_dtype = X.dtype if X.dtype in DTYPES else BF16  # rows are copied bit for bit: either 16-bit format
+    _check(lib().dash_scatter(_t(Y, x_dtype, "Y", (idx.numel(), X.shape[1])), _t(idx, I32, "idx"), idx.numel(),
+                              X.shape[1], _t(X, x_dtype, "X"), X.shape[0], _stream(stream)), "dash_scatter")
     return X
 
 
@@ -297,13 +304,18 @@ def attention(Q, K, V, hq, hkv, hd, qpos=None, kstart=None, out=None, stream=Non
 # --------------------------------------------------------------- stack
 class Stack:
     """A decoder stack's dims plus its weights laid out for the library
-    (w_qkv = [wq; wk; wv] concatenated once, at load time)."""
+    (w_qkv = [wq; wk; wv] concatenated once, at load time).  The weights'
+    torch dtype (bfloat16 or float16) is the model's 16-bit format; hidden
+    states and caches passed with this stack must use it too."""
 
     def __init__(self, dims, layers):
         self.model = dims
+        self.dtype = layers[0]["wq"].dtype
+        if self.dtype not in DTYPES or any(t.dtype != self.dtype for w in layers for t in w.values()):
+            raise ValueError(f"weights must all be bfloat16 or all float16, got {self.dtype}")
         self.dims = Dims(dims.n_layers if len(layers) == dims.n_layers else len(layers), dims.d_model,
                          dims.n_heads, dims.n_kv_heads, dims.head_dim, dims.ffn_dim, dims.rms_eps,
-                         dims.rope_theta)
+                         dims.rope_theta, DTYPES[self.dtype])
         self.tensors = []
         arr = (LayerWeights * len(layers))()
         for i, w in enumerate(layers):
@@ -325,7 +337,7 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
         active, halted, h_full = halt
         T_kv = h_full.shape[0]
         _t(active, I32, "active_idx", (M,))
-        _t(h_full, BF16, "h_full", (T_kv, H.shape[1]))
+        _t(h_full, stack.dtype, "h_full", (T_kv, H.shape[1]))
         if halted.numel():
             _t(halted, I32, "halted_idx", (T_kv - M,))
         hctx = HaltCtx(active.data_ptr(), halted.data_ptr() if halted.numel() else None, h_full.data_ptr(), T_kv)
@@ -335,7 +347,7 @@ def layer_forward(stack, l, H, pos=None, max_pos=None, halt=None, delta=None, re
     need = lib().dash_layer_workspace_size(ctypes.byref(stack.dims), M, T_kv, max_pos)
     ws = workspace(need, H.device)
     w = ctypes.pointer(stack.layers[l])
-    _check(lib().dash_layer_forward(ctypes.byref(stack.dims), w, _t(H, BF16, "H", (M, stack.dims.d_model)),
+    _check(lib().dash_layer_forward(ctypes.byref(stack.dims), w, _t(H, stack.dtype, "H", (M, stack.dims.d_model)),
                                     M, _t(pos, I32, "pos", (M,)), max_pos,
                                     ctypes.byref(hctx) if hctx is not None else None, _out(delta, F32, "delta", M),
                                     int(relative),
@@ -360,7 +372,8 @@ def prefill_varlen(stack, H, cu_seqlens, cfg, idx_out=None, delta_out=None, stre
     cu_arr = (c_i32 * (nseq + 1))(*cu)
     counts = (c_i32 * nseq)()
     K = c_i64(0)
-    _check(lib().dash_prefill_varlen(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)),
+    _check(lib().dash_prefill_varlen(ctypes.byref(stack.dims), stack.layers,
+                                     _t(H, stack.dtype, "H", (T, stack.dims.d_model)),
                                      cu_arr, nseq, ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T),
                                      ctypes.byref(K), counts, _out(delta_out, F32, "delta_out", T), _p(ws), ws.numel(),
                                      _stream(stream)), "dash_prefill_varlen")
@@ -373,7 +386,7 @@ def prefill(stack, H, cfg, idx_out=None, delta_out=None, stream=None):
     need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
     ws = workspace(need, H.device)
     K = c_i64(0)
-    _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)), T,
+    _check(lib().dash_prefill(ctypes.byref(stack.dims), stack.layers, _t(H, stack.dtype, "H", (T, stack.dims.d_model)), T,
                               ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T), ctypes.byref(K),
                               _out(delta_out, F32, "delta_out", T), _p(ws), ws.numel(), _stream(stream)),
            "dash_prefill")
@@ -398,7 +411,7 @@ class KVCache:
         self.desc = (KVCacheDesc * (nseq * L))()
         for s in range(nseq):
             for l in range(L):
-                k = torch.zeros(max(caps[l], 1), kvd, dtype=torch.bfloat16, device=device)
+                k = torch.zeros(max(caps[l], 1), kvd, dtype=stack.dtype, device=device)
                 v = torch.zeros_like(k)
                 p = torch.full((max(caps[l], 1),), -1, dtype=torch.int32, device=device) if with_pos else None
                 self.k.append(k)
@@ -423,7 +436,8 @@ def prefill_kv(stack, H, cfg, cache, idx_out=None, delta_out=None, stream=None):
     need = lib().dash_prefill_workspace_size(ctypes.byref(stack.dims), T, ctypes.byref(cfg))
     ws = workspace(need, H.device)
     K = c_i64(0)
-    _check(lib().dash_prefill_kv(ctypes.byref(stack.dims), stack.layers, _t(H, BF16, "H", (T, stack.dims.d_model)), T,
+    _check(lib().dash_prefill_kv(ctypes.byref(stack.dims), stack.layers, _t(H, stack.dtype, "H", (T, stack.dims.d_model)),
+                                 T,
                                  ctypes.byref(cfg), _out(idx_out, I32, "idx_out", T), ctypes.byref(K),
                                  _out(delta_out, F32, "delta_out", T), cache.desc, _p(ws), ws.numel(),
                                  _stream(stream)), "dash_prefill_kv")
@@ -441,7 +455,7 @@ def prefill_varlen_kv(stack, H, cu_seqlens, cfg, cache, idx_out=None, delta_out=
     counts = (c_i32 * nseq)()
     K = c_i64(0)
     _check(lib().dash_prefill_varlen_kv(ctypes.byref(stack.dims), stack.layers,
-                                        _t(H, BF16, "H", (T, stack.dims.d_model)), cu_arr, nseq, ctypes.byref(cfg),
+                                        _t(H, stack.dtype, "H", (T, stack.dims.d_model)), cu_arr, nseq, ctypes.byref(cfg),
                                         _out(idx_out, I32, "idx_out", T), ctypes.byref(K), counts,
                                         _out(delta_out, F32, "delta_out", T), cache.desc, _p(ws), ws.numel(),
                                         _stream(stream)), "dash_prefill_varlen_kv")
@@ -455,7 +469,7 @@ def decode_step(stack, X, pos, cache, stream=None):
     need = lib().dash_decode_workspace_size(ctypes.byref(stack.dims), n)
     ws = workspace(need, X.device)
     pos_arr = (c_i32 * n)(*[int(p) for p in pos])
-    _check(lib().dash_decode_step(ctypes.byref(stack.dims), stack.layers, _t(X, BF16, "X", (n, stack.dims.d_model)),
+    _check(lib().dash_decode_step(ctypes.byref(stack.dims), stack.layers, _t(X, stack.dtype, "X", (n, stack.dims.d_model)),
                                   n, pos_arr, cache.desc, _p(ws), ws.numel(), _stream(stream)), "dash_decode_step")
     return X
 

@@ -65,6 +65,8 @@ def test_argument_errors_are_caught_on_the_host(L):
     assert call(_dims(head_dim=96), layers, FAKE, 512, cfg) == 2         # unsupported head_dim
     assert call(_dims(n_heads=3), layers, FAKE, 512, cfg) == 2           # hq % hkv != 0
     assert call(_dims(d_model=200), layers, FAKE, 512, cfg) == 2         # d % 128 != 0
+    assert call(_dims(dtype=2), layers, FAKE, 512, cfg) == 2             # no such 16-bit format
+    assert call(_dims(dtype=1), layers, FAKE, 512, cfg, None, 0) == 4    # fp16 accepted (then: no workspace)
     assert call(dims, layers, FAKE + 2, 512, cfg) == 1                   # misaligned H
     bad = dash.make_config(halt_layer=4, mode="prune")
     assert call(dims, layers, FAKE, 512, bad) == 1                       # halt layer out of range
@@ -198,6 +200,15 @@ def test_binding_refuses_tensors_the_library_would_misread(L):
     assert dash._t(None, torch.bfloat16, "x") is None
     with pytest.raises(ValueError, match="at least 9"):
         dash._out(torch.zeros(8, dtype=torch.int32), torch.int32, "idx_out", 9)
+    # a stack takes its 16-bit format from its weights, all of one format
+    w = {k: v.half() for k, v in inputs.make_layers(inputs.TINY, n_layers=1)[0].items()}
+    st = dash.Stack(inputs.TINY, [w])
+    assert st.dtype == torch.float16 and st.dims.dtype == 1
+    mixed = dict(w, wo=w["wo"].bfloat16())
+    with pytest.raises(ValueError, match="all float16"):
+        dash.Stack(inputs.TINY, [mixed])
+    with pytest.raises(ValueError, match="float16"):
+        dash.prefill(st, bf, dash.make_config())         # bf16 hidden states for an fp16 stack
 
 
 def test_headers_compile_and_link_as_plain_c(L, tmp_path):
