@@ -180,7 +180,7 @@ def cpu_threads():
 
 
 def oracle_sample_time(dims, layer_np, T_s, seed=0):
-    """Seconds for the oracle to run one Qwen-shaped decoder block on T_s tokens."""
+    """Seconds for the oracle to run one decoder block of the stack on T_s tokens."""
     import numpy as np
     import oracle as O
     h = inputs.make_hidden(T_s, dims.d_model, seed=seed)[0].double().numpy()
@@ -195,49 +195,62 @@ def cpu_layer_np(dims):
     return {k: v.double().numpy() for k, v in layer.items()}
 
 
-def cpu_baseline(dims, T, target_flops, budget_s=15.0):
-    """The oracle timed on host cores on a bounded sample (one decoder block
-    on T_s tokens), extrapolated by algorithmic FLOPs to the whole workload."""
+def cpu_sample_tokens(dims, T):
+    """Tokens of the bounded CPU sample: one decoder block on 2048 tokens for
+    the 7B/8B-shaped stacks (a few seconds of fp64 work on 16 cores), the
+    whole sequence for the tiny stack."""
+    return min(T, 2048)
+
+
+def cpu_rate(dims, T, target_flops, t, T_s):
+    """tokens/s of the whole workload from one sample: T_s tokens through one
+    block in t seconds, extrapolated by algorithmic FLOPs."""
+    f_s = T_s * costs.linear_flops_per_token(dims) + costs.attn_flops(dims, costs.causal_pairs(T_s))
+    return T / (t * target_flops / f_s), f_s
+
+
+def cpu_baseline(dims, T, target_flops, samples=3):
+    """The oracle timed on host cores on a bounded sample of the workload --
+    the same sample the reference arm times per step -- median of `samples`."""
     layer_np = cpu_layer_np(dims)
-    lin = costs.linear_flops_per_token(dims)
-    T_s, t = 32, oracle_sample_time(dims, layer_np, 32)
-    while t < budget_s / 4 and T_s < 2048:
-        T_s = min(2048, int(T_s * max(2.0, budget_s / 2 / max(t, 1e-3))))
-        t = oracle_sample_time(dims, layer_np, T_s)
-    f_s = T_s * lin + costs.attn_flops(dims, costs.causal_pairs(T_s))
-    est_s = t * target_flops / f_s
-    return {"value": T / est_s, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+    T_s = cpu_sample_tokens(dims, T)
+    ts = [oracle_sample_time(dims, layer_np, T_s) for _ in range(samples)]
+    t = statistics.median(ts)
+    value, f_s = cpu_rate(dims, T, target_flops, t, T_s)
+    return {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
             "sample": f"one decoder block of the same stack on {T_s} tokens ({f_s / 1e9:.0f} GFLOP fp64, "
-                      f"{t:.1f} s), extrapolated by algorithmic FLOPs to the full prefill",
+                      f"median {t:.2f} s of {samples}), extrapolated by algorithmic FLOPs to the full prefill",
             "sample_seconds": t}
 
 
 # ------------------------------------------------------------ reference
 def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores: each step is the bounded
+    sample cpu_baseline takes (one block on the same tokens), extrapolated
+    the same way; rank 0 alone runs it."""
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
     dims, T = wl["dims"], wl["T"]
+    mode = args.mode or wl["mode"]
     K = math.floor(wl["keep"] * T)
-    target = costs.prefill_flops(dims, T, wl["halt_layer"], K, "prune")
+    target = costs.prefill_flops(dims, T, wl["halt_layer"], K, mode)
     layer_np = cpu_layer_np(dims)
-    T_s = 64 if dims.d_model > 1024 else T
-    lin = costs.linear_flops_per_token(dims)
-    f_s = T_s * lin + costs.attn_flops(dims, costs.causal_pairs(T_s))
+    T_s = cpu_sample_tokens(dims, T)
     for _ in range(args.warmup):
         oracle_sample_time(dims, layer_np, T_s)
     ts = [oracle_sample_time(dims, layer_np, T_s) for _ in range(args.steps)]
     t = sum(ts) / len(ts)
-    value = T / (t * target / f_s)
+    value, f_s = cpu_rate(dims, T, target, t, T_s)
     cb = {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-          "sample": f"each step: one decoder block on {T_s} tokens ({f_s / 1e9:.1f} GFLOP fp64), "
-                    f"extrapolated by algorithmic FLOPs to the full halted prefill"}
+          "sample": f"each step: one decoder block of the same stack on {T_s} tokens ({f_s / 1e9:.0f} GFLOP fp64, "
+                    f"mean {t:.2f} s), extrapolated by algorithmic FLOPs to the full halted prefill"}
     print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
                       "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                       "ms_per_step": t * target / f_s * 1e3, "higher_is_better": True, "scaling": "weak",
                       "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                       "config": {"workload": wl["name"], "seq_len": T, "halt_layer": wl["halt_layer"],
-                                 "keep": wl["keep"], "mode": "prune"},
+                                 "keep": wl["keep"], "mode": mode},
                       "cpu_baseline": cb,
                       "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                               "d2h_bytes_per_step": 0}}), flush=True)
@@ -324,6 +337,224 @@ def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, 
     return out
 
 
+# ------------------------------------------------------------ prefill legs
+class Prefill:
+    """One workload's buffers and its prefill step on a stack (inputs resident)."""
+
+    def __init__(self, dash, stack, h0, cu, world):
+        self.dash, self.stack, self.h0, self.cu, self.world = dash, stack, h0, cu, world
+        T = h0.shape[0]
+        self.H = torch.empty_like(h0)
+        self.idx = torch.empty(T, dtype=torch.int32, device=h0.device)
+        self.delta = torch.empty(T, dtype=torch.float32, device=h0.device)
+
+    def run(self, c, H=None, stream=None):
+        H = self.H if H is None else H
+        if self.cu:
+            return self.dash.prefill_varlen(self.stack, H, self.cu, c, idx_out=self.idx, delta_out=self.delta,
+                                            stream=stream)[0]
+        return self.dash.prefill(self.stack, H, c, idx_out=self.idx, delta_out=self.delta, stream=stream)
+
+    def step(self, c):
+        self.H.copy_(self.h0)
+        return self.run(c)
+
+    def timed(self, c, k, record=False):
+        """ms per step over k steps (max over ranks), the last K, and the launch
+        records when record is set (CUDA events around every launch)."""
+        torch.cuda.synchronize()
+        barrier(self.world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if record:
+            self.dash.timing_start()
+        e0.record()
+        K = None
+        for _ in range(k):
+            K = self.step(c)
+        e1.record()
+        torch.cuda.synchronize()
+        recs = self.dash.timing_stop() if record else None
+        barrier(self.world)
+        return max_over_ranks(e0.elapsed_time(e1) / k, self.world), K, recs
+
+    def calibrate_threshold(self, wl, mode):
+        """The relative-Δ threshold that keeps ~wl['keep'] of the tokens: Δ at
+        rank floor(keep T) of a top-k prefill on the same input, then frozen."""
+        cal = self.dash.make_config(halt_layer=wl["halt_layer"], mode=mode, select="topk", keep=wl["keep"],
+                                    relative=wl["relative"])
+        self.step(cal)
+        k = math.floor(wl["keep"] * self.h0.shape[0])
+        return float(torch.sort(self.delta.cpu(), descending=True).values[k - 1])
+
+
+def work_accounting(dims, T, cu, mode, halt_layer, K, active):
+    """(halted FLOPs, visible pairs by attention query rows) of one prefill."""
+    if cu:
+        counts = [int(((active >= a) & (active < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
+        flops = costs.varlen_prefill_flops(dims, cu, halt_layer, counts, mode, active)
+        seq_of = lambda i: max(s for s in range(len(cu) - 1) if cu[s] <= i)
+        pairs = {T: sum(costs.causal_pairs(b - a) for a, b in zip(cu[:-1], cu[1:]))}
+        pairs[K] = (sum(costs.causal_pairs(k) for k in counts) if mode == "prune"
+                    else int(sum(int(i) - cu[seq_of(int(i))] + 1 for i in active)))
+    else:
+        flops = costs.prefill_flops(dims, T, halt_layer, K, mode, active)
+        pairs = {T: costs.causal_pairs(T), K: int(sum(int(i) + 1 for i in active))
+                 if mode == "halt" else costs.causal_pairs(K)}
+    return flops, pairs
+
+
+def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
+    """Per-kernel time and rate of `steps` instrumented steps, and the roofline
+    of the dominant kernel (the kind with the most time)."""
+    per = {}
+    for r in recs:
+        unit, amount = costs.launch_work(r, dims, pairs_by_rows)
+        p = per.setdefault(r["kind"], {"launches": 0, "ms": 0.0, "unit": unit, "work": 0})
+        p["launches"] += 1
+        p["ms"] += r["ms"]
+        p["work"] += amount
+    total_ms = sum(p["ms"] for p in per.values())
+    kernels = {}
+    for kind, p in sorted(per.items(), key=lambda kv: -kv[1]["ms"]):
+        rate = p["work"] / (p["ms"] / 1e3) if p["ms"] > 0 else 0.0
+        kernels[kind] = {"launches_per_step": p["launches"] // steps, "ms_per_step": p["ms"] / steps,
+                         "share": p["ms"] / total_ms if total_ms else 0.0,
+                         ("tflops" if p["unit"] == "flop" else "gbs"): rate / 1e12 if p["unit"] == "flop"
+                         else rate / 1e9}
+    dom_kind = max(per, key=lambda k: per[k]["ms"])
+    dom = per[dom_kind]
+    if dom["unit"] == "flop":
+        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+    else:
+        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof.update({"kernel": dom_kind, "traffic": recorded_traffic(dom_kind, recs),
+                 "peak_source": f"{peaks['source']} ({'sustained bf16' if dom['unit'] == 'flop' else 'HBM copy'})"})
+    return kernels, roof, len(recs) // steps
+
+
+def long_context_leg(dash, stack, dims, dev, peaks, world, rounds=2):
+    """The T = 131072 workload on the same stack: halt mode with the relative-Δ
+    threshold calibrated to keep ~30 %, against the dense prefill on the same
+    kernels (single steps alternating), with its own kernel roofline."""
+    wl = WORKLOADS["qwen7b-128k"]
+    T = wl["T"]
+    h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=dev, span_rows=wl["span_rows"],
+                               span_len=wl["span_len"])
+    pf = Prefill(dash, stack, h0, None, world)
+    thr = pf.calibrate_threshold(wl, wl["mode"])
+    cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=wl["mode"], select="threshold", threshold=thr,
+                           relative=True)
+    cfg_dense = dash.make_config(mode="dense")
+    pf.step(cfg)
+    pf.step(cfg_dense)
+    legs = [(cfg, []), (cfg_dense, [])]
+    for r in range(rounds):
+        for c, times in (legs if r % 2 == 0 else legs[::-1]):
+            times.append(pf.timed(c, 1)[0])
+    ms_h, ms_d = (statistics.median(t) for _, t in legs)
+    _, K, recs = pf.timed(cfg, 1, record=True)
+    active = pf.idx[:K].cpu().numpy()
+    flops, pairs = work_accounting(dims, T, None, wl["mode"], wl["halt_layer"], K, active)
+    dense_flops = costs.prefill_flops(dims, T)
+    kernels, roof, launches = kernel_breakdown(recs, dims, pairs, 1, peaks)
+    dash.check_device()
+    out = {"workload": wl["name"], "threshold": thr, "K": K, "kept": K / T,
+           "value": world * T / (ms_h / 1e3), "unit": "tokens/s", "ms_per_step": ms_h,
+           "dense": {"tokens_per_s": world * T / (ms_d / 1e3), "ms_per_step": ms_d,
+                     "tflops": dense_flops / (ms_d / 1e3) / 1e12},
+           "speedup_vs_dense": ms_d / ms_h, "flop_bound": dense_flops / flops,
+           "halted_tflop_per_step": flops / 1e12, "step_tflops": flops / (ms_h / 1e3) / 1e12,
+           "roofline": roof, "kernels": {k: v for k, v in list(kernels.items())[:6]},
+           "gpu_launches_per_step": launches,
+           "timing": f"median of {rounds} single steps per leg, halt / dense alternating; inputs larger than L2"}
+    del pf, h0
+    torch.cuda.empty_cache()
+    return out
+
+
+def fp16_leg(dash, wl, dims, h0, cu, cfg, pf16_of, pf_bf16, world, rounds=3):
+    """The same workload with the model stored in fp16 (dash_dims.dtype =
+    fp16: weights and every stored activation 16-bit fp16, fp32 accumulation),
+    timed in single steps alternating with the bf16 path."""
+    pf16 = pf16_of()
+    pf16.step(cfg)
+    legs = [(pf_bf16, []), (pf16, [])]
+    for r in range(rounds):
+        for p, times in (legs if r % 2 == 0 else legs[::-1]):
+            times.append(p.timed(cfg, 1)[0])
+    ms_b, ms_h = (statistics.median(t) for _, t in legs)
+    dash.check_device()
+    T = h0.shape[0]
+    out = {"dtype": "f16", "value": world * T / (ms_h / 1e3), "unit": "tokens/s", "ms_per_step": ms_h,
+           "bf16_ms_per_step": ms_b, "cost_vs_bf16": ms_h / ms_b,
+           "timing": f"median of {rounds} single steps per format, alternating",
+           "note": "fp16 storage holds the stated delta tolerance at the halting depth (tests/test_gpu_fp16.py)"}
+    del pf16
+    torch.cuda.empty_cache()
+    return out
+
+
+def score_select_leg(dash, dev, peaks, reps=20):
+    """The score / select / compaction workload on its own: U, H bf16
+    [32768, 3584] N(0,1), 10 % of U's rows x4 in 64-row spans (seed 1); Δ
+    absolute and relative; top-k keep 0.5 and threshold = the median Δ
+    (sorted int32 lists); gather of the K = 16384 kept rows.  Each launch is
+    timed alone after a write of 256 MB (larger than L2), median of reps."""
+    T, d = 32768, inputs.QWEN7B.d_model
+    U, H, mask = inputs.make_score_bench_inputs(T, d, seed=1, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = dash.lib()
+    delta = torch.empty(T, device=dev)
+    delta_r = torch.empty(T, device=dev)
+    idx = torch.empty(T, dtype=torch.int32, device=dev)
+    count = torch.empty(1, dtype=torch.int32, device=dev)
+    dash.score(U, out=delta)
+    med = float(torch.median(delta).item())
+    K = math.floor(0.5 * T)
+    sel = dash.select(delta, "topk", 0.5)[0].clone()
+    Y = torch.empty(K, d, dtype=torch.bfloat16, device=dev)
+
+    def cold(fn):
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    def select_call(kind, keep, thr):
+        return lambda: L.dash_select(dash._p(delta), T, dash.SELECTS[kind], keep, thr, 0, 0, dash._p(idx), None,
+                                     dash._p(count), None, 0, None)
+    cases = {
+        "score_abs": (lambda: dash.score(U, out=delta), T * d * 2 + 4 * T),
+        "score_rel": (lambda: dash.score(U, H, relative=True, out=delta_r), 2 * T * d * 2 + 4 * T),
+        "select_topk_keep0.5": (select_call("topk", 0.5, 0.0), 4 * T + 4 * K + 4),
+        "select_threshold_median": (select_call("threshold", 0.0, med), 4 * T + 4 * (T // 2) + 4),
+        "gather_K16384": (lambda: dash.compact(U, sel), 2 * K * d * 2 + 4 * K),
+    }
+    out = {}
+    for name, (fn, nbytes) in cases.items():
+        ms = cold(fn)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"us": ms * 1e3, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+    dash.check_device()
+    out["workload"] = ("U, H bf16 [32768, 3584] N(0,1), 3264 rows of U x4 in 51 spans of 64 (seed 1); "
+                       "top-k keep 0.5 (K = 16384) and threshold = median delta")
+    out["timing"] = f"each launch alone after a 256 MB L2-flushing write, median of {reps}"
+    del U, H, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ ours
 def main():
     ap = argparse.ArgumentParser()
@@ -334,8 +565,10 @@ def main():
     ap.add_argument("--mode", default=None, choices=["prune", "halt"], help="default: the workload's mode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extra", action="store_true", help="skip the dense / other-mode / e2e legs")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the dense / other-mode / e2e / fp16 / 128K / score-select legs")
     ap.add_argument("--no-decode", action="store_true", help="skip the generation leg")
+    ap.add_argument("--no-128k", action="store_true", help="skip the T=131072 leg")
     args = ap.parse_args()
     if args.impl == "reference":
         # rank 0 alone times the oracle on the host cores; the other ranks exit at once
@@ -357,7 +590,8 @@ def main():
     args.mode = args.mode or wl["mode"]
     peaks = load_peaks()
 
-    stack = dash.Stack(dims, inputs.make_layers(dims, seed=0, device=dev))
+    layers = inputs.make_layers(dims, seed=0, device=dev)
+    stack = dash.Stack(dims, layers)
     varlen = wl.get("varlen", False)
     cu = None
     if varlen:
@@ -366,97 +600,30 @@ def main():
     else:
         h0, _ = inputs.make_hidden(T, dims.d_model, seed=0, device=dev, span_rows=wl["span_rows"],
                                    span_len=wl["span_len"])
-    H = torch.empty_like(h0)
-    idx = torch.empty(T, dtype=torch.int32, device=dev)
-    delta = torch.empty(T, dtype=torch.float32, device=dev)
-    def run(c):
-        if varlen:
-            return dash.prefill_varlen(stack, H, cu, c, idx_out=idx, delta_out=delta)[0]
-        return dash.prefill(stack, H, c, idx_out=idx, delta_out=delta)
-
-    threshold = 0.0
-    if wl.get("calibrate"):
-        cal = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select="topk", keep=wl["keep"],
-                               relative=wl["relative"])
-        H.copy_(h0)
-        run(cal)
-        kcal = math.floor(wl["keep"] * T)
-        threshold = float(torch.sort(delta.cpu(), descending=True).values[kcal - 1])
+    pf = Prefill(dash, stack, h0, cu, world)
+    threshold = pf.calibrate_threshold(wl, args.mode) if wl.get("calibrate") else 0.0
     cfg = dash.make_config(halt_layer=wl["halt_layer"], mode=args.mode, select=wl["select"], keep=wl["keep"],
                            threshold=threshold, relative=wl["relative"])
     cfg_dense = dash.make_config(mode="dense")
 
-    def step(c):
-        H.copy_(h0)
-        return run(c)
-
-    def timed(c, k, record=False):
-        torch.cuda.synchronize()
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if record:
-            dash.timing_start()
-        e0.record()
-        K = None
-        for _ in range(k):
-            K = step(c)
-        e1.record()
-        torch.cuda.synchronize()
-        recs = dash.timing_stop() if record else None
-        barrier(world)
-        return max_over_ranks(e0.elapsed_time(e1) / k, world), K, recs
-
     for _ in range(args.warmup):
-        step(cfg)
+        pf.step(cfg)
     dash.check_device()
+    # The headline: K steps with no per-launch instrumentation.
     clock = ClockSampler(local)
     clock.start()
-    ms, K, recs = timed(cfg, args.steps, record=True)
+    ms, K, _ = pf.timed(cfg, args.steps)
     clocks = clock.stop()
     dash.check_device()
-    active = idx[:K].cpu().numpy()
-    if varlen:
-        counts = [int(((active >= a) & (active < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
-        halted_flops = costs.varlen_prefill_flops(dims, cu, wl["halt_layer"], counts, args.mode, active)
-        seq_of = lambda i: max(s for s in range(len(cu) - 1) if cu[s] <= i)
-        pairs_by_rows = {T: sum(costs.causal_pairs(b - a) for a, b in zip(cu[:-1], cu[1:]))}
-        pairs_by_rows[K] = (sum(costs.causal_pairs(k) for k in counts) if args.mode == "prune"
-                            else int(sum(int(i) - cu[seq_of(int(i))] + 1 for i in active)))
-    else:
-        halted_flops = costs.prefill_flops(dims, T, wl["halt_layer"], K, args.mode, active)
-        pairs_by_rows = {T: costs.causal_pairs(T), K: int(sum(int(i) + 1 for i in active))
-                         if args.mode == "halt" else costs.causal_pairs(K)}
+    active = pf.idx[:K].cpu().numpy()
+    halted_flops, pairs_by_rows = work_accounting(dims, T, cu, args.mode, wl["halt_layer"], K, active)
     value = world * T / (ms / 1e3)
-
-    # per-kernel breakdown of the timed steps (CUDA events around every launch)
-    per = {}
-    for r in recs:
-        unit, amount = costs.launch_work(r, dims, pairs_by_rows)
-        p = per.setdefault(r["kind"], {"launches": 0, "ms": 0.0, "unit": unit, "work": 0})
-        p["launches"] += 1
-        p["ms"] += r["ms"]
-        p["work"] += amount
-    total_ms = sum(p["ms"] for p in per.values())
-    kernels = {}
-    for kind, p in sorted(per.items(), key=lambda kv: -kv[1]["ms"]):
-        rate = p["work"] / (p["ms"] / 1e3) if p["ms"] > 0 else 0.0
-        kernels[kind] = {"launches_per_step": p["launches"] // args.steps, "ms_per_step": p["ms"] / args.steps,
-                         "share": p["ms"] / total_ms if total_ms else 0.0,
-                         ("tflops" if p["unit"] == "flop" else "gbs"): rate / 1e12 if p["unit"] == "flop"
-                         else rate / 1e9}
-    dom_kind = max(per, key=lambda k: per[k]["ms"])
-    dom = per[dom_kind]
-    if dom["unit"] == "flop":
-        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    else:
-        achieved = dom["work"] / (dom["ms"] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
-    roof.update({"kernel": dom_kind, "traffic": recorded_traffic(dom_kind, recs),
-                 "peak_source": f"{peaks['source']} ({'sustained bf16' if dom['unit'] == 'flop' else 'HBM copy'})",
-                 "step_tflops": halted_flops / (ms / 1e3) / 1e12})
+    # A separate instrumented pass (CUDA events around every launch) gives the
+    # per-kernel breakdown and the dominant kernel's roofline.
+    n_rec = 2
+    _, _, recs = pf.timed(cfg, n_rec, record=True)
+    kernels, roof, launches_per_step = kernel_breakdown(recs, dims, pairs_by_rows, n_rec, peaks)
+    roof["step_tflops"] = halted_flops / (ms / 1e3) / 1e12
 
     extra = {}
     if not args.no_extra:
@@ -467,20 +634,15 @@ def main():
         # Dense, this mode and the other mode are timed in alternating single
         # steps (medians over the rounds), so a drift of the power-capped clock
         # during the run does not bias their ratios.
-        step(cfg_dense)
-        step(cfg_o)
+        pf.step(cfg_dense)
+        pf.step(cfg_o)
         legs = [(cfg_dense, []), (cfg, []), (cfg_o, [])]
         for r in range(max(3, args.steps)):
             for c, times in legs[r % 3:] + legs[:r % 3]:
-                times.append(timed(c, 1)[0])
+                times.append(pf.timed(c, 1)[0])
         ms_d, ms_m, ms_o = (statistics.median(t) for _, t in legs)
-        _, K_o, _ = timed(cfg_o, 1)  # the other mode's active set, for its FLOP count
-        act_o = idx[:K_o].cpu().numpy()
-        if varlen:
-            cnt_o = [int(((act_o >= a) & (act_o < b)).sum()) for a, b in zip(cu[:-1], cu[1:])]
-            flops_o = costs.varlen_prefill_flops(dims, cu, wl["halt_layer"], cnt_o, other, act_o)
-        else:
-            flops_o = costs.prefill_flops(dims, T, wl["halt_layer"], K_o, other, act_o)
+        _, K_o, _ = pf.timed(cfg_o, 1)  # the other mode's active set, for its FLOP count
+        flops_o, _ = work_accounting(dims, T, cu, other, wl["halt_layer"], K_o, pf.idx[:K_o].cpu().numpy())
         extra = {
             "dense": {"tokens_per_s": world * T / (ms_d / 1e3), "ms_per_step": ms_d,
                       "tflops": dense_flops / (ms_d / 1e3) / 1e12},
@@ -501,14 +663,9 @@ def main():
         h_host = h0.cpu().pin_memory()
         out_host = torch.empty(T, dims.d_model, dtype=torch.bfloat16).pin_memory()
         comp, copy = torch.cuda.Stream(), torch.cuda.Stream()
-        bufs = [H, torch.empty_like(H)]
+        bufs = [pf.H, torch.empty_like(pf.H)]
         ready = [torch.cuda.Event(), torch.cuda.Event()]
         done = [torch.cuda.Event(), torch.cuda.Event()]
-
-        def run_on(buf, c):
-            if varlen:
-                return dash.prefill_varlen(stack, buf, cu, c, idx_out=idx, delta_out=delta, stream=comp)[0]
-            return dash.prefill(stack, buf, c, idx_out=idx, delta_out=delta, stream=comp)
 
         def e2e_run(n):
             rows = T
@@ -522,7 +679,7 @@ def main():
                         nxt.copy_(h_host, non_blocking=True)
                         ready[(i + 1) % 2].record(copy)
                 comp.wait_event(ready[i % 2])
-                k = run_on(cur, cfg)
+                k = pf.run(cfg, H=cur, stream=comp)
                 done[i % 2].record(comp)
                 rows = k if args.mode == "prune" else T
                 copy.wait_event(done[i % 2])
@@ -541,6 +698,16 @@ def main():
         ms_e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
         extra["e2e"] = {"value": world * T / (ms_e / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": T * dims.d_model * 2, "d2h_bytes_per_step": rows * dims.d_model * 2}
+        del bufs, h_host, out_host
+        torch.cuda.empty_cache()
+
+        def pf16_of():
+            s16 = dash.Stack(dims, [{k: v.half() for k, v in w.items()} for w in layers])
+            return Prefill(dash, s16, h0.half(), cu, world)
+        extra["fp16"] = fp16_leg(dash, wl, dims, h0, cu, cfg, pf16_of, pf, world)
+        if args.workload == "qwen7b-32k" and not args.no_128k:
+            extra["t128k"] = long_context_leg(dash, stack, dims, dev, peaks, world)
+        extra["score_select"] = score_select_leg(dash, dev, peaks)
     dash.check_device()
     if not args.no_decode:
         # the cache of a prune-mode prefill with the workload's selection
@@ -561,7 +728,9 @@ def main():
                    "l2": (f"inputs larger than L2 ({wbytes / 1e9:.1f} GB of weights per step)" if wbytes > 126e6 else
                           "inputs fit in L2 (a small parity workload, not a headline figure)")},
         "K": K, "halted_tflop_per_step": halted_flops / 1e12,
-        "gpu_launches": len(recs), "roofline": roof, "kernels": kernels, "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps, "roofline": roof, "kernels": kernels,
+        "kernels_timing": f"separate pass of {n_rec} steps with CUDA events around every launch",
+        "clocks": clocks,
     }
     out.update(extra)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -1,23 +1,26 @@
 """Runs one kernel of the DASH prefill path at a chosen shape (for timing and
 for ncu captures of a single kernel on a small case).
 
-    python -m long_context_prefill_tcgen05_b200.kernel_cases attention --T 8192
-    python -m long_context_prefill_tcgen05_b200.kernel_cases linear --M 4096 --N 37888 --K 3584
-    python -m long_context_prefill_tcgen05_b200.kernel_cases layer --T 4096
-    python -m long_context_prefill_tcgen05_b200.kernel_cases select --T 32768
-    python -m long_context_prefill_tcgen05_b200.kernel_cases decode --T 32768 --M 1
-    python -m long_context_prefill_tcgen05_b200.kernel_cases decode_attention --T 32768 --M 1
-    python -m long_context_prefill_tcgen05_b200.kernel_cases rows --T 32768
+    python benchmarks/kernel_cases.py attention --T 8192
+    python benchmarks/kernel_cases.py linear --M 4096 --N 37888 --K 3584
+    python benchmarks/kernel_cases.py layer --T 4096
+    python benchmarks/kernel_cases.py select --T 32768
+    python benchmarks/kernel_cases.py decode --T 32768 --M 1
+    python benchmarks/kernel_cases.py decode_attention --T 32768 --M 1
+    python benchmarks/kernel_cases.py rows --T 32768
 
 Shapes default to the Qwen2.5-7B-shaped stack (28 q / 4 kv heads, hd 128,
 d 3584, FFN 18944).  Prints one JSON line with the mean CUDA-event time.
 """
 import argparse
 import json
+import os
+import sys
 
 import torch
 
-from . import build, costs, dash, inputs
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+from long_context_prefill_tcgen05_b200 import build, costs, dash, inputs  # noqa: E402
 
 
 def _time(fn, iters, warmup):

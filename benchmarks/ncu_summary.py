@@ -2,7 +2,7 @@
 of a bench.py run: per kernel, the launches, total time and share of the last
 prefill step (the launches from the last RoPE-table build to the end).
 
-    python -m long_context_prefill_tcgen05_b200.ncu_summary launches.csv
+    python benchmarks/ncu_summary.py launches.csv
 """
 import collections
 import csv
@@ -13,14 +13,14 @@ SHORT = [
     ("gemv_kernel<0", "gemv_qkv_rope_append"), ("gemv_kernel<1", "gemv_resid (o_proj / down)"),
     ("gemv_kernel<2", "gemv_gate_up_swiglu"), ("kv_store_kernel", "kv_store"),
     ("attn_kernel", "attention"),
-    ("gemm_kernel<256, 4>", "gemm_qkv_rope"), ("gemm_kernel<128, 4>", "gemm_qkv_rope"),
-    ("gemm_kernel<256, 2>", "gemm_o_resid_delta"), ("gemm_kernel<128, 2>", "gemm_o_resid_delta"),
-    ("gemm_kernel<256, 3>", "gemm_gate_up_swiglu"), ("gemm_kernel<128, 3>", "gemm_gate_up_swiglu"),
-    ("gemm_kernel<256, 1>", "gemm_resid (o_proj / down)"), ("gemm_kernel<128, 1>", "gemm_resid (o_proj / down)"),
-    ("gemm_kernel<256, 0>", "gemm_store"), ("gemm_kernel<128, 0>", "gemm_store"),
-    ("gemm_pair_kernel<4>", "gemm_qkv_rope"), ("gemm_pair_kernel<2>", "gemm_o_resid_delta"),
-    ("gemm_pair_kernel<3>", "gemm_gate_up_swiglu"), ("gemm_pair_kernel<1>", "gemm_resid (o_proj / down)"),
-    ("gemm_pair_kernel<0>", "gemm_store"),
+    ("gemm_kernel<256, 4,", "gemm_qkv_rope"), ("gemm_kernel<128, 4,", "gemm_qkv_rope"),
+    ("gemm_kernel<256, 2,", "gemm_o_resid_delta"), ("gemm_kernel<128, 2,", "gemm_o_resid_delta"),
+    ("gemm_kernel<256, 3,", "gemm_gate_up_swiglu"), ("gemm_kernel<128, 3,", "gemm_gate_up_swiglu"),
+    ("gemm_kernel<256, 1,", "gemm_resid (o_proj / down)"), ("gemm_kernel<128, 1,", "gemm_resid (o_proj / down)"),
+    ("gemm_kernel<256, 0,", "gemm_store"), ("gemm_kernel<128, 0,", "gemm_store"),
+    ("gemm_pair_kernel<4,", "gemm_qkv_rope"), ("gemm_pair_kernel<2,", "gemm_o_resid_delta"),
+    ("gemm_pair_kernel<3,", "gemm_gate_up_swiglu"), ("gemm_pair_kernel<1,", "gemm_resid (o_proj / down)"),
+    ("gemm_pair_kernel<0,", "gemm_store"),
     ("rmsnorm_kernel", "rmsnorm"), ("score_from_ssq", "score"), ("score_kernel", "score"),
     ("select_kernel", "select"), ("move_rows_kernel<false>", "gather"), ("move_rows_kernel<true>", "scatter"),
     ("move_rows_kernel<0>", "gather"), ("move_rows_kernel<1>", "scatter"),

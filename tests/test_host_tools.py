@@ -3,7 +3,11 @@ summary and the nvidia-smi clock sampler that decides whether a bench run is
 kept (throttle reasons, median SM clock under load)."""
 import csv
 
-from long_context_prefill_tcgen05_b200 import ncu_summary
+import os
+import sys
+
+sys.path.insert(0, os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "benchmarks"))
+import ncu_summary  # noqa: E402
 
 
 def _launch_csv(path, launches):
@@ -19,12 +23,12 @@ def test_ncu_summary_takes_the_last_step_and_groups_kernels(tmp_path):
     p = tmp_path / "launches.csv"
     _launch_csv(p, [
         ("dash::rows::rope_table_kernel(float2 *, long, int, double)", "us", "9"),  # an earlier step
-        ("dash::attn::attn_kernel<128>(...)", "ms", "50"),
+        ("dash::attn::attn_kernel<128, 0>(...)", "ms", "50"),
         ("dash::rows::rope_table_kernel(float2 *, long, int, double)", "us", "10"),  # last step starts
-        ("void dash::gemm::gemm_pair_kernel<3>(...)", "ms", "3"),
-        ("void dash::attn::attn_kernel<128>(...)", "us", "2,000"),
-        ("void dash::attn::attn_kernel<128>(...)", "ns", "1000000"),
-        ("void dash::rows::rmsnorm_kernel(...)", "us", "500"),
+        ("void dash::gemm::gemm_pair_kernel<3, 0>(...)", "ms", "3"),
+        ("void dash::attn::attn_kernel<128, 0>(...)", "us", "2,000"),
+        ("void dash::attn::attn_kernel<128, 1>(...)", "ns", "1000000"),
+        ("void dash::rows::rmsnorm_kernel<0>(...)", "us", "500"),
     ])
     lines = ncu_summary.summarise(str(p)).splitlines()
     rows = {ln[:34].strip(): ln[34:].split() for ln in lines[1:]}
