@@ -531,15 +531,26 @@ def score_select_leg(dash, dev, peaks, reps=20):
                 ts.append(e0.elapsed_time(e1))
         return statistics.median(ts)
 
+    sel_ws = torch.empty(L.dash_select_workspace_size(T), dtype=torch.uint8, device=dev)
+
     def select_call(kind, keep, thr):
         return lambda: L.dash_select(dash._p(delta), T, dash.SELECTS[kind], keep, thr, 0, 0, dash._p(idx), None,
-                                     dash._p(count), None, 0, None)
+                                     dash._p(count), dash._p(sel_ws), sel_ws.numel(), None)
+    T2 = 131072  # the long-context length: selection over a 4x longer score vector
+    g = torch.Generator(device=dev).manual_seed(1)
+    delta2 = torch.rand(T2, generator=g, device=dev)
+    idx2 = torch.empty(T2, dtype=torch.int32, device=dev)
+    sel_ws2 = torch.empty(L.dash_select_workspace_size(T2), dtype=torch.uint8, device=dev)
+    K2 = math.floor(0.5 * T2)
     cases = {
         "score_abs": (lambda: dash.score(U, out=delta), T * d * 2 + 4 * T),
         "score_rel": (lambda: dash.score(U, H, relative=True, out=delta_r), 2 * T * d * 2 + 4 * T),
         "select_topk_keep0.5": (select_call("topk", 0.5, 0.0), 4 * T + 4 * K + 4),
         "select_threshold_median": (select_call("threshold", 0.0, med), 4 * T + 4 * (T // 2) + 4),
         "gather_K16384": (lambda: dash.compact(U, sel), 2 * K * d * 2 + 4 * K),
+        "select_topk_keep0.5_T131072": (
+            lambda: L.dash_select(dash._p(delta2), T2, dash.SELECTS["topk"], 0.5, 0.0, 0, 0, dash._p(idx2), None,
+                                  dash._p(count), dash._p(sel_ws2), sel_ws2.numel(), None), 4 * T2 + 4 * K2 + 4),
     }
     out = {}
     for name, (fn, nbytes) in cases.items():
@@ -548,7 +559,8 @@ def score_select_leg(dash, dev, peaks, reps=20):
         out[name] = {"us": ms * 1e3, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
     dash.check_device()
     out["workload"] = ("U, H bf16 [32768, 3584] N(0,1), 3264 rows of U x4 in 51 spans of 64 (seed 1); "
-                       "top-k keep 0.5 (K = 16384) and threshold = median delta")
+                       "top-k keep 0.5 (K = 16384) and threshold = median delta; top-k keep 0.5 also over "
+                       "131072 uniform scores")
     out["timing"] = f"each launch alone after a 256 MB L2-flushing write, median of {reps}"
     del U, H, flush
     torch.cuda.empty_cache()

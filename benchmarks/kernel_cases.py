@@ -119,6 +119,7 @@ def main():
         sel_idx = torch.empty(T, dtype=torch.int32, device=dev)
         count = torch.empty(1, dtype=torch.int32, device=dev)
         L = dash.lib()
+        sel_ws = torch.empty(L.dash_select_workspace_size(T), dtype=torch.uint8, device=dev)
         gain = (1 + 0.1 * torch.randn(d, generator=g, device=dev)).bfloat16()
         Yn = torch.empty_like(H)
         ms = {
@@ -129,7 +130,8 @@ def main():
             "gather": cold(lambda: dash.compact(U, idx)),
             "scatter": cold(lambda: dash.scatter(Y, idx, H)),
             "select": cold(lambda: L.dash_select(dash._p(s), T, dash.SELECTS["topk"], 0.5, 0.0, 0, 0,
-                                                 dash._p(sel_idx), None, dash._p(count), None, 0, None)),
+                                                 dash._p(sel_idx), None, dash._p(count), dash._p(sel_ws),
+                                                 sel_ws.numel(), None)),
         }
         nbytes = {"rmsnorm": 2 * T * d * 2, "score": T * d * 2, "score_relative": 2 * T * d * 2, "gather": 2 * K * d * 2,
                   "scatter": 2 * K * d * 2, "select": T * 4 + K * 4}

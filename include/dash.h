@@ -156,8 +156,9 @@ dash_status dash_score(const dash_bf16* U, const dash_bf16* H, int64_t T, int32_
  * keep_first and the last keep_last tokens.  Host-only arithmetic in double. */
 int64_t dash_topk_count(int64_t T, double keep_ratio, int32_t keep_first, int32_t keep_last);
 
-/* Workspace bytes dash_select needs for T scores (currently 0: all scratch
- * lives in shared memory). */
+/* Workspace bytes dash_select needs for T scores: the key histogram, the
+ * candidates of the bucket holding the cut (up to T of them, so ties never
+ * truncate) and per-chunk counts. */
 size_t dash_select_workspace_size(int64_t T);
 
 /* Active-set selection ([DASH blog] §3.1 and the final sort of §3.3;
@@ -173,7 +174,12 @@ size_t dash_select_workspace_size(int64_t T);
  *   count:   [1] int32 device out: number of active tokens, or -3
  *            (= -DASH_ERR_NONFINITE) if any score is NaN/Inf (then idx is
  *            not written and the NONFINITE device error is set).
- * Identical fp32 inputs give bit-identical outputs. */
+ *   ws:      dash_select_workspace_size(T) bytes (DASH_ERR_NO_MEMORY if
+ *            smaller); may be NULL when T == 0.
+ * All SMs take part: one pass over the scores builds a histogram of the
+ * keys' top 11 bits, the bucket holding the cut is resolved exactly, and
+ * every SM compacts its own chunk of tokens at offsets known from per-chunk
+ * counts.  Identical fp32 inputs give bit-identical outputs. */
 dash_status dash_select(const float* scores, int64_t T, int32_t kind, double keep_ratio,
                         float threshold, int32_t keep_first, int32_t keep_last,
                         int32_t* idx, int32_t* halted, int32_t* count,

@@ -2,6 +2,7 @@
 // argument checks, workspace carving, tensor-map encoding, kernel launches,
 // and the host-side layer loop of the single-shot DASH prefill.
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -521,8 +522,28 @@ bool weights_ok(const dash_layer_weights* w) {
          aligned16(w->w_gate) && aligned16(w->w_up) && aligned16(w->w_down);
 }
 
+// Scratch of the multi-SM selection of one sequence (none for varlen
+// batches, whose sequences each take one CTA).
+struct SelWs {
+  dash::rows::SelState* st = nullptr;
+  uint32_t* cand_key = nullptr;
+  int32_t* cand_idx = nullptr;
+  uint32_t* chunk = nullptr;  // 6 arrays of n_chunks entries
+  int64_t n_chunks = 0;
+};
+
+void carve_select(int64_t T, Carver& c, SelWs& w) {
+  namespace r = dash::rows;
+  w.n_chunks = (T + r::kSelCtaTok - 1) / r::kSelCtaTok;
+  w.st = c.take<r::SelState>(1);
+  w.cand_key = c.take<uint32_t>(static_cast<size_t>(T > 0 ? T : 1));
+  w.cand_idx = c.take<int32_t>(static_cast<size_t>(T > 0 ? T : 1));
+  w.chunk = c.take<uint32_t>(static_cast<size_t>(6 * (w.n_chunks > 0 ? w.n_chunks : 1)));
+}
+
 struct PrefillWs {
   LayerWs L;
+  SelWs sel_ws;     // single-sequence selection scratch
   s16* Hc;         // [T, d] compacted active rows
   float* delta;     // [T]
   int32_t* idx;     // [T]
@@ -553,17 +574,61 @@ void carve_prefill(const dash_dims& D, int64_t T, int nseq, Carver& c, PrefillWs
   w.pos = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
   w.kst = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
   w.hpos = varlen ? c.take<int32_t>(static_cast<size_t>(T)) : nullptr;
+  if (!varlen) carve_select(T, c, w.sel_ws);
 }
 
+// Selection ([DASH blog] §3.1; threshold form from [DASH news]).  One
+// sequence (seg == NULL): the multi-SM kernels over sel's scratch; nseg
+// sequences of a varlen batch (seg = their starts on the device): one CTA each.
 dash_status select_impl(const float* scores, int64_t T, const int32_t* seg, int nseg, int kind, double keep,
                         float thr, int keep_first, int keep_last, int32_t* idx, int32_t* halted, int32_t* count,
-                        cudaStream_t st) {
+                        const SelWs* sel, const DeviceInfo& di, cudaStream_t st) {
+  (void)di;
+  namespace r = dash::rows;
   if (T == 0 || nseg == 0)
     return cudaMemsetAsync(count, 0, sizeof(int32_t) * (nseg > 0 ? nseg : 1), st) == cudaSuccess ? DASH_OK
                                                                                             : DASH_ERR_CUDA;
   TimedLaunch tl(DASH_K_SELECT, T, nseg, 0, st);
-  dash::rows::select_kernel<<<nseg, dash::rows::kSelThreads, 0, st>>>(scores, T, seg, kind, keep, thr, keep_first,
-                                                                       keep_last, idx, halted, count);
+  if (seg) {
+    r::select_kernel<<<nseg, r::kSelThreads, 0, st>>>(scores, T, seg, kind, keep, thr, keep_first, keep_last, idx,
+                                                      halted, count);
+    return launch_status();
+  }
+  if (!sel || !sel->st) return DASH_ERR_NO_MEMORY;
+  // the same middle range, k and mode as select_kernel computes on the device
+  const int64_t lo = keep_first < T ? keep_first : T;
+  int64_t hi = keep_last > 0 ? T - keep_last : T;
+  if (hi < lo) hi = lo;
+  const int64_t k_dyn = kind == DASH_SELECT_TOPK ? static_cast<int64_t>(std::floor(keep * static_cast<double>(hi - lo)))
+                                                  : 0;
+  r::SelArgs a;
+  a.scores = scores;
+  a.T = T;
+  a.lo = lo;
+  a.hi = hi;
+  a.k_dyn = k_dyn;
+  a.mode = kind == DASH_SELECT_THRESHOLD ? 3 : (k_dyn <= 0 ? 0 : (k_dyn >= hi - lo ? 1 : 2));
+  a.thr = thr;
+  a.n_chunks = sel->n_chunks;
+  a.st = sel->st;
+  a.cand_key = sel->cand_key;
+  a.cand_idx = sel->cand_idx;
+  const int64_t G = sel->n_chunks;
+  a.n_flag = sel->chunk;
+  a.gt_extra = sel->chunk + G;
+  a.eq_cnt = sel->chunk + 2 * G;
+  a.sel_off = sel->chunk + 3 * G;
+  a.hal_off = sel->chunk + 4 * G;
+  a.eq_before = sel->chunk + 5 * G;
+  a.idx = idx;
+  a.halted = halted;
+  a.count = count;
+  if (cudaMemsetAsync(sel->st, 0, offsetof(r::SelState, kth), st) != cudaSuccess) return DASH_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(G);
+  if (a.mode == 2) r::sel_hist_kernel<<<grid, r::kSelCtaThreads, 0, st>>>(a);
+  r::sel_scan_kernel<<<grid, r::kSelCtaThreads, 0, st>>>(a);
+  r::sel_resolve_kernel<<<1, r::kResolveThreads, 0, st>>>(a);
+  r::sel_compact_kernel<<<grid, r::kSelCtaThreads, 0, st>>>(a);
   return launch_status();
 }
 
@@ -771,7 +836,7 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
   std::vector<int32_t> counts(static_cast<size_t>(nseq));
   if ((s = select_impl(delta, T, varlen ? P.cu : nullptr, nseq, cfg->select, cfg->keep_ratio, cfg->threshold,
                        cfg->keep_first, cfg->keep_last, varlen ? P.sel : idx, varlen ? P.selh : P.halted, P.count,
-                       st)) != DASH_OK)
+                       varlen ? nullptr : &P.sel_ws, *di, st)) != DASH_OK)
     return s;
   if (cudaMemcpyAsync(counts.data(), P.count, sizeof(int32_t) * nseq, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
@@ -1185,20 +1250,31 @@ int64_t dash_topk_count(int64_t T, double keep_ratio, int32_t keep_first, int32_
   return (T - (hi - lo)) + static_cast<int64_t>(std::floor(keep_ratio * static_cast<double>(hi - lo)));
 }
 
-size_t dash_select_workspace_size(int64_t) { return 0; }
+size_t dash_select_workspace_size(int64_t T) {
+  if (T < 0) return 0;
+  Carver c{nullptr};
+  SelWs w;
+  carve_select(T, c, w);
+  return c.off + 256;
+}
 
 dash_status dash_select(const float* scores, int64_t T, int32_t kind, double keep_ratio, float threshold,
                         int32_t keep_first, int32_t keep_last, int32_t* idx, int32_t* halted, int32_t* count,
                         void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (T < 0 || T > INT32_MAX) return DASH_ERR_SHAPE;
   if (!count || (T > 0 && (!scores || !idx))) return DASH_ERR_INVALID_ARG;
   if (kind != DASH_SELECT_TOPK && kind != DASH_SELECT_THRESHOLD) return DASH_ERR_INVALID_ARG;
   if (keep_first < 0 || keep_last < 0) return DASH_ERR_INVALID_ARG;
   if (kind == DASH_SELECT_TOPK && !(keep_ratio >= 0.0 && keep_ratio <= 1.0)) return DASH_ERR_INVALID_ARG;
+  if (T > 0 && (!ws || ws_bytes < dash_select_workspace_size(T))) return DASH_ERR_NO_MEMORY;
+  DeviceInfo* di;
+  dash_status s = device_info(&di);
+  if (s != DASH_OK) return s;
+  Carver c{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255))};
+  SelWs w;
+  carve_select(T, c, w);
   return select_impl(scores, T, nullptr, 1, kind, keep_ratio, threshold, keep_first, keep_last, idx, halted, count,
-                     as_stream(stream));
+                     &w, *di, as_stream(stream));
 }
 
 dash_status dash_compact(const dash_bf16* X, int64_t T, const int32_t* idx, int64_t K, int32_t d, dash_bf16* Y,

@@ -361,6 +361,380 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (tid == 0) count[0] = static_cast<int32_t>(sel_base);
 }
 
+// ------------------------------------------------------ multi-SM select
+// Selection for one sequence spread over all SMs ([DASH blog] §3.1 step 3
+// and the final ascending sort of §3.3; threshold form from [DASH news]).
+// Same result, bit for bit, as select_kernel on one segment:
+//   1. sel_hist_kernel     one pass over the scores: a histogram of the 11
+//                          most significant bits of every middle token's
+//                          monotone key, summed over the CTAs (top-k only)
+//   2. sel_scan_kernel     every CTA finds the bucket holding the cut from
+//                          that histogram, counts the tokens of its chunk
+//                          whose fate is certain (bucket above the cut, or
+//                          the threshold test), and appends the cut bucket's
+//                          tokens to a candidate list
+//   3. sel_resolve_kernel  one CTA resolves the exact cut key among the
+//                          candidates and how many keys equal to it are
+//                          taken (lowest indices first), then the output
+//                          offset of every chunk
+//   4. sel_compact_kernel  every CTA writes its chunk's kept and halted
+//                          indices in ascending order at those offsets
+// A chunk is kSelCtaTok consecutive tokens; its CTA owns them in every pass.
+constexpr int kSelCtaThreads = 256;
+constexpr int kSelCtaTok = kSelCtaThreads * kSelPerThread;  // tokens per chunk
+constexpr int kSelBits = 11;
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelShift = 32 - kSelBits;
+constexpr int kResolveThreads = 1024;
+
+// Scratch in the caller's workspace; the header (hist, n_cand, bad) must be
+// zero when sel_hist_kernel starts.
+struct SelState {
+  uint32_t hist[kSelBins];  // middle tokens per key bucket
+  uint32_t n_cand;          // candidates appended
+  int32_t bad;              // a non-finite score was seen
+  uint32_t kth;             // the cut key (top-k)
+  uint32_t k_rem;           // keys equal to kth that are kept, lowest indices first
+};
+struct SelArgs {
+  const float* scores;
+  int64_t T, lo, hi;   // the middle [lo, hi) is ranked; the rest is forced
+  int64_t k_dyn;       // middle tokens to keep (top-k)
+  int mode;            // 0 none of the middle, 1 all of it, 2 top-k cut, 3 threshold
+  float thr;
+  int64_t n_chunks;
+  SelState* st;
+  uint32_t* cand_key;  // [T]
+  int32_t* cand_idx;   // [T]
+  uint32_t* n_flag;    // [n_chunks] middle tokens kept for certain
+  uint32_t* gt_extra;  // [n_chunks] candidates above the cut key
+  uint32_t* eq_cnt;    // [n_chunks] candidates equal to the cut key
+  uint32_t* sel_off;   // [n_chunks] first output slot of the chunk's kept tokens
+  uint32_t* hal_off;   // [n_chunks] ... and of its halted tokens
+  uint32_t* eq_before; // [n_chunks] keys equal to the cut in earlier chunks
+  int32_t* idx;        // [T] kept indices, ascending
+  int32_t* halted;     // [T] or NULL: the others, ascending
+  int32_t* count;      // [1] kept count, or -3 after a non-finite score
+};
+
+// Exclusive prefix sum over a block of NT threads (one value each) and the total.
+template <int NT>
+__device__ __forceinline__ uint32_t block_scan_excl(uint32_t v, uint32_t* sh, uint32_t& total) {
+  constexpr int kWarps = NT / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t wv = lane < kWarps ? sh[lane] : 0u;
+    uint32_t wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    sh[32 + lane] = wi - wv;
+    if (lane == 31) sh[64] = wi;
+  }
+  __syncthreads();
+  const uint32_t res = sh[32 + warp] + incl - v;
+  total = sh[64];
+  __syncthreads();
+  return res;
+}
+
+// The bucket holding the k-th largest middle key and the count above it,
+// from the global histogram (every caller gets the same answer).
+template <int NT>
+__device__ __forceinline__ void find_cut_bucket(const SelState* st, int64_t k, uint32_t* sh, int& bucket,
+                                                uint32_t& above) {
+  constexpr int kPerT = kSelBins / NT;
+  __shared__ int s_bucket;
+  __shared__ uint32_t s_above;
+  if (threadIdx.x == 0) {  // no bucket when fewer than k keys are finite (then the caller sees `bad`)
+    s_bucket = -1;
+    s_above = 0;
+  }
+  // thread i owns buckets [kSelBins - (i + 1) * kPerT, kSelBins - i * kPerT): thread 0 the highest
+  uint32_t c[kPerT], own = 0;
+#pragma unroll
+  for (int j = 0; j < kPerT; ++j) {
+    c[j] = st->hist[kSelBins - 1 - (threadIdx.x * kPerT + j)];
+    own += c[j];
+  }
+  uint32_t tot;
+  const uint32_t before = block_scan_excl<NT>(own, sh, tot);  // keys in higher buckets
+  if (before < static_cast<uint64_t>(k) && static_cast<uint64_t>(k) <= static_cast<uint64_t>(before) + own) {
+    uint32_t acc = before;
+    int j = 0;
+    for (; j < kPerT - 1; ++j) {
+      if (acc + c[j] >= k) break;
+      acc += c[j];
+    }
+    s_bucket = kSelBins - 1 - (threadIdx.x * kPerT + j);
+    s_above = acc;
+  }
+  __syncthreads();
+  bucket = s_bucket;
+  above = s_above;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) sel_hist_kernel(const SelArgs a) {
+  __shared__ uint32_t h[kSelBins];
+  for (int i = threadIdx.x; i < kSelBins; i += kSelCtaThreads) h[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kSelCtaTok + threadIdx.x * kSelPerThread;
+#pragma unroll
+  for (int i = 0; i < kSelPerThread; ++i) {
+    const int64_t t = t0 + i;
+    bool in = t >= a.lo && t < a.hi;
+    uint32_t bin = 0;
+    if (in) {
+      const float f = a.scores[t];
+      in = isfinite(f);
+      bin = score_key(f) >> kSelShift;
+    }
+    const uint32_t active = __ballot_sync(0xffffffffu, in);
+    if (in) {  // one shared atomic per distinct bucket of the warp
+      const uint32_t peers = __match_any_sync(active, bin);
+      if (lane == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kSelBins; i += kSelCtaThreads)
+    if (h[i]) atomicAdd(&a.st->hist[i], h[i]);
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) sel_scan_kernel(const SelArgs a) {
+  __shared__ uint32_t sh[65];
+  const int lane = threadIdx.x & 31;
+  const int64_t c = blockIdx.x;
+  int bucket = -1;
+  uint32_t above = 0;
+  if (a.mode == 2) find_cut_bucket<kSelCtaThreads>(a.st, a.k_dyn, sh, bucket, above);
+  const int64_t t0 = c * kSelCtaTok + threadIdx.x * kSelPerThread;
+  uint32_t n = 0;
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < kSelPerThread; ++i) {
+    const int64_t t = t0 + i;
+    bool cand = false;
+    uint32_t key = 0;
+    if (t < a.T) {
+      const float f = a.scores[t];
+      bad |= !isfinite(f);
+      if (t >= a.lo && t < a.hi) {
+        if (a.mode == 1) n += 1;
+        else if (a.mode == 3) n += f >= a.thr;
+        else if (a.mode == 2 && isfinite(f)) {
+          key = score_key(f);
+          const int b = static_cast<int>(key >> kSelShift);
+          n += b > bucket;
+          cand = b == bucket;
+        }
+      }
+    }
+    // warp-aggregated append of the cut bucket's tokens
+    const uint32_t m = __ballot_sync(0xffffffffu, cand);
+    if (m) {
+      uint32_t base = 0;
+      if (lane == __ffs(m) - 1) base = atomicAdd(&a.st->n_cand, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+      if (cand) {
+        const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
+        a.cand_key[slot] = key;
+        a.cand_idx[slot] = static_cast<int32_t>(t);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&a.st->bad, 1);
+  uint32_t tot;
+  block_scan_excl<kSelCtaThreads>(n, sh, tot);
+  if (threadIdx.x == 0) {
+    a.n_flag[c] = tot;
+    a.gt_extra[c] = 0;
+    a.eq_cnt[c] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(kResolveThreads, 1) sel_resolve_kernel(const SelArgs a) {
+  __shared__ uint32_t sh[65];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix, s_k;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (a.st->bad) {
+    if (tid == 0) {
+      a.count[0] = -3;
+      flag_error(kDevErrNonfinite);
+    }
+    return;
+  }
+  uint32_t kth = 0, k_rem = 0;
+  if (a.mode == 2) {
+    int bucket;
+    uint32_t above;
+    find_cut_bucket<kResolveThreads>(a.st, a.k_dyn, sh, bucket, above);
+    const uint32_t C = a.st->n_cand;
+    // radix select of the (k_dyn - above)-th largest candidate key over the
+    // bits below the bucket's, 8 at a time
+    uint32_t prefix = static_cast<uint32_t>(bucket) << kSelShift, mask = ~0u << kSelShift;
+    uint32_t k = static_cast<uint32_t>(a.k_dyn - above);
+    for (int shift = 16; shift >= 0; shift -= 8) {
+      for (int b = tid; b < 256; b += kResolveThreads) hist[b] = 0;
+      __syncthreads();
+      for (uint32_t base = 0; base < C; base += kResolveThreads) {
+        const uint32_t j = base + tid;
+        const uint32_t key = j < C ? a.cand_key[j] : 0u;
+        const bool match = j < C && (key & mask) == prefix;
+        const uint32_t bin = (key >> shift) & 255u;
+        const uint32_t active = __ballot_sync(0xffffffffu, match);
+        if (match) {
+          const uint32_t peers = __match_any_sync(active, bin);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (tid < 32) {  // lane l owns bins [8l, 8l + 8)
+        uint32_t cnt[8], own = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          cnt[i] = hist[8 * lane + i];
+          own += cnt[i];
+        }
+        uint32_t incl = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += n;
+        }
+        const uint32_t abv = incl - own;
+        if (abv < k && k <= incl) {
+          uint32_t acc = abv;
+          int b = 7;
+          for (; b > 0; --b) {
+            if (acc + cnt[b] >= k) break;
+            acc += cnt[b];
+          }
+          s_prefix = prefix | (static_cast<uint32_t>(8 * lane + b) << shift);
+          s_k = k - acc;
+        }
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      k = s_k;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    kth = prefix;
+    k_rem = k;
+    // per chunk: candidates above the cut key, and equal to it
+    for (uint32_t j = tid; j < C; j += kResolveThreads) {
+      const uint32_t key = a.cand_key[j];
+      const int64_t ch = a.cand_idx[j] / kSelCtaTok;
+      if (key > kth) atomicAdd(&a.gt_extra[ch], 1u);
+      else if (key == kth) atomicAdd(&a.eq_cnt[ch], 1u);
+    }
+    __syncthreads();
+  }
+  // output offsets of every chunk, in chunk order
+  uint32_t sel_carry = 0, hal_carry = 0, eq_carry = 0;
+  for (int64_t c0 = 0; c0 < a.n_chunks; c0 += kResolveThreads) {
+    const int64_t c = c0 + tid;
+    uint32_t n_sel = 0, n_hal = 0, n_eq = 0;
+    if (c < a.n_chunks) {
+      const int64_t b = c * kSelCtaTok, e = min(b + kSelCtaTok, a.T);
+      const int64_t mid = max(int64_t(0), min(e, a.hi) - max(b, a.lo));
+      n_sel = static_cast<uint32_t>((e - b) - mid) + a.n_flag[c];
+      if (a.mode == 2) {
+        n_eq = a.eq_cnt[c];
+        n_sel += a.gt_extra[c];
+      }
+      n_hal = static_cast<uint32_t>(e - b);  // minus the kept ones, below
+    }
+    uint32_t tot_eq;
+    const uint32_t eq_b = eq_carry + block_scan_excl<kResolveThreads>(n_eq, sh, tot_eq);
+    if (a.mode == 2 && c < a.n_chunks) {
+      const uint32_t taken = eq_b >= k_rem ? 0u : min(n_eq, k_rem - eq_b);
+      n_sel += taken;
+    }
+    n_hal -= n_sel;
+    uint32_t tot_sel, tot_hal;
+    const uint32_t so = sel_carry + block_scan_excl<kResolveThreads>(n_sel, sh, tot_sel);
+    const uint32_t ho = hal_carry + block_scan_excl<kResolveThreads>(n_hal, sh, tot_hal);
+    if (c < a.n_chunks) {
+      a.sel_off[c] = so;
+      a.hal_off[c] = ho;
+      a.eq_before[c] = eq_b;
+    }
+    sel_carry += tot_sel;
+    hal_carry += tot_hal;
+    eq_carry += tot_eq;
+  }
+  if (tid == 0) {
+    a.st->kth = kth;
+    a.st->k_rem = k_rem;
+    a.count[0] = static_cast<int32_t>(sel_carry);
+  }
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) sel_compact_kernel(const SelArgs a) {
+  __shared__ uint32_t sh[65];
+  if (a.st->bad) return;  // uniform
+  const int64_t c = blockIdx.x;
+  const uint32_t kth = a.st->kth, k_rem = a.st->k_rem;
+  const int64_t t0 = c * kSelCtaTok + threadIdx.x * kSelPerThread;
+  bool gt[kSelPerThread], eq[kSelPerThread], valid[kSelPerThread], forced[kSelPerThread];
+  uint32_t n_eq = 0;
+#pragma unroll
+  for (int i = 0; i < kSelPerThread; ++i) {
+    const int64_t t = t0 + i;
+    valid[i] = t < a.T;
+    forced[i] = valid[i] && (t < a.lo || t >= a.hi);
+    gt[i] = eq[i] = false;
+    if (valid[i] && !forced[i]) {
+      const float f = a.scores[t];
+      if (a.mode == 1) gt[i] = true;
+      else if (a.mode == 3) gt[i] = f >= a.thr;
+      else if (a.mode == 2) {
+        const uint32_t key = score_key(f);
+        gt[i] = key > kth;
+        eq[i] = key == kth;
+      }
+    }
+    n_eq += eq[i];
+  }
+  uint32_t tot;
+  uint32_t eq_rank = a.eq_before[c] + block_scan_excl<kSelCtaThreads>(n_eq, sh, tot);
+  bool sel[kSelPerThread];
+  uint32_t n_sel = 0, n_hal = 0;
+#pragma unroll
+  for (int i = 0; i < kSelPerThread; ++i) {
+    bool take_eq = false;
+    if (eq[i]) {
+      take_eq = eq_rank < k_rem;
+      ++eq_rank;
+    }
+    sel[i] = valid[i] && (forced[i] || gt[i] || take_eq);
+    n_sel += sel[i];
+    n_hal += valid[i] && !sel[i];
+  }
+  const uint32_t pk = block_scan_excl<kSelCtaThreads>((n_sel << 16) | n_hal, sh, tot);
+  uint32_t ps = a.sel_off[c] + (pk >> 16), ph = a.hal_off[c] + (pk & 0xffffu);
+#pragma unroll
+  for (int i = 0; i < kSelPerThread; ++i) {
+    if (!valid[i]) continue;
+    if (sel[i]) a.idx[ps++] = static_cast<int32_t>(t0 + i);
+    else if (a.halted) a.halted[ph++] = static_cast<int32_t>(t0 + i);
+  }
+}
+
 // ---------------------------------------------------------- varlen layout
 // For each row i (original token orig = rows ? rows[i] : i) of a varlen batch
 // with sequence starts cu[0..nseq]: pos[i] = orig - cu[s] (the RoPE position

@@ -238,8 +238,9 @@ def select(scores, kind="topk", keep=0.5, threshold=0.0, keep_first=0, keep_last
     idx = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
     halted = torch.empty(max(T, 1), dtype=torch.int32, device=dev) if want_halted else None
     count = torch.empty(1, dtype=torch.int32, device=dev)
+    ws = workspace(lib().dash_select_workspace_size(T), dev)
     _check(lib().dash_select(_t(scores, F32, "scores"), T, SELECTS[kind], keep, threshold, keep_first, keep_last, _p(idx),
-                             _p(halted), _p(count), None, 0, _stream(stream)), "dash_select")
+                             _p(halted), _p(count), _p(ws), ws.numel(), _stream(stream)), "dash_select")
     n = int(count.item())
     if n < 0:
         raise DashError(-n, "dash_select")

@@ -148,4 +148,6 @@ def adversarial_scores(kind: str, T: int, seed: int = 0):
         x = torch.full((T,), 1e-3)
         x[torch.randint(0, T, (max(1, T // 100),), generator=gen)] = 10.0
         return x
+    if kind == "narrow":          # distinct values sharing their top key bits (one bucket holds them all)
+        return 1.0 + torch.rand(T, generator=gen) * 1e-3
     raise ValueError(kind)

@@ -89,6 +89,10 @@ def test_argument_errors_are_caught_on_the_host(L):
     assert L.dash_select(FAKE, 10, 0, -0.1, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 1
     assert L.dash_select(FAKE, 10, 0, 0.5, 0.0, -1, 0, FAKE, None, cnt, None, 0, None) == 1
     assert L.dash_select(None, 10, 0, 0.5, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 1
+    need = L.dash_select_workspace_size(100000)
+    assert need > 8 * 100000 and L.dash_select_workspace_size(-1) == 0
+    assert L.dash_select(FAKE, 100000, 0, 0.5, 0.0, 0, 0, FAKE, None, cnt, None, 0, None) == 4    # no workspace
+    assert L.dash_select(FAKE, 100000, 0, 0.5, 0.0, 0, 0, FAKE, None, cnt, FAKE, need - 1, None) == 4
     assert L.dash_score(FAKE, None, 10, 7, 0, FAKE, None) == 2
     assert L.dash_score(FAKE, None, 10, 64, 1, FAKE, None) == 1          # relative needs H
     assert L.dash_compact(FAKE, 10, FAKE, 5, 12, FAKE, None) == 2

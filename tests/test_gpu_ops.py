@@ -31,7 +31,7 @@ def test_score_matches_oracle(gpu_lib, T, d, relative):
 
 
 # ----------------------------------------------------------------- select
-KINDS = ["random", "all_equal", "few_values", "signed_zero", "denormal", "negative", "spiky"]
+KINDS = ["random", "all_equal", "few_values", "signed_zero", "denormal", "negative", "spiky", "narrow"]
 
 
 def _check_select(s, kind, keep=0.5, thr=0.0, nf=0, nl=0):
@@ -47,7 +47,7 @@ def _check_select(s, kind, keep=0.5, thr=0.0, nf=0, nl=0):
 
 
 @pytest.mark.parametrize("pattern", KINDS)
-@pytest.mark.parametrize("T", [1, 33, 1000, 4097, 32768, 100003])
+@pytest.mark.parametrize("T", [1, 33, 1000, 1025, 4097, 32768, 100003, 131072])
 def test_select_topk_bit_exact(gpu_lib, pattern, T):
     s = inputs.adversarial_scores(pattern, T, seed=T)
     for keep in (0.0, 1.0 / T, 0.5, 0.9, (T - 1) / T, 1.0):
@@ -58,7 +58,7 @@ def test_select_topk_bit_exact(gpu_lib, pattern, T):
 
 
 @pytest.mark.parametrize("pattern", KINDS)
-@pytest.mark.parametrize("T", [1, 1000, 32768])
+@pytest.mark.parametrize("T", [1, 1000, 32768, 131072])
 def test_select_threshold_bit_exact(gpu_lib, pattern, T):
     s = inputs.adversarial_scores(pattern, T, seed=T + 1)
     vals = s.numpy()
