@@ -421,6 +421,19 @@ def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
                          "share": p["ms"] / total_ms if total_ms else 0.0,
                          ("tflops" if p["unit"] == "flop" else "gbs"): rate / 1e12 if p["unit"] == "flop"
                          else rate / 1e9}
+    # GEMMs and attention split by the rows each launch processes (full-length
+    # layers vs the compacted ones after the halting layer)
+    by_rows = {}
+    for r in recs:
+        if r["kind"].startswith("gemm") or r["kind"] == "attention":
+            unit, amount = costs.launch_work(r, dims, pairs_by_rows)
+            q = by_rows.setdefault(f"{r['kind']}@{r['m']}", {"ms": 0.0, "work": 0, "launches": 0})
+            q["ms"] += r["ms"]
+            q["work"] += amount
+            q["launches"] += 1
+    for k, q in by_rows.items():
+        kernels.setdefault("by_rows", {})[k] = {"launches_per_step": q["launches"] // steps,
+                                                "tflops": q["work"] / (q["ms"] / 1e3) / 1e12 if q["ms"] else 0.0}
     dom_kind = max(per, key=lambda k: per[k]["ms"])
     dom = per[dom_kind]
     if dom["unit"] == "flop":

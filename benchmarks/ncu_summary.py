@@ -1,6 +1,8 @@
 """Summarises an ncu launch list (``--metrics gpu__time_duration.sum --csv``)
 of a bench.py run: per kernel, the launches, total time and share of the last
-prefill step (the launches from the last RoPE-table build to the end).
+complete prefill step -- the launches between the last two RoPE-table builds
+(every prefill starts with one), since a capture limit (-c) may cut the final
+step short; with a single build, the launches from it to the end.
 
     python benchmarks/ncu_summary.py launches.csv
 """
@@ -22,7 +24,8 @@ SHORT = [
     ("gemm_pair_kernel<3,", "gemm_gate_up_swiglu"), ("gemm_pair_kernel<1,", "gemm_resid (o_proj / down)"),
     ("gemm_pair_kernel<0,", "gemm_store"),
     ("rmsnorm_kernel", "rmsnorm"), ("score_from_ssq", "score"), ("score_kernel", "score"),
-    ("select_kernel", "select"), ("move_rows_kernel<false>", "gather"), ("move_rows_kernel<true>", "scatter"),
+    ("select_kernel", "select"), ("sel_hist_kernel", "select"), ("sel_scan_kernel", "select"),
+    ("sel_resolve_kernel", "select"), ("sel_compact_kernel", "select"), ("move_rows_kernel<false>", "gather"), ("move_rows_kernel<true>", "scatter"),
     ("move_rows_kernel<0>", "gather"), ("move_rows_kernel<1>", "scatter"),
     ("rope_table_kernel", "rope_table"),
 ]
@@ -52,7 +55,10 @@ def load(path):
 def summarise(path):
     launches = load(path)
     starts = [i for i, (n, _) in enumerate(launches) if "rope_table_kernel" in n]
-    step = launches[starts[-1]:] if starts else launches
+    if len(starts) >= 2:
+        step = launches[starts[-2]:starts[-1]]
+    else:
+        step = launches[starts[-1]:] if starts else launches
     agg = collections.OrderedDict()
     for name, ms in step:
         k = short(name)
@@ -63,7 +69,7 @@ def summarise(path):
     lines = [f"{'kernel':34s} {'launches':>8s} {'total ms':>10s} {'share':>7s}"]
     for k, (n, ms) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
         lines.append(f"{k:34s} {n:8d} {ms:10.3f} {ms / total:7.1%}")
-    lines.append(f"{'total (last step)':34s} {sum(v[0] for v in agg.values()):8d} {total:10.3f}")
+    lines.append(f"{'total (one step)':34s} {sum(v[0] for v in agg.values()):8d} {total:10.3f}")
     return "\n".join(lines)
 
 

@@ -19,7 +19,7 @@ def _launch_csv(path, launches):
             w.writerow([i, name, "gpu__time_duration.sum", unit, value])
 
 
-def test_ncu_summary_takes_the_last_step_and_groups_kernels(tmp_path):
+def test_ncu_summary_takes_the_last_complete_step_and_groups_kernels(tmp_path):
     p = tmp_path / "launches.csv"
     _launch_csv(p, [
         ("dash::rows::rope_table_kernel(float2 *, long, int, double)", "us", "9"),  # an earlier step
@@ -29,6 +29,8 @@ def test_ncu_summary_takes_the_last_step_and_groups_kernels(tmp_path):
         ("void dash::attn::attn_kernel<128, 0>(...)", "us", "2,000"),
         ("void dash::attn::attn_kernel<128, 1>(...)", "ns", "1000000"),
         ("void dash::rows::rmsnorm_kernel<0>(...)", "us", "500"),
+        ("dash::rows::rope_table_kernel(float2 *, long, int, double)", "us", "11"),  # a step cut short
+        ("void dash::attn::attn_kernel<128, 0>(...)", "ms", "7"),
     ])
     lines = ncu_summary.summarise(str(p)).splitlines()
     rows = {ln[:34].strip(): ln[34:].split() for ln in lines[1:]}
@@ -36,7 +38,7 @@ def test_ncu_summary_takes_the_last_step_and_groups_kernels(tmp_path):
     assert rows["gemm_gate_up_swiglu"] == ["1", "3.000", "46.1%"]
     assert rows["rmsnorm"][:2] == ["1", "0.500"]
     assert rows["rope_table"][:2] == ["1", "0.010"]
-    assert rows["total (last step)"] == ["5", "6.510"]
+    assert rows["total (one step)"] == ["5", "6.510"]
     # rows are ordered by time, largest first
     shares = [float(ln.split()[-1].rstrip("%")) for ln in lines[1:-1]]
     assert shares == sorted(shares, reverse=True)
