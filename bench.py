@@ -436,6 +436,7 @@ def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
                                                 "tflops": q["work"] / (q["ms"] / 1e3) / 1e12 if q["ms"] else 0.0}
     dom_kind = max(per, key=lambda k: per[k]["ms"])
     dom = per[dom_kind]
+    n_launch = sum(r.get("launches", 1) for r in recs)
     if dom["unit"] == "flop":
         achieved = dom["work"] / (dom["ms"] / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -446,7 +447,7 @@ def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     roof.update({"kernel": dom_kind, "traffic": recorded_traffic(dom_kind, recs),
                  "peak_source": f"{peaks['source']} ({'sustained bf16' if dom['unit'] == 'flop' else 'HBM copy'})"})
-    return kernels, roof, len(recs) // steps
+    return kernels, roof, n_launch // steps
 
 
 def long_context_leg(dash, stack, dims, dev, peaks, world, rounds=2):

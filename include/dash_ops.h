@@ -63,9 +63,10 @@ dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_k
                                   int32_t hkv, int32_t hd, dash_bf16* O, void* ws, size_t ws_bytes,
                                   void* stream);
 
-/* The FMA-pipe exponential the attention softmax uses for half of its
- * elements (no page counterpart; exported so tests can hold it to its error
- * bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
+/* An exponential on the FMA pipe, which the attention softmax can take for a
+ * fraction of its elements in place of MUFU (a compile-time option, off: it
+ * measured slower; no page counterpart; exported so tests can hold it to its
+ * error bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
  * (max relative error 7.5e-5) and an exponent-field add; inputs below -125
  * are clamped (result ~2e-38).  x, y: [n] fp32 device arrays. */
 dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream);
@@ -90,12 +91,14 @@ typedef enum dash_kernel_kind {
 } dash_kernel_kind;
 
 typedef struct dash_launch_record {
-  int32_t kind;   /* dash_kernel_kind */
-  int32_t layer;  /* decoder layer, -1 outside the layer loop */
-  int64_t m;      /* rows (GEMM M, attention query rows, selection T, decode sequences) */
-  int64_t n;      /* GEMM N, attention key rows (decode: cached keys summed over sequences) */
-  int64_t k;      /* GEMM K, attention causal (query, key) pairs (decode: CTAs) */
-  float ms;       /* device time between the two events */
+  int32_t kind;     /* dash_kernel_kind */
+  int32_t layer;    /* decoder layer, -1 outside the layer loop */
+  int64_t m;        /* rows (GEMM M, attention query rows, selection T, decode sequences) */
+  int64_t n;        /* GEMM N, attention key rows (decode: cached keys summed over sequences) */
+  int64_t k;        /* GEMM K, attention causal (query, key) pairs (decode: CTAs) */
+  float ms;         /* device time between the two events */
+  int32_t launches; /* kernel launches inside the record (a GEMM whose last wave runs as a
+                       separate launch, the selection's passes) */
 } dash_launch_record;
 
 /* Starts recording (clears earlier records).  capacity = max launches kept. */

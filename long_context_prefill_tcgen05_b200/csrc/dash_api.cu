@@ -99,8 +99,10 @@ cudaEvent_t next_event() {
 
 class TimedLaunch {
  public:
-  TimedLaunch(int kind, int64_t m, int64_t n, int64_t k, cudaStream_t st) : st_(st) {
-    if (!g_timing.on || static_cast<int>(g_timing.recs.size()) >= g_timing.cap) return;
+  // kind < 0: not recorded (a launch inside another record's span);
+  // launches: kernel launches the record spans
+  TimedLaunch(int kind, int64_t m, int64_t n, int64_t k, cudaStream_t st, int launches = 1) : st_(st) {
+    if (!g_timing.on || kind < 0 || static_cast<int>(g_timing.recs.size()) >= g_timing.cap) return;
     cudaEvent_t e0 = next_event(), e1 = next_event();
     if (!e0 || !e1) return;
     TimingRec t;
@@ -110,6 +112,7 @@ class TimedLaunch {
     t.r.n = n;
     t.r.k = k;
     t.r.ms = 0.f;
+    t.r.launches = launches;
     t.e0 = e0;
     t.e1 = e1;
     g_timing.recs.push_back(t);
@@ -209,7 +212,8 @@ int gemm_pair_capacity(const DeviceInfo& di) {
 
 template <int EPI, int DT>
 dash_status launch_gemm_pair(int max_pairs, const s16* A, int64_t lda, int64_t M, int K, const s16* B,
-                             const s16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind) {
+                             const s16* B2, int N, const EpiArgs& ep, cudaStream_t st, int kind,
+                             int64_t tile_limit = 0) {
   using C = dash::gemm::PairCfg;
   auto kernel = dash::gemm::gemm_pair_kernel<EPI, DT>;
   if (M == 0) return DASH_OK;
@@ -230,6 +234,7 @@ dash_status launch_gemm_pair(int max_pairs, const s16* A, int64_t lda, int64_t M
   sh.tiles_m = static_cast<int>((M + C::kRows - 1) / C::kRows);
   sh.tiles_n = N / C::BN;
   sh.num_tiles = sh.tiles_m * sh.tiles_n;
+  if (tile_limit > 0 && tile_limit < sh.num_tiles) sh.num_tiles = static_cast<int>(tile_limit);
   const int pairs = sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -260,7 +265,42 @@ dash_status gemm(const DeviceInfo& di, const s16* A, int64_t lda, int64_t M, int
     if (bn_used) *bn_used = 256;
     if (M > dash::gemm::BM && g_gemm_pairs.load(std::memory_order_relaxed)) {
       const int pairs = gemm_pair_capacity<EPI, DT>(di);
-      if (pairs > 0) return launch_gemm_pair<EPI, DT>(pairs, A, lda, M, K, B, B2, N, ep, st, kind);
+      if (pairs > 0) {
+        // Tiles run in waves of `pairs`; a last wave that is only partly full
+        // idles most SM pairs.  Its tiles come last in the grouped raster, so
+        // (once rounded up to whole columns of the last group) they form the
+        // rectangle rows [m0, M) x columns [n0, N).  When that rectangle fits
+        // one wave of 128 x 128 single-SM tiles, the pair kernel stops before
+        // it and the single-SM kernel computes it: each output element is
+        // still one tile's sum over k in the same order.
+        constexpr bool kSplittable = EPI == dash::gemm::kEpiStore || EPI == dash::gemm::kEpiResid ||
+                                     EPI == dash::gemm::kEpiQkv;
+        using PC = dash::gemm::PairCfg;
+        const int64_t tiles_m = (M + PC::kRows - 1) / PC::kRows, tiles_n = N / PC::BN;
+        const int64_t num = tiles_m * tiles_n, rem = num % pairs;
+        const int64_t g_last = tiles_m - ((tiles_m - 1) / PC::kGroupM) * PC::kGroupM;
+        const int64_t cols = (rem + g_last - 1) / g_last, rect = cols * g_last;
+        if (kSplittable && num > pairs && rem > 0 && cols < tiles_n && 4 * rect <= di.num_sms) {
+          TimedLaunch tl(kind, M, N, K, st, 2);  // one record for both launches
+          dash_status r = launch_gemm_pair<EPI, DT>(pairs, A, lda, M, K, B, B2, N, ep, st, -1, num - rect);
+          if (r != DASH_OK) return r;
+          const int64_t m0 = (tiles_m - g_last) * PC::kRows, n0 = (tiles_n - cols) * PC::BN;
+          EpiArgs e = ep;
+          if (EPI == dash::gemm::kEpiQkv) {
+            e.q = ep.q ? ep.q + m0 * ep.ldq : nullptr;
+            if (ep.pos) e.pos = ep.pos + m0;
+            if (ep.kv_rowmap) e.kv_rowmap = ep.kv_rowmap + m0;
+            if (ep.row_scale) e.row_scale = ep.row_scale + m0;
+            e.row0 = ep.row0 + static_cast<int>(m0);
+            e.col_offset = ep.col_offset + static_cast<int>(n0);
+          } else {
+            e.out = ep.out + m0 * ep.ldo + n0;
+          }
+          return launch_gemm<128, EPI, DT>(di, A + m0 * lda, lda, M - m0, K, B + n0 * K, nullptr,
+                                           static_cast<int>(cols * PC::BN), e, st, -1);
+        }
+        return launch_gemm_pair<EPI, DT>(pairs, A, lda, M, K, B, B2, N, ep, st, kind);
+      }
     }
     return launch_gemm<256, EPI, DT>(di, A, lda, M, K, B, B2, N, ep, st, kind);
   }
@@ -588,26 +628,28 @@ dash_status select_impl(const float* scores, int64_t T, const int32_t* seg, int 
   if (T == 0 || nseg == 0)
     return cudaMemsetAsync(count, 0, sizeof(int32_t) * (nseg > 0 ? nseg : 1), st) == cudaSuccess ? DASH_OK
                                                                                             : DASH_ERR_CUDA;
-  TimedLaunch tl(DASH_K_SELECT, T, nseg, 0, st);
-  if (seg) {
-    r::select_kernel<<<nseg, r::kSelThreads, 0, st>>>(scores, T, seg, kind, keep, thr, keep_first, keep_last, idx,
-                                                      halted, count);
-    return launch_status();
-  }
-  if (!sel || !sel->st) return DASH_ERR_NO_MEMORY;
   // the same middle range, k and mode as select_kernel computes on the device
   const int64_t lo = keep_first < T ? keep_first : T;
   int64_t hi = keep_last > 0 ? T - keep_last : T;
   if (hi < lo) hi = lo;
   const int64_t k_dyn = kind == DASH_SELECT_TOPK ? static_cast<int64_t>(std::floor(keep * static_cast<double>(hi - lo)))
                                                   : 0;
+  const int mode = kind == DASH_SELECT_THRESHOLD ? 3 : (k_dyn <= 0 ? 0 : (k_dyn >= hi - lo ? 1 : 2));
+  // one CTA per sequence, or the multi-SM passes (the histogram only for a top-k cut)
+  TimedLaunch tl(DASH_K_SELECT, T, nseg, 0, st, seg ? 1 : (mode == 2 ? 4 : 3));
+  if (seg) {
+    r::select_kernel<<<nseg, r::kSelThreads, 0, st>>>(scores, T, seg, kind, keep, thr, keep_first, keep_last, idx,
+                                                      halted, count);
+    return launch_status();
+  }
+  if (!sel || !sel->st) return DASH_ERR_NO_MEMORY;
   r::SelArgs a;
   a.scores = scores;
   a.T = T;
   a.lo = lo;
   a.hi = hi;
   a.k_dyn = k_dyn;
-  a.mode = kind == DASH_SELECT_THRESHOLD ? 3 : (k_dyn <= 0 ? 0 : (k_dyn >= hi - lo ? 1 : 2));
+  a.mode = mode;
   a.thr = thr;
   a.n_chunks = sel->n_chunks;
   a.st = sel->st;

@@ -51,6 +51,8 @@ struct EpiArgs {
   int hq, hkv, hd;
   int64_t rope_rows;         // kEpiQkv: positions in the RoPE table (pos must lie in [0, rope_rows))
   int64_t kv_rows;           // kEpiQkv: rows of the k / v buffers (kv rows must lie in [0, kv_rows))
+  int row0;                  // kEpiQkv: row m of this launch is row row0 + m of the whole GEMM (its
+                             // position and k/v row when pos / kv_rowmap are NULL)
 };
 
 struct Shape {
@@ -165,8 +167,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int m, int tn, con
     float sc = 1.f;
     bool ok = live;
     if (ok) {
-      p = ep.pos ? ep.pos[m] : m;
-      kvrow = ep.kv_rowmap ? ep.kv_rowmap[m] : m;
+      p = ep.pos ? ep.pos[m] : ep.row0 + m;
+      kvrow = ep.kv_rowmap ? ep.kv_rowmap[m] : ep.row0 + m;
       // Caller-supplied positions index the RoPE table and row maps pick the
       // k / v row written: a row with either out of range is flagged and
       // left unwritten.

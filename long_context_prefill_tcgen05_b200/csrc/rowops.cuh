@@ -634,12 +634,23 @@ __global__ void __launch_bounds__(kResolveThreads, 1) sel_resolve_kernel(const S
     }
     kth = prefix;
     k_rem = k;
-    // per chunk: candidates above the cut key, and equal to it
-    for (uint32_t j = tid; j < C; j += kResolveThreads) {
-      const uint32_t key = a.cand_key[j];
-      const int64_t ch = a.cand_idx[j] / kSelCtaTok;
-      if (key > kth) atomicAdd(&a.gt_extra[ch], 1u);
-      else if (key == kth) atomicAdd(&a.eq_cnt[ch], 1u);
+    // per chunk: candidates above the cut key, and equal to it (one atomic
+    // per distinct (chunk, kind) of a warp: a warp's candidates mostly share
+    // a chunk, appended together)
+    for (uint32_t base = 0; base < C; base += kResolveThreads) {
+      const uint32_t j = base + tid;
+      uint32_t kind = 0;
+      int64_t ch = 0;
+      if (j < C) {
+        const uint32_t key = a.cand_key[j];
+        ch = a.cand_idx[j] / kSelCtaTok;
+        kind = key > kth ? 1u : (key == kth ? 2u : 0u);
+      }
+      const uint32_t active = __ballot_sync(0xffffffffu, kind != 0u);
+      if (kind != 0u) {
+        const uint32_t peers = __match_any_sync(active, static_cast<uint32_t>(ch) * 4u + kind);
+        if (lane == __ffs(peers) - 1) atomicAdd(kind == 1u ? &a.gt_extra[ch] : &a.eq_cnt[ch], __popc(peers));
+      }
     }
     __syncthreads();
   }

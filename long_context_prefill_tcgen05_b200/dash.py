@@ -50,7 +50,8 @@ class Config(ctypes.Structure):
 
 
 class LaunchRecord(ctypes.Structure):
-    _fields_ = [("kind", c_i32), ("layer", c_i32), ("m", c_i64), ("n", c_i64), ("k", c_i64), ("ms", c_f32)]
+    _fields_ = [("kind", c_i32), ("layer", c_i32), ("m", c_i64), ("n", c_i64), ("k", c_i64), ("ms", c_f32),
+                ("launches", c_i32)]
 
 
 class HaltCtx(ctypes.Structure):
@@ -197,7 +198,7 @@ def timing_stop(capacity=1 << 16):
     if n < 0:
         raise DashError(5, "dash_timing_stop")
     return [{"kind": lib().dash_kernel_name(r.kind).decode(), "layer": r.layer, "m": r.m, "n": r.n,
-             "k": r.k, "ms": r.ms} for r in buf[:n]]
+             "k": r.k, "ms": r.ms, "launches": r.launches} for r in buf[:n]]
 
 
 # ----------------------------------------------------------- workspaces

@@ -229,3 +229,27 @@ def test_bf16_depth11_departure(gpu_lib):
     assert err <= 3e-2
     del stack
     torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_fp16_qwen_layer_full_T_sampled_rows(gpu_lib):
+    """One Qwen-width layer at the benchmark's launch shape (T = 32768: SM-pair
+    GEMM tiles, the full-length attention), fp16, checked on sampled rows."""
+    dims = inputs.QWEN7B
+    layers = _to(inputs.make_layers(dims, seed=11, n_layers=1), F16, DEV)
+    stack = dash.Stack(dims, layers)
+    W = {k: to_np(v) for k, v in layers[0].items()}
+    T = 32768
+    h0 = inputs.make_hidden(T, dims.d_model, seed=21, device=DEV)[0].to(F16)
+    H = h0.clone()
+    delta = torch.empty(T, device=DEV)
+    dash.layer_forward(stack, 0, H, delta=delta)
+    assert dash.device_error() == 0
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 4095, T - 1],
+                                     np.random.default_rng(0).choice(T, 250, replace=False)]))
+    hin = to_np(h0)
+    ref, u = O.decoder_block(hin[rows], rows, hin, np.arange(T), W, dims.as_dict())
+    assert row_rel_err(to_np(H)[rows], ref) < HIDDEN_TOL
+    assert _rel(delta.cpu().numpy()[rows], O.delta_scores(u)).max() < DELTA_TOL
+    del stack, layers
+    torch.cuda.empty_cache()

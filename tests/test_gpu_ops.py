@@ -134,6 +134,32 @@ def test_linear_matches_fp64(gpu_lib, M, K, N):
     _no_device_error()
 
 
+@pytest.mark.parametrize("M,K,N", [(16384, 256, 3584), (32768, 128, 3584), (9700, 512, 4608)])
+def test_linear_last_wave_rectangle_matches_single_sm_tiles(gpu_lib, M, K, N):
+    """Shapes whose last wave of SM-pair tiles is mostly idle (896 = 12 x 74 + 8,
+    1792 = 24 x 74 + 16 and 684 = 9 x 74 + 18 pair tiles, the last with a
+    ragged 38th row tile): those tiles run as a rectangle of 128 x 128
+    single-SM tiles after the others.  Every element is still one tile's sum
+    over k in the same order, so it equals the all-single-SM result."""
+    g = torch.Generator().manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(DEV)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
+    prev = dash.set_gemm_pairs(True)
+    try:
+        pair = dash.linear(A, W).cpu()
+        dash.set_gemm_pairs(False)
+        single = dash.linear(A, W).cpu()
+    finally:
+        dash.set_gemm_pairs(prev)
+    _no_device_error()
+    diff = (pair.float() - single.float()).abs().max().item()
+    print(f"M={M} N={N} K={K}: max |pair - single| = {diff}")
+    assert diff == 0.0
+    rows = np.unique(np.r_[0, M - 1, np.arange(M - 300, M), np.random.default_rng(0).choice(M, 200, replace=False)])
+    ref = to_np(A.cpu())[rows] @ to_np(W.cpu()).T
+    assert row_rel_err(to_np(pair)[rows], ref) < 5e-3
+
+
 @pytest.mark.parametrize("M,K,N", [(129, 64, 256), (300, 3584, 4608), (1000, 18944, 512), (4096, 3584, 4608),
                                    (8192, 3584, 3584)])
 def test_linear_pair_tiles_match_fp64_and_single_sm_tiles(gpu_lib, M, K, N):

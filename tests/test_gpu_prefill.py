@@ -323,6 +323,48 @@ def test_qwen_layer_pair_tiles_match_single_sm_tiles(qwen_layer, mode):
                        np.arange(T), dp)
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+def test_qwen_layer_last_wave_rectangle(qwen_layer, mode):
+    """9700 rows at Qwen2.5-7B widths: the QKV GEMM's 684 pair tiles leave a
+    last wave of 18, which runs as a rectangle of single-SM tiles (rows 8192
+    onwards, the last 768 qkv columns: k and v heads) -- with positions
+    (prune) and with the k/v row map of halt mode.  Bitwise equal to the
+    all-single-SM layer; sampled rows, including rows of the rectangle,
+    against the oracle."""
+    dims, stack, W = qwen_layer
+    T, M = 16384, 9700
+    rng = np.random.default_rng(7)
+    idx = np.sort(rng.choice(T, M, replace=False))
+    halted = np.setdiff1d(np.arange(T), idx)
+    hfull, _ = inputs.make_hidden(T, dims.d_model, seed=25, device=DEV)
+    ti = torch.tensor(idx, dtype=torch.int32, device=DEV)
+    th = torch.tensor(halted, dtype=torch.int32, device=DEV)
+
+    def run(pairs):
+        prev = dash.set_gemm_pairs(pairs)
+        try:
+            H = hfull[ti.long()].contiguous()
+            if mode == "prune":
+                dash.layer_forward(stack, 0, H, pos=ti, max_pos=T)
+            else:
+                dash.layer_forward(stack, 0, H, halt=(ti, th, hfull))
+        finally:
+            dash.set_gemm_pairs(prev)
+        assert dash.device_error() == 0
+        return H.cpu()
+
+    Hp, Hs = run(True), run(False)
+    assert torch.equal(Hp, Hs)
+    rows = np.unique(np.r_[0, M - 1, rng.choice(np.arange(8192, M), 40, replace=False),
+                           rng.choice(8192, 24, replace=False)])
+    h_in = hfull[ti.long()].cpu()
+    if mode == "prune":
+        _sampled_check(dims, W, h_in, Hp, rows, idx[rows], h_in, idx)
+    else:
+        _sampled_check(dims, W, h_in, Hp, rows, idx[rows], hfull.cpu(), np.arange(T))
+
+
 # ------------------------------------- reduced Qwen-shaped, end to end
 def _clear_keep(delta, q, window=400):
     """A keep fraction near q whose top-k cut falls in the widest relative gap
