@@ -963,7 +963,6 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
 namespace dec = dash::decode;
 
 struct DecodeWs {
-  int* counters;   // [kMaxSegs] finished decode-attention CTAs per segment
   s16* Q;         // [n, hq*hd]
   s16* O;         // [n, hq*hd] attention output
   s16* Act;       // [n, F]
@@ -973,7 +972,6 @@ struct DecodeWs {
 
 void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
-  w.counters = c.take<int>(dec::kMaxSegs);
   w.Q = c.take<s16>(n * qd);
   w.O = c.take<s16>(n * qd);
   w.Act = c.take<s16>(static_cast<size_t>(n) * D.ffn_dim);
@@ -1000,11 +998,12 @@ cudaError_t launch_pdl(void (*kernel)(ExpTypes...), unsigned grid, unsigned bloc
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<ActTypes>(args)...);
 }
 
-constexpr size_t kGemvSmemMax = 160 * 1024;  // x staged in shared memory up to this size
+constexpr size_t kGemvSmemMax = 160 * 1024;    // x staged in shared memory up to this size
+constexpr size_t kGemvSmemTotal = 224 * 1024;  // staged x + the warps' first-task weight slots
 
 template <int EPI, int NS, int DT>
 dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out,
-                           cudaStream_t st) {
+                           bool preload, cudaStream_t st) {
   if (gp.tasks == 0) return DASH_OK;
   constexpr bool kNorm = EPI != dec::kGvResid;
   const size_t xbytes = static_cast<size_t>(gp.n) * gp.K * 2;
@@ -1012,12 +1011,24 @@ dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int 
   if (kNorm && xbytes > kGemvSmemMax) return DASH_ERR_SHAPE;
   dec::GemvParams q = gp;
   q.stage_x = !kNorm && stage;
-  const size_t smem = stage ? xbytes : 0;
+  const size_t xs = stage ? xbytes : 0;
+  // preload: the rest of shared memory holds two rows' leading bytes per
+  // warp, loaded before the PDL wait (whole rows when they fit).  Only for
+  // the down projection: a kernel's PDL wait is released after the copies
+  // then in flight on the device complete, so behind a short predecessor
+  // (the attention merge before o_proj, the down projection before QKV)
+  // a preload delays the kernel more than it saves.
+  size_t pre = !preload || kNorm ? 0 : (kGemvSmemTotal - xs) / (2 * dec::kGemvWarps) & ~static_cast<size_t>(15);
+  if (pre > static_cast<size_t>(gp.K) * 2) pre = static_cast<size_t>(gp.K) * 2;
+  if (pre < 1024) pre = 0;
+  q.x_smem = static_cast<int>(xs);
+  q.pre_bytes = static_cast<int>(pre);
+  const size_t smem = xs + 2 * dec::kGemvWarps * pre;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
     attr_err = cudaFuncSetAttribute(dec::gemv_kernel<EPI, NS, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(kGemvSmemMax));
+                                    static_cast<int>(kNorm ? kGemvSmemMax : kGemvSmemTotal));
   });
   if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
   // one CTA per SM (tasks strided over the grid), so every SM streams weights
@@ -1029,11 +1040,12 @@ dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int 
 }
 
 template <int EPI, int DT>
-dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st) {
-  if (gp.n <= 1) return launch_gemv_ns<EPI, 1, DT>(di, gp, kind, n_out, st);
-  if (gp.n <= 2) return launch_gemv_ns<EPI, 2, DT>(di, gp, kind, n_out, st);
-  if (gp.n <= 4) return launch_gemv_ns<EPI, 4, DT>(di, gp, kind, n_out, st);
-  return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, st);
+dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st,
+                        bool preload = false) {
+  if (gp.n <= 1) return launch_gemv_ns<EPI, 1, DT>(di, gp, kind, n_out, preload, st);
+  if (gp.n <= 2) return launch_gemv_ns<EPI, 2, DT>(di, gp, kind, n_out, preload, st);
+  if (gp.n <= 4) return launch_gemv_ns<EPI, 4, DT>(di, gp, kind, n_out, preload, st);
+  return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, preload, st);
 }
 
 // Split-key decode attention of one layer: the CTA count is held to one
@@ -1041,8 +1053,7 @@ dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kin
 // tiles_per_cta key tiles of one (sequence, kv head) segment.
 template <int HD, int DT>
 dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n, const int64_t* len,
-                                const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st,
-                                const dec::Prefetch* next = nullptr) {
+                                const dash_kv_cache* const* layer_caches, const DecodeWs& w, cudaStream_t st) {
   using C = dec::ACfg<HD>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -1090,7 +1101,6 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   ap.seg_cta0[n * hkv] = c0;
   ap.q = w.Q;
   ap.out = w.O;
-  ap.counters = w.counters;
   ap.part_o = w.part_o;
   ap.part_ml = w.part_ml;
   ap.n = n;
@@ -1099,11 +1109,30 @@ dash_status decode_attention_hd(const DeviceInfo& di, const dash_dims& D, int n,
   ap.group = D.n_heads / hkv;
   ap.tiles_per_cta = static_cast<int>(per);
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HD)));
-  if (next) ap.next = *next;
-  TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, nctas, st);
+  dec::MergeParams mp;
+  std::memset(&mp, 0, sizeof(mp));
+  mp.part_o = w.part_o;
+  mp.part_ml = w.part_ml;
+  mp.out = w.O;
+  mp.n = n;
+  mp.hq = D.n_heads;
+  mp.hkv = hkv;
+  mp.group = ap.group;
+  mp.hd = HD;
+  mp.items = n * hkv * ap.group * (HD / 32);
+  std::memcpy(mp.seg_cta0, ap.seg_cta0, sizeof(mp.seg_cta0));
+  TimedLaunch tl(DASH_K_DEC_ATTENTION, n, keys, nctas, st, 2);
   if (launch_pdl(dec::decode_attn_kernel<HD, DT>, static_cast<unsigned>(nctas), dec::kAttnThreads, C::kSmemBytes, st,
                  maps, ap) != cudaSuccess)
     return DASH_ERR_CUDA;
+  // The merge is launched in plain stream order (it starts once the attention
+  // has completed).  Launched with PDL it was resident early, and o_proj's
+  // CTAs, which cannot start before the attention grid completes, then
+  // started ~3 us after the attention's CTAs exited and the merge's wait was
+  // released ~4 us after the attention ended; the step measured 2% slower.
+  const unsigned mgrid = static_cast<unsigned>((mp.items + dec::kMergeWarps - 1) / dec::kMergeWarps);
+  dec::decode_merge_kernel<DT><<<mgrid, 32 * dec::kMergeWarps, 0, st>>>(mp);
+  if (cudaGetLastError() != cudaSuccess) return DASH_ERR_CUDA;
   return launch_status();
 }
 
@@ -1140,7 +1169,6 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
   s16* x = reinterpret_cast<s16*>(X);
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd;
-  if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
 
   for (int l = 0; l < D.n_layers; ++l) {
     g_timing.layer = l;
@@ -1171,21 +1199,10 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     qkv.hkv = hkv;
     qkv.hd = hd;
     qkv.theta = D.rope_theta;
-    for (int q = 0; q < n; ++q) {  // the attention streams this layer's cache next
-      const uint64_t bytes = static_cast<uint64_t>(lc[q]->len) * hkv * hd * 2;
-      qkv.next.ptr[qkv.next.count] = reinterpret_cast<const uint8_t*>(lc[q]->k);
-      qkv.next.bytes[qkv.next.count++] = bytes;
-      qkv.next.ptr[qkv.next.count] = reinterpret_cast<const uint8_t*>(lc[q]->v);
-      qkv.next.bytes[qkv.next.count++] = bytes;
-    }
     if ((s = launch_gemv<dec::kGvQkv, DT>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
     // attention over each sequence's cache (including the new row)
-    dec::Prefetch wo{};  // o_proj streams W_o next
-    wo.ptr[0] = reinterpret_cast<const uint8_t*>(lw.w_o);
-    wo.bytes[0] = static_cast<uint64_t>(d) * qd * 2;
-    wo.count = 1;
-    s = hd == 128 ? decode_attention_hd<128, DT>(*di, D, n, len, lc, w, st, &wo)
-                  : decode_attention_hd<64, DT>(*di, D, n, len, lc, w, st, &wo);
+    s = hd == 128 ? decode_attention_hd<128, DT>(*di, D, n, len, lc, w, st)
+                  : decode_attention_hd<64, DT>(*di, D, n, len, lc, w, st);
     if (s != DASH_OK) break;
     // o_proj + residual
     dec::GemvParams o;
@@ -1197,14 +1214,6 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     o.tasks = d / 2;
     o.out = x;
     o.ldo = d;
-    {  // gate/up's first round of rows (every warp of the grid takes one task)
-      const int64_t first = std::min<int64_t>(F, static_cast<int64_t>(di->num_sms) * dec::kGemvWarps);
-      o.next.ptr[0] = reinterpret_cast<const uint8_t*>(lw.w_gate);
-      o.next.bytes[0] = static_cast<uint64_t>(first) * d * 2;
-      o.next.ptr[1] = reinterpret_cast<const uint8_t*>(lw.w_up);
-      o.next.bytes[1] = static_cast<uint64_t>(first) * d * 2;
-      o.next.count = 2;
-    }
     if ((s = launch_gemv<dec::kGvResid, DT>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
     // RMSNorm (fused) -> gate/up with SwiGLU
     dec::GemvParams gu;
@@ -1230,12 +1239,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     dn.tasks = d / 2;
     dn.out = x;
     dn.ldo = d;
-    if (l + 1 < D.n_layers) {  // the next layer's QKV weights
-      dn.next.ptr[0] = reinterpret_cast<const uint8_t*>(layers[l + 1].w_qkv);
-      dn.next.bytes[0] = static_cast<uint64_t>(qd + 2 * hkv * hd) * d * 2;
-      dn.next.count = 1;
-    }
-    if ((s = launch_gemv<dec::kGvResid, DT>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid, DT>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st, true)) != DASH_OK) break;
     for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
   }
   g_timing.layer = -1;
@@ -1518,8 +1522,7 @@ dash_status dash_prefill_varlen_kv(const dash_dims* dims, const dash_layer_weigh
 
 size_t dash_decode_attention_workspace_size(int32_t hd) {
   if (hd != 64 && hd != 128) return 0;
-  return static_cast<size_t>(dash::decode::kMaxCtas) * dash::decode::kGroupPad * (hd + 2) * sizeof(float) +
-         dash::decode::kMaxSegs * sizeof(int) + 1024;
+  return static_cast<size_t>(dash::decode::kMaxCtas) * dash::decode::kGroupPad * (hd + 2) * sizeof(float) + 1024;
 }
 
 dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_kv_cache* caches, int32_t hq,
@@ -1554,11 +1557,9 @@ dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_k
   DecodeWs w{};
   w.Q = const_cast<s16*>(reinterpret_cast<const s16*>(Q));
   w.O = reinterpret_cast<s16*>(O);
-  w.counters = c.take<int>(dec::kMaxSegs);
   w.part_o = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * hd);
   w.part_ml = c.take<float>(static_cast<size_t>(dec::kMaxCtas) * dec::kGroupPad * 2);
   cudaStream_t st = as_stream(stream);
-  if (cudaMemsetAsync(w.counters, 0, sizeof(int) * dec::kMaxSegs, st) != cudaSuccess) return DASH_ERR_CUDA;
   return hd == 128 ? decode_attention_hd<128, kBf16>(*di, D, nseq, len, lc, w, st)
                    : decode_attention_hd<64, kBf16>(*di, D, nseq, len, lc, w, st);
 }

@@ -42,38 +42,24 @@ constexpr int kMaxCtas = 256;  // decode-attention CTAs (partial-result slots)
 constexpr int kGroupPad = 16;  // query heads per kv head, padded (MMA N)
 constexpr int BKV = 128;       // keys per tile (MMA M)
 constexpr int kStages = 3;
+constexpr int kPrefetchTiles = 3;  // decode attention: tiles sent to L2 before the PDL wait
 constexpr int kAttnThreads = 192;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units, as in the prefill softmax
 
-// ========================================================= L2 prefetch
-// Regions the NEXT kernel of the step will stream (its weights or the
-// cache), fetched into L2 by the TMA engine while this kernel runs: the
-// kernels of a decode step alternate between latency-bound phases (launch,
-// prologue, merge) and bandwidth-bound streaming, so the prefetch fills the
-// former with the latter's bytes.
-constexpr int kMaxPrefetch = 2 * kMaxSeq;
-struct Prefetch {
-  const uint8_t* ptr[kMaxPrefetch];
-  uint64_t bytes[kMaxPrefetch];
-  int count;
-};
-
+// ============================================================ async copies
+// (Prefetching the next kernel's weights or cache into L2 during a kernel
+// measured slower: a step's kernels are bandwidth-bound while they stream,
+// and the prefetch only moved bytes between them.)
 __device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(ptr)), "r"(bytes)
                : "memory");
 }
 
-// Thread 0 of every CTA prefetches its share of each region (16-byte
-// aligned starts and sizes; a region's last partial 16 bytes are skipped).
-__device__ __forceinline__ void prefetch_share(const Prefetch& pf) {
-  if (threadIdx.x != 0) return;
-  for (int r = 0; r < pf.count; ++r) {
-    const uint64_t total = pf.bytes[r] & ~15ull;
-    const uint64_t per = ((total + gridDim.x - 1) / gridDim.x + 15) & ~15ull;
-    uint64_t a = per * blockIdx.x;
-    const uint64_t e = a + per < total ? a + per : total;
-    for (; a < e; a += 65536) prefetch_l2(pf.ptr[r] + a, static_cast<uint32_t>(e - a < 65536 ? e - a : 65536));
-  }
+// Bulk async copy global -> shared (no tensor map), completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // =================================================================== GEMV
@@ -95,13 +81,15 @@ struct GemvParams {
   float eps;
   int n, K, tasks;
   int stage_x;                // kGvResid: copy x to shared memory first (it fits)
+  int x_smem;                 // bytes of dynamic shared memory taken by staged x (16-byte multiple)
+  int pre_bytes;              // leading bytes of each row of a warp's first task loaded to shared
+                              // memory before the PDL wait (16-byte multiple, <= 2K; 0: none)
   s16* out;  // kGvResid: residual stream [n, ldo] (in/out); kGvSwiglu: act [n, ldo]
   int64_t ldo;
   s16* q;  // kGvQkv: [n, hq*hd]
   int hq, hkv, hd;
   double theta;
   SeqSlots seq;
-  Prefetch next;  // what the next kernel streams
 };
 
 constexpr int kGemvWarps = 16;  // one CTA per SM; warps take tasks strided over the grid
@@ -162,17 +150,88 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* ptr) {
 // input row's 1/rms and stages x * gain in shared memory, in the model's
 // 16-bit format (exact for unit gains); the 1/rms multiplies the finished dot products, as the
 // prefill's GEMM epilogues do.  kGvResid stages x as is when it fits.
+//
+// Weights are never written during a step, so they need not wait for the
+// previous kernel: before its PDL wait every warp starts bulk copies of the
+// leading pre_bytes of its first task's two rows into its own shared-memory
+// slot.  A CTA starts as soon as the previous kernel's CTA on its SM exits,
+// so these copies fill the previous kernel's tail (its SMs finish unevenly,
+// the attention's merge runs on a few) with this kernel's own bytes.
 template <int EPI, int NS, int DT>
 __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvParams p) {
   constexpr bool kNorm = EPI != kGvResid;
   extern __shared__ uint4 xg_smem[];  // kNorm: [n][K/8]
   __shared__ float red[kGemvWarps][kMaxSeq];
   __shared__ float rs_s[kMaxSeq];
+  __shared__ __align__(8) uint64_t pre_bar[kGemvWarps];
+  __shared__ float2 rope_cs[EPI == kGvQkv ? kMaxSeq * 64 : 1];  // [m][i]: (cos, sin)
   pdl_trigger();
-  prefetch_share(p.next);  // independent of the previous kernel
-  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = p.K, nv = K >> 3;
+  if constexpr (EPI == kGvQkv) {
+    // RoPE rotation of every (input row, frequency) pair: the positions are
+    // launch arguments, so this fp64 work runs before the PDL wait, off the
+    // critical path (fp64 angle, as the prefill's table)
+    const int half = p.hd >> 1;
+    if (threadIdx.x < p.n * half) {
+      const int m = threadIdx.x / half, i = threadIdx.x - m * half;
+      const double inv = pow(p.theta, -2.0 * i / static_cast<double>(p.hd));
+      double sn, cs;
+      sincos(static_cast<double>(p.seq.p[m]) * inv, &sn, &cs);
+      rope_cs[threadIdx.x] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
+  }
+  // the two weight rows of a task
+  auto rows = [&](int task, const s16*& w0, const s16*& w1) {
+    if constexpr (EPI == kGvQkv) {
+      const int half = p.hd >> 1;
+      const int head = task / half, i = task - head * half;
+      w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
+      w1 = w0 + static_cast<int64_t>(half) * K;
+    } else if constexpr (EPI == kGvSwiglu) {
+      w0 = p.W + static_cast<int64_t>(task) * K;
+      w1 = p.W2 + static_cast<int64_t>(task) * K;
+    } else {
+      w0 = p.W + static_cast<int64_t>(2 * task) * K;
+      w1 = w0 + K;
+    }
+  };
+  const int task0 = blockIdx.x + gridDim.x * warp;
+  const bool pre = p.pre_bytes > 0 && task0 < p.tasks;  // warp-uniform
+  const uint4* pre_w = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(xg_smem) + p.x_smem +
+                                                      static_cast<int64_t>(warp) * 2 * p.pre_bytes);
+  const uint32_t bar = smem_u32(&pre_bar[warp]);
+  if (pre && lane == 0) {
+    const s16* r0;
+    const s16* r1;
+    rows(task0, r0, r1);
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, 2u * p.pre_bytes);
+    bulk_load(smem_u32(pre_w), r0, p.pre_bytes, bar);
+    bulk_load(smem_u32(pre_w) + p.pre_bytes, r1, p.pre_bytes, bar);
+  }
+  constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
+  // A round of a task's two rows: U 16-byte chunks per row per lane.
+  // Without a shared-memory preload, the first task's first round is loaded
+  // into these registers before the PDL wait (weights do not depend on the
+  // previous kernel), so its latency overlaps the wait and the staging of x.
+  uint4 ra[U], rb[U];
+  const bool reg0 = !pre && task0 < p.tasks;  // warp-uniform
+  if (reg0) {
+    const s16* r0;
+    const s16* r1;
+    rows(task0, r0, r1);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = lane + 32 * u;
+      if (c < nv) {
+        ra[u] = ldg_stream(reinterpret_cast<const uint4*>(r0) + c);
+        rb[u] = ldg_stream(reinterpret_cast<const uint4*>(r1) + c);
+      }
+    }
+  }
+  pdl_wait();
   const uint4* xg = reinterpret_cast<const uint4*>(p.x);
   if constexpr (kNorm) {
     float ss[NS];
@@ -209,24 +268,19 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
     xg = xg_smem;
   }
   const bool from_smem = kNorm || p.stage_x;
-  constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
   const int stride = gridDim.x * kGemvWarps;
-  // the two weight rows of a task
-  auto rows = [&](int task, const s16*& w0, const s16*& w1) {
-    if constexpr (EPI == kGvQkv) {
-      const int half = p.hd >> 1;
-      const int head = task / half, i = task - head * half;
-      w0 = p.W + static_cast<int64_t>(head * p.hd + i) * K;
-      w1 = w0 + static_cast<int64_t>(half) * K;
-    } else if constexpr (EPI == kGvSwiglu) {
-      w0 = p.W + static_cast<int64_t>(task) * K;
-      w1 = p.W2 + static_cast<int64_t>(task) * K;
-    } else {
-      w0 = p.W + static_cast<int64_t>(2 * task) * K;
-      w1 = w0 + K;
+  // chunks of the first task's rows in shared memory
+  int pv = 0;
+  if (pre) {
+    // every lane observes the phase (the copies' writes are then visible to it)
+    if (!__all_sync(0xffffffffu, mbar_wait(bar, 0))) {  // bounded; flagged as a timeout
+      if (lane == 0) mbar_wait_drain(bar, 0);
+      return;
     }
-  };
-  for (int task = blockIdx.x + gridDim.x * warp; task < p.tasks; task += stride) {
+    pv = p.pre_bytes >> 4;
+  }
+  // One task; `first` (the warp's first task) takes the preloaded bytes.
+  auto run_task = [&](int task, bool first) {
     int head = 0, i = 0;
     if constexpr (EPI == kGvQkv) {
       head = task / (p.hd >> 1);
@@ -235,6 +289,12 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
     const s16* w0;
     const s16* w1;
     rows(task, w0, w1);
+    // kGvResid: lane m loads the two residual values of input row m now, so
+    // the load's latency hides behind the task's dot products
+    uint32_t res = 0;
+    if constexpr (EPI == kGvResid) {
+      if (lane < p.n) res = *reinterpret_cast<const uint32_t*>(p.out + static_cast<int64_t>(lane) * p.ldo + 2 * task);
+    }
     // The next task's rows go to L2 while this one streams.  (Prefetching the
     // current task's rows as well measured slower: the demand loads race
     // their own prefetch.)
@@ -252,14 +312,19 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
     float a0[NS], a1[NS];
 #pragma unroll
     for (int m = 0; m < NS; ++m) a0[m] = a1[m] = 0.f;
+    const int npv = first ? pv : 0;
     for (int c0 = lane; c0 < nv; c0 += 32 * U) {
-      uint4 ra[U], rb[U];
+      if (!(first && reg0 && c0 == lane)) {  // else: the first round is in ra, rb already
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = c0 + 32 * u;
-        if (c < nv) {
-          ra[u] = ldg_stream(wa + c);  // weights stream through once per step
-          rb[u] = ldg_stream(wb + c);
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + 32 * u;
+          if (c < npv) {
+            ra[u] = pre_w[c];
+            rb[u] = pre_w[npv + c];
+          } else if (c < nv) {
+            ra[u] = ldg_stream(wa + c);  // weights stream through once per step
+            rb[u] = ldg_stream(wb + c);
+          }
         }
       }
 #pragma unroll
@@ -294,11 +359,9 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
       if constexpr (EPI == kGvQkv) {
         const int hd = p.hd, half = hd >> 1;
         float o0 = y0, o1 = y1;
-        if (head < p.hq + p.hkv) {  // rotate-half RoPE at the token's position (fp64 angle)
-          const double inv = pow(p.theta, -2.0 * i / static_cast<double>(hd));
-          double sn, cs;
-          sincos(static_cast<double>(p.seq.p[m]) * inv, &sn, &cs);
-          const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+        if (head < p.hq + p.hkv) {  // rotate-half RoPE at the token's position
+          const float2 r = rope_cs[m * half + i];
+          const float c = r.x, s = r.y;
           o0 = y0 * c - y1 * s;
           o1 = y1 * c + y0 * s;
         }
@@ -318,11 +381,13 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
         p.out[static_cast<int64_t>(m) * p.ldo + task] = Num<DT>::from_f(y0 / (1.f + __expf(-y0)) * y1);
       } else {
         s16* o = p.out + static_cast<int64_t>(m) * p.ldo + 2 * task;
-        const float r0 = Num<DT>::to_f(o[0]) + y0, r1 = Num<DT>::to_f(o[1]) + y1;
+        const float r0 = Num<DT>::lo(res) + y0, r1 = Num<DT>::hi(res) + y1;
         *reinterpret_cast<uint32_t*>(o) = Num<DT>::pack(r0, r1);
       }
     }
-  }
+  };
+  if (task0 < p.tasks) run_task(task0, true);
+  for (int task = task0 + stride; task < p.tasks; task += stride) run_task(task, false);
 }
 
 // ========================================================= decode attention
@@ -332,12 +397,10 @@ struct AttnParams {
   float* part_o;           // [CTA c][g < group][HD]: unnormalised O of each CTA (a segment's CTAs adjacent)
   float* part_ml;          // [CTA c][16][2]: (running max in log2 units, sum); 128 bytes per CTA, so
                            // a segment's block starts 16-byte aligned for the bulk copy
-  int* counters;           // [kMaxSegs] finished CTAs per segment (zero before the launch; left zero)
   int n, hq, hkv, group, tiles_per_cta;
   int len[kMaxSeq];                // keys of each sequence (cache rows incl. the new one)
   int seg_cta0[kMaxSegs + 1];      // first CTA of segment s * hkv + h; [nseg] = CTA count
   float scale_log2;                // log2(e) / sqrt(HD)
-  Prefetch next;                   // what the next kernel streams
 };
 
 struct AttnMaps {
@@ -359,8 +422,8 @@ struct ACfg {
   static constexpr int kOffP = kOffQ + kPanels * 2048;  // 2 buffers of [16, 128 keys] K-major, 2 x 2 KB each
   static constexpr int kOffRed = kOffP + 2 * 4096;      // [2][4 warps][16] floats
   static constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 4;
-  // full[kStages], empty[kStages], q_ready, s_full[2], p_full[2], pv_done[2], red[2], drain, pub, merge
-  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 1 + 1 + 1;
+  // full[kStages], empty[kStages], q_ready, s_full[2], p_full[2], pv_done[2], red[2], drain
+  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
   static constexpr uint32_t kTmemCols = 64;  // S^T buffers [0,16) [16,32), O^T [32,48)
 };
@@ -395,106 +458,6 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int panel_byt
 }
 
 
-// Bulk async copy global -> shared (no tensor map), completing on `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
-// Merge of one (sequence, kv head) segment's partial results by all threads
-// of its last CTA (after the CTA's final barrier; the K/V stages are free):
-//   M_g = max_c m_cg,  w_cg = 2^(m_cg - M_g) / sum_c' 2^(m_c'g - M_g) l_c'g,
-//   O_g = sum_c w_cg o_cg.
-// A segment's partial results are adjacent in memory, so they come into
-// shared memory by a few large bulk async copies (one L2 round trip each).
-template <int HD, int DT>
-__device__ void merge_segment(const AttnParams& p, int seg, int s, int kvh, uint8_t* scratch, int scratch_bytes,
-                              uint32_t bar) {
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int G = p.group;
-  const int c0 = p.seg_cta0[seg], nch = p.seg_cta0[seg + 1] - c0;
-  float2* ml = reinterpret_cast<float2*>(scratch);                         // [nch][16] (m, l)
-  float* wt = reinterpret_cast<float*>(scratch + kMaxCtas * kGroupPad * 8);  // [nch][G] weights
-  float* os = wt + kMaxCtas * kGroupPad;                                    // [chunk][G][HD]
-  const int row_bytes = G * HD * 4;
-  const int chunk = (scratch_bytes - kMaxCtas * kGroupPad * 12) / row_bytes;
-  const float* po = p.part_o + static_cast<int64_t>(c0) * G * HD;
-  uint32_t phase = 0;
-  if (t == 0) {
-    __threadfence();
-    asm volatile("fence.proxy.async.global;" ::: "memory");  // other CTAs' partials -> the async proxy
-    const uint32_t ml_bytes = nch * kGroupPad * 8;  // source offset c0 * 128 bytes: 16-byte aligned
-    const int cn = min(chunk, nch);
-    mbar_arrive_expect_tx(bar, ml_bytes + cn * row_bytes);
-    bulk_load(smem_u32(ml), p.part_ml + static_cast<int64_t>(c0) * kGroupPad * 2, ml_bytes, bar);
-    bulk_load(smem_u32(os), po, cn * row_bytes, bar);
-  }
-  constexpr int kOut4 = kGroupPad * HD / 4;
-  constexpr int kMaxOut = (kOut4 + kAttnThreads - 1) / kAttnThreads;
-  float4 acc[kMaxOut];
-#pragma unroll
-  for (int j = 0; j < kMaxOut; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int n4 = G * HD / 4;
-  for (int cs = 0; cs < nch; cs += chunk) {
-    const int cn = min(chunk, nch - cs);
-    if (cs > 0) {
-      __syncthreads();  // previous chunk consumed
-      if (t == 0) {
-        mbar_arrive_expect_tx(bar, cn * row_bytes);
-        bulk_load(smem_u32(os), po + static_cast<int64_t>(cs) * G * HD, cn * row_bytes, bar);
-      }
-    }
-    mbar_wait(bar, phase);
-    phase ^= 1u;
-    if (cs == 0) {
-      for (int g = warp; g < G; g += kAttnThreads / 32) {
-        float M = -INFINITY;
-        for (int c = lane; c < nch; c += 32) M = fmaxf(M, ml[c * kGroupPad + g].x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
-        for (int c = lane; c < nch; c += 32) L = fmaf(ex2f(ml[c * kGroupPad + g].x - M), ml[c * kGroupPad + g].y, L);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        const float inv = 1.f / L;
-        for (int c = lane; c < nch; c += 32) wt[c * G + g] = ex2f(ml[c * kGroupPad + g].x - M) * inv;
-      }
-      __syncthreads();
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxOut; ++j) {
-      const int i = t + j * kAttnThreads;  // float4 output: head g, dimensions 4 * (i % (HD/4))
-      if (i < n4) {
-        const int g = i / (HD / 4);
-        float4 a = acc[j];
-        const float4* src = reinterpret_cast<const float4*>(os) + i;
-#pragma unroll 4
-        for (int c = 0; c < cn; ++c) {
-          const float w = wt[(cs + c) * G + g];
-          const float4 o = src[c * n4];
-          a.x = fmaf(w, o.x, a.x);
-          a.y = fmaf(w, o.y, a.y);
-          a.z = fmaf(w, o.z, a.z);
-          a.w = fmaf(w, o.w, a.w);
-        }
-        acc[j] = a;
-      }
-    }
-  }
-  s16* dst = p.out + static_cast<int64_t>(s) * p.hq * HD + static_cast<int64_t>(kvh) * G * HD;
-#pragma unroll
-  for (int j = 0; j < kMaxOut; ++j) {
-    const int i = t + j * kAttnThreads;
-    if (i < n4) {
-      uint2 v;
-      v.x = Num<DT>::pack(acc[j].x, acc[j].y);
-      v.y = Num<DT>::pack(acc[j].z, acc[j].w);
-      *reinterpret_cast<uint2*>(dst + 4 * i) = v;
-    }
-  }
-}
-
 // One CTA = a run of up to tiles_per_cta key tiles of one (sequence, kv head)
 // segment.  Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.
 // Warps 2..5: Q staging, softmax (lane r = key r of the tile), and the
@@ -507,8 +470,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   pdl_trigger();
-  prefetch_share(p.next);
-  pdl_wait();  // q and the appended cache row come from the previous kernel
   const int b = blockIdx.x;
   const int nseg = p.n * p.hkv;
   int seg = 0;
@@ -518,6 +479,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int tiles = (L + BKV - 1) / BKV;
   const int t0 = (b - p.seg_cta0[seg]) * p.tiles_per_cta;
   const int nt = min(t0 + p.tiles_per_cta, tiles) - t0;
+  // The CTA's first tiles go to L2 while the previous kernel finishes (an L2
+  // prefetch is only a hint: the tile holding the row that kernel appends is
+  // read again, coherently, after the wait).
+  if (threadIdx.x == 0)
+    for (int i = 0; i < min(nt, kPrefetchTiles); ++i)
+      for (int pn = 0; pn < HD / 64; ++pn) {
+        tma_prefetch_l2_2d(&maps.k[s], kvh * HD + pn * 64, (t0 + i) * BKV);
+        tma_prefetch_l2_2d(&maps.v[s], kvh * HD + pn * 64, (t0 + i) * BKV);
+      }
+  pdl_wait();  // q and the appended cache row come from the previous kernel
   if (nt <= 0) return;  // uniform for the whole CTA
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -529,10 +500,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar_pvdone = bar_q + 40;  // [2] P^T(i) V(i) finished, buffer i & 1 free
   const uint32_t bar_red = bar_q + 56;     // [2]
   const uint32_t bar_drain = bar_q + 72;
-  const uint32_t bar_pub = bar_q + 80;    // 128 epilogue threads published their partials
-  const uint32_t bar_merge = bar_q + 88;  // bulk copies of the merge
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
-  int* ticket = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -550,9 +518,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar_red, 128);
     mbar_init(bar_red + 8, 128);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_pub, 128);
-    mbar_init(bar_merge, 1);
-    *ticket = 0;
     fence_mbar_init();
   }
   if (HD == 64) {  // zero panel read as the upper half of V^T
@@ -802,18 +767,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pm[0] = mr;
           pm[1] = lr;
         }
-        // The last CTA of the segment to finish merges every CTA's partial
-        // result, after the CTA's final barrier.
-        // (The fence of the counting thread, after it has seen every
-        // thread's stores through the mbarrier, orders them before its atomic.)
-        mbar_arrive(bar_pub);
-        if (r == 0) {
-          const int c0 = p.seg_cta0[seg], c1 = p.seg_cta0[seg + 1];
-          if (mbar_wait(bar_pub, 0)) {
-            __threadfence();
-            *ticket = atomicAdd(&p.counters[seg], 1) == c1 - c0 - 1 ? 1 : 0;
-          }
-        }
       }
     }
   }
@@ -823,10 +776,82 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  if (*ticket == 1) {  // uniform: written before the barrier above
-    merge_segment<HD, DT>(p, seg, s, kvh, smem + C::kOffK, C::kOffZero - C::kOffK, bar_merge);
-    if (threadIdx.x == 0) p.counters[seg] = 0;  // ready for the next launch
+}
+
+// Merge of every (sequence, kv head) segment's partial results, launched
+// after the attention kernel (PDL).  One warp per (segment, head g of its
+// group, 32 dimensions); lane = dimension:
+//   M_g = max_c m_cg,  w_cg = 2^(m_cg - M_g) / sum_c' 2^(m_c'g - M_g) l_c'g,
+//   O_g = sum_c w_cg o_cg  (c ascending).
+// (The last CTA of each segment used to merge inside the attention kernel:
+// one SM then read all of the segment's partials while the others idled.)
+struct MergeParams {
+  const float* part_o;   // as AttnParams
+  const float* part_ml;
+  s16* out;              // [n, hq*hd]
+  int n, hq, hkv, group, hd, items;
+  int seg_cta0[kMaxSegs + 1];
+};
+constexpr int kMergeWarps = 4;
+
+template <int DT>
+__global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const MergeParams p) {
+  __shared__ float wsm[kMergeWarps][kMaxCtas];
+  pdl_trigger();
+  pdl_wait();  // the partials come from the attention kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * kMergeWarps + warp;
+  if (item >= p.items) return;
+  const int slices = p.hd >> 5, G = p.group;
+  const int seg = item / (G * slices);
+  const int rem = item - seg * G * slices;
+  const int g = rem / slices, sl = rem - g * slices;
+  const int c0 = p.seg_cta0[seg], nch = p.seg_cta0[seg + 1] - c0;
+  // the first batch of o values and every (m, l) are loaded together (one
+  // round trip); later batches (segments of more than kBatch CTAs) follow
+  constexpr int kBatch = 64;
+  const float* po = p.part_o + (static_cast<int64_t>(c0) * G + g) * p.hd + sl * 32 + lane;
+  const int64_t cstride = static_cast<int64_t>(G) * p.hd;
+  float o[kBatch];
+#pragma unroll
+  for (int k = 0; k < kBatch; ++k) o[k] = k < nch ? po[k * cstride] : 0.f;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + static_cast<int64_t>(c0) * kGroupPad + g;
+  constexpr int kPer = kMaxCtas / 32;
+  float2 v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int c = lane + 32 * k;
+    v[k] = c < nch ? ml[static_cast<int64_t>(c) * kGroupPad] : make_float2(-INFINITY, 0.f);
   }
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) M = fmaxf(M, v[k].x);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k)
+    if (lane + 32 * k < nch) L = fmaf(ex2f(v[k].x - M), v[k].y, L);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k)
+    if (lane + 32 * k < nch) wsm[warp][lane + 32 * k] = ex2f(v[k].x - M) * inv;
+  __syncwarp();
+  float acc = 0.f;
+  for (int cb = 0;;) {
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      if (cb + k < nch) acc = fmaf(wsm[warp][cb + k], o[k], acc);
+    cb += kBatch;
+    if (cb >= nch) break;
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) o[k] = cb + k < nch ? po[(cb + k) * cstride] : 0.f;
+  }
+  const int s = seg / p.hkv, kvh = seg - s * p.hkv;
+  p.out[static_cast<int64_t>(s) * p.hq * p.hd + static_cast<int64_t>(kvh * G + g) * p.hd + sl * 32 + lane] =
+      Num<DT>::from_f(acc);
 }
 
 // ============================================================ cache store
