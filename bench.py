@@ -313,7 +313,7 @@ def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, 
             q = per.setdefault(r["kind"], {"ms": 0.0, "bytes": 0, "launches": 0})
             q["ms"] += r["ms"]
             q["bytes"] += amount
-            q["launches"] += 1
+            q["launches"] += r.get("launches", 1)
         dom = max(per, key=lambda k: per[k]["ms"])
         gbs = per[dom]["bytes"] / (per[dom]["ms"] / 1e3) / 1e9
         ms = statistics.median(leg["ms"])
@@ -322,7 +322,7 @@ def decode_leg(dash, stack, dims, wl, h0, cu, cfg_cache, cfg_dense, dev, peaks, 
                      "cached_rows_per_layer": leg["rows"],
                      "step_gb": step_bytes / 1e9, "step_gbs": step_bytes / (ms / 1e3) / 1e9,
                      "step_frac_of_hbm": step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                     "gpu_launches_per_step": len(recs) // block,
+                     "gpu_launches_per_step": sum(r.get("launches", 1) for r in recs) // block,
                      "kernels": {k: {"ms_per_step": v["ms"] / block, "launches_per_step": v["launches"] // block,
                                      "gbs": v["bytes"] / (v["ms"] / 1e3) / 1e9 if v["ms"] else 0.0}
                                  for k, v in sorted(per.items(), key=lambda kv: -kv[1]["ms"])},
@@ -410,7 +410,7 @@ def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
     for r in recs:
         unit, amount = costs.launch_work(r, dims, pairs_by_rows)
         p = per.setdefault(r["kind"], {"launches": 0, "ms": 0.0, "unit": unit, "work": 0})
-        p["launches"] += 1
+        p["launches"] += r.get("launches", 1)
         p["ms"] += r["ms"]
         p["work"] += amount
     total_ms = sum(p["ms"] for p in per.values())
@@ -430,7 +430,7 @@ def kernel_breakdown(recs, dims, pairs_by_rows, steps, peaks):
             q = by_rows.setdefault(f"{r['kind']}@{r['m']}", {"ms": 0.0, "work": 0, "launches": 0})
             q["ms"] += r["ms"]
             q["work"] += amount
-            q["launches"] += 1
+            q["launches"] += r.get("launches", 1)
     for k, q in by_rows.items():
         kernels.setdefault("by_rows", {})[k] = {"launches_per_step": q["launches"] // steps,
                                                 "tflops": q["work"] / (q["ms"] / 1e3) / 1e12 if q["ms"] else 0.0}
