@@ -11,7 +11,7 @@ import csv
 import sys
 
 SHORT = [
-    ("decode_attn_kernel", "decode_attention"),
+    ("decode_attn_kernel", "decode_attention"), ("decode_merge_kernel", "decode_merge"),
     ("gemv_kernel<0", "gemv_qkv_rope_append"), ("gemv_kernel<1", "gemv_resid (o_proj / down)"),
     ("gemv_kernel<2", "gemv_gate_up_swiglu"), ("kv_store_kernel", "kv_store"),
     ("attn_kernel", "attention"),
