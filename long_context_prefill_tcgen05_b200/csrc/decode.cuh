@@ -422,8 +422,8 @@ struct ACfg {
   static constexpr int kOffP = kOffQ + kPanels * 2048;  // 2 buffers of [16, 128 keys] K-major, 2 x 2 KB each
   static constexpr int kOffRed = kOffP + 2 * 4096;      // [2][4 warps][16] floats
   static constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 4;
-  // full[kStages], empty[kStages], q_ready, s_full[2], p_full[2], pv_done[2], red[2], drain
-  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 1;
+  // full[kStages], empty[kStages], q_ready, s_full[2], p_full[2], pv_done[2], red[2], drain, o_read
+  static constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2 + 1 + 1;
   static constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 16 + 1024;
   static constexpr uint32_t kTmemCols = 64;  // S^T buffers [0,16) [16,32), O^T [32,48)
 };
@@ -500,6 +500,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar_pvdone = bar_q + 40;  // [2] P^T(i) V(i) finished, buffer i & 1 free
   const uint32_t bar_red = bar_q + 56;     // [2]
   const uint32_t bar_drain = bar_q + 72;
+  const uint32_t bar_oread = bar_q + 80;  // the 128 epilogue threads no longer read TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -518,6 +519,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar_red, 128);
     mbar_init(bar_red + 8, 128);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_oread, 128);
     fence_mbar_init();
   }
   if (HD == 64) {  // zero panel read as the upper half of V^T
@@ -537,6 +539,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  bool tmem_freed = false;  // warp 1
 
   if (warp == 0) {
     if (lane == 0) {
@@ -614,6 +617,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) umma_commit(bar_drain);
     __syncwarp();
     mbar_wait_drain(bar_drain, 0);
+    // TMEM is freed as soon as the epilogue has read O (a dealloc takes a
+    // few microseconds; it then overlaps the partials' stores)
+    if (warp_wait(bar_oread, 0)) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, C::kTmemCols);
+      tmem_freed = true;
+    }
   } else {
     // ---------------------------------------------- Q staging, softmax, epilogue
     const int wq = warp & 3;
@@ -730,11 +740,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     // MMAs complete in order: PV(nt-1) done means all are.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone + 8 * ((nt - 1) & 1), ((nt - 1) >> 1) & 1));
+    uint32_t o[kGroupPad];
     if (ok) {
       tc_fence_after();
-      uint32_t o[kGroupPad];
       tmem_ld16(tmem_base + lane_off + 2 * kGroupPad, o);
       tmem_ld_wait();
+    }
+    tc_fence_before();
+    mbar_arrive(bar_oread);  // on every path, so the MMA warp's wait ends
+    if (ok) {
       // sum of each head's exponentials over the CTA's keys
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
@@ -772,14 +786,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 1 && !tmem_freed) {  // the early free's wait gave up
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
 // Merge of every (sequence, kv head) segment's partial results, launched
-// after the attention kernel (PDL).  One warp per (segment, head g of its
+// after the attention kernel.  One warp per (segment, head g of its
 // group, 32 dimensions); lane = dimension:
 //   M_g = max_c m_cg,  w_cg = 2^(m_cg - M_g) / sum_c' 2^(m_c'g - M_g) l_c'g,
 //   O_g = sum_c w_cg o_cg  (c ascending).
