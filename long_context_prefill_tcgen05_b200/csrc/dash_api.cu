@@ -1040,12 +1040,36 @@ dash_status launch_gemv_ns(const DeviceInfo& di, const dec::GemvParams& gp, int 
 }
 
 template <int EPI, int DT>
-dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st,
-                        bool preload = false) {
+dash_status launch_gemv_n(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st,
+                          bool preload) {
   if (gp.n <= 1) return launch_gemv_ns<EPI, 1, DT>(di, gp, kind, n_out, preload, st);
   if (gp.n <= 2) return launch_gemv_ns<EPI, 2, DT>(di, gp, kind, n_out, preload, st);
   if (gp.n <= 4) return launch_gemv_ns<EPI, 4, DT>(di, gp, kind, n_out, preload, st);
   return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, preload, st);
+}
+
+template <int EPI, int DT>
+dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st,
+                        bool preload = false) {
+  // o_proj / down whose input rows do not all fit in shared memory: one launch
+  // per group of rows that does (the weights are read once per group, at the
+  // streaming rate; read from global memory per chunk, x cost ~5x more)
+  if constexpr (EPI == dec::kGvResid) {
+    const int per = static_cast<int>(kGemvSmemMax / (static_cast<size_t>(gp.K) * 2));
+    if (gp.n > 1 && per >= 1 && gp.n > per) {
+      TimedLaunch tl(kind, gp.n, n_out, gp.K, st, (gp.n + per - 1) / per);
+      for (int m0 = 0; m0 < gp.n; m0 += per) {
+        dec::GemvParams q = gp;
+        q.n = gp.n - m0 < per ? gp.n - m0 : per;
+        q.x = gp.x + static_cast<int64_t>(m0) * gp.K;
+        q.out = gp.out + static_cast<int64_t>(m0) * gp.ldo;
+        const dash_status s = launch_gemv_n<EPI, DT>(di, q, -1, n_out, st, preload);
+        if (s != DASH_OK) return s;
+      }
+      return DASH_OK;
+    }
+  }
+  return launch_gemv_n<EPI, DT>(di, gp, kind, n_out, st, preload);
 }
 
 // Split-key decode attention of one layer: the CTA count is held to one

@@ -205,3 +205,37 @@ def test_decode_qwen_layer_full_size(gpu_lib, T):
     rows = np.r_[np.arange(0, T, 997), T]
     assert row_rel_err(to_np(ck[rows].cpu()), _kv_rows(kv[0][0][rows])) < KV_TOL
     assert row_rel_err(to_np(cv[rows].cpu()), _kv_rows(kv[0][1][rows])) < KV_TOL
+
+
+@pytest.mark.parametrize("nseq", [5, 8])
+def test_decode_qwen_layer_many_sequences(gpu_lib, nseq):
+    # One Qwen2.5-7B-shaped layer, nseq sequences with short caches of seeded
+    # random rows.  The down projection's input rows (nseq x 18944 values)
+    # exceed what its GEMV stages in shared memory, so it runs in groups of 4.
+    dims = inputs.QWEN7B
+    layers = inputs.make_layers(dims, seed=3, n_layers=1)
+    stack = dash.Stack(dims, _dev_layers(layers))
+    lens = [37, 300, 129, 1, 200, 64, 255, 90][:nseq]
+    cache = dash.KVCache(stack, nseq, max(lens) + 1)
+    hkv, hd = dims.n_kv_heads, dims.head_dim
+    g = torch.Generator().manual_seed(5)
+    ref_kv = []
+    for s, n in enumerate(lens):
+        k = torch.randn(n, hkv * hd, generator=g).to(torch.bfloat16)
+        v = torch.randn(n, hkv * hd, generator=g).to(torch.bfloat16)
+        cache.k[s][:n] = k.to(DEV)
+        cache.v[s][:n] = v.to(DEV)
+        cache.pos[s][:n] = torch.arange(n, dtype=torch.int32, device=DEV)
+        cache.desc[s].len = n
+        ref_kv.append((to_np(k).reshape(n, hkv, hd), to_np(v).reshape(n, hkv, hd), np.arange(n)))
+    x = _new_tokens(nseq, dims.d_model, seed=23)
+    X = x.to(DEV).clone()
+    dash.decode_step(stack, X, lens, cache)
+    assert dash.device_error() == 0
+    Ln = layers_np(layers)
+    for s, n in enumerate(lens):
+        y, kv = O.dash_decode(to_np(x[s:s + 1]), [n], [ref_kv[s]], Ln, dims.as_dict())
+        assert row_rel_err(to_np(X[s:s + 1].cpu()), y) < HIDDEN_TOL, s
+        ck, cv, cp = cache.layer(s, 0)
+        assert ck.shape[0] == n + 1 and int(cp[-1]) == n
+        assert row_rel_err(to_np(ck[-1:].cpu()), _kv_rows(kv[0][0][-1:])) < KV_TOL, s

@@ -206,6 +206,34 @@ def test_fp16_depth11_matches_free_oracle(qwen_depth16, mode):
     assert err <= HIDDEN_TOL
 
 
+@pytest.fixture(scope="module")
+def qwen_reduced16(gpu_lib):
+    """Qwen widths, 4 layers, T = 2048, halting at layer 1 (the bf16 twin of
+    this case in test_gpu_prefill holds Δ to 5e-3 for 99 % of the tokens)."""
+    dims = inputs.QWEN7B
+    layers = _to(inputs.make_layers(dims, seed=31, n_layers=4), F16, "cpu")
+    h0 = inputs.make_hidden(2048, dims.d_model, seed=32)[0].to(F16)
+    L = layers_np(layers)
+    d0 = O.dash_prefill(to_np(h0), L[:2], dims.as_dict(), 1, "prune", keep=1.0)["delta"]
+    yield dims, h0, dash.Stack(dims, _to(layers, F16, DEV)), L, _clear_keep(d0, 0.5)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", ["prune", "halt"])
+def test_fp16_reduced_prefill_matches_free_oracle(qwen_reduced16, mode):
+    """Free-running, 4 layers, halt at layer 1: the stated tolerances hold."""
+    dims, h0, stack, L, keep = qwen_reduced16
+    T = h0.shape[0]
+    Hg, idx, delta, K = _prefill(stack, h0, halt_layer=1, mode=mode, keep=keep)
+    free = O.dash_prefill(to_np(h0), L, dims.as_dict(), 1, mode, keep=keep)
+    assert K == O.topk_count(T, keep) == len(free["idx"])
+    assert _rel(delta, free["delta"]).max() <= DELTA_TOL
+    assert np.array_equal(idx, O.select_topk(delta, keep))
+    _sets_within(idx, free["idx"], free["delta"], _topk_cut(free["delta"], keep), CUT_BAND)
+    assert _compare_rows(mode, Hg, idx, K, free, T) <= HIDDEN_TOL
+
+
 @pytest.mark.slow
 def test_bf16_depth11_departure(gpu_lib):
     """The bf16 path at the same depth (the benchmark's format): its drift,

@@ -400,8 +400,10 @@ def test_qwen_reduced_prefill_matches_free_oracle(qwen_reduced, mode):
     assert K == O.topk_count(T, keep) == len(free["idx"])
     # Δ at layer 1 sees layer 0's output through the bf16 residual stream
     # (up to 2^-8 relative per element, which the fp64 oracle does not round):
-    # 5e-3 holds for 99 % of the tokens, twice that for the worst one (the
-    # per-layer 5e-3 bound is checked teacher-forced in test_qwen_layer_*).
+    # 5e-3 holds for 99 % of the tokens, twice that for the worst one.  This
+    # is the bf16 path's documented departure from the stated 5e-3; the fp16
+    # format holds it on the same case (test_fp16_reduced_prefill_matches_free_oracle),
+    # and the per-layer 5e-3 bound is checked teacher-forced in test_qwen_layer_*.
     rel = np.abs(delta.astype(np.float64) - free["delta"]) / free["delta"]
     assert np.quantile(rel, 0.99) < DELTA_TOL
     assert rel.max() < 2 * DELTA_TOL
