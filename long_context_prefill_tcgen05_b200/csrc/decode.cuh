@@ -100,18 +100,20 @@ constexpr int kGemvWarps = 16;  // one CTA per SM; warps take tasks strided over
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Dot product of 8 16-bit pairs: the even and the odd elements accumulate in
+// two fp32 chains, each step one packed fp32x2 multiply-add (two IEEE fmaf,
+// one instruction on sm_100), and the chains are added at the end.
+template <int DT>
+__device__ __forceinline__ float2 pair(uint32_t v) {
+  return make_float2(Num<DT>::lo(v), Num<DT>::hi(v));
+}
 template <int DT>
 __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
-  using N = Num<DT>;
-  float a = N::lo(w.x) * N::lo(x.x);
-  float b = N::hi(w.x) * N::hi(x.x);
-  a = fmaf(N::lo(w.y), N::lo(x.y), a);
-  b = fmaf(N::hi(w.y), N::hi(x.y), b);
-  a = fmaf(N::lo(w.z), N::lo(x.z), a);
-  b = fmaf(N::hi(w.z), N::hi(x.z), b);
-  a = fmaf(N::lo(w.w), N::lo(x.w), a);
-  b = fmaf(N::hi(w.w), N::hi(x.w), b);
-  return a + b;
+  float2 c = __fmul2_rn(pair<DT>(w.x), pair<DT>(x.x));
+  c = __ffma2_rn(pair<DT>(w.y), pair<DT>(x.y), c);
+  c = __ffma2_rn(pair<DT>(w.z), pair<DT>(x.z), c);
+  c = __ffma2_rn(pair<DT>(w.w), pair<DT>(x.w), c);
+  return c.x + c.y;
 }
 
 template <int DT>
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(32 * kGemvWarps, 1) gemv_kernel(const GemvPara
     bulk_load(smem_u32(pre_w), r0, p.pre_bytes, bar);
     bulk_load(smem_u32(pre_w) + p.pre_bytes, r1, p.pre_bytes, bar);
   }
-  constexpr int U = NS <= 2 ? 8 : (NS <= 4 ? 4 : 2);  // 16-byte chunks per row in flight per lane
+  constexpr int U = NS <= 4 ? 8 : 4;  // 16-byte chunks per row in flight per lane
   // A round of a task's two rows: U 16-byte chunks per row per lane.
   // Without a shared-memory preload, the first task's first round is loaded
   // into these registers before the PDL wait (weights do not depend on the
