@@ -38,6 +38,16 @@ dash_status dash_linear(const dash_bf16* A, int64_t M, int32_t K, const dash_bf1
  * other host threads. */
 int32_t dash_set_gemm_pairs(int32_t enable);
 
+/* Selects the form of the generation step's projections (dash_decode_step)
+ * for 3 or more sequences: enable != 0 (the default) runs them on the tensor
+ * cores (weight rows on the MMA's M dimension, the sequences' rows padded to
+ * 16 on N, K split over SMs with a fixed-order reduction) when the shapes
+ * suit it (rows a multiple of 128, K of 64); enable == 0: the CUDA-core
+ * GEMV.  Both accumulate in fp32; the summation order differs.  Returns the
+ * previous setting.  Not synchronised with launches in flight on other host
+ * threads. */
+int32_t dash_set_decode_tensor_cores(int32_t enable);
+
 /* Causal grouped-query attention (the attention module of §2.1):
  *   Q: [M, hq*hd], K, V: [T_kv, hkv*hd], O: [M, hq*hd] bf16.
  *   Query i sees key j iff kstart(i) <= j <= qpos(i) and j < T_kv, where

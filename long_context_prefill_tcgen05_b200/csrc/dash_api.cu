@@ -16,6 +16,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_tc.cuh"
 #include "gemm.cuh"
 #include "rowops.cuh"
 
@@ -963,6 +964,8 @@ dash_status prefill_impl(const dash_dims* dims, const dash_layer_weights* layers
 namespace dec = dash::decode;
 
 struct DecodeWs {
+  float* tc_part;    // [kTcMaxItems][128][32] partial sums of split tensor-core GEMVs
+  int* tc_counters;  // [kTcMaxItems] (zeroed per step; the kernels leave them zero)
   s16* Q;         // [n, hq*hd]
   s16* O;         // [n, hq*hd] attention output
   s16* Act;       // [n, F]
@@ -972,6 +975,8 @@ struct DecodeWs {
 
 void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
+  w.tc_part = c.take<float>(static_cast<size_t>(dec::kTcMaxItems) * dec::kTcRows * 2 * dec::kTcN);
+  w.tc_counters = c.take<int>(dec::kTcMaxItems);
   w.Q = c.take<s16>(n * qd);
   w.O = c.take<s16>(n * qd);
   w.Act = c.take<s16>(static_cast<size_t>(n) * D.ffn_dim);
@@ -1048,9 +1053,80 @@ dash_status launch_gemv_n(const DeviceInfo& di, const dec::GemvParams& gp, int k
   return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, preload, st);
 }
 
+constexpr size_t kTcSmemBudget = 208 * 1024;
+bool g_gemv_tc = true;  // dash_set_decode_tensor_cores  // weight ring + x slice (dynamic shared memory)
+
+// The tensor-core form (decode_tc.cuh) for gp.n >= kTcMinRows.  Returns
+// DASH_ERR_SHAPE, before launching anything, when the shape does not suit it.
+template <int EPI, int DT>
+dash_status launch_gemv_tc(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out,
+                           const DecodeWs& w, cudaStream_t st) {
+  using C = dec::TcCfg<EPI>;
+  const int R = EPI == dec::kGvSwiglu ? gp.tasks : 2 * gp.tasks;  // weight rows
+  if (R % dec::kTcRows != 0 || gp.K % 64 != 0 || gp.n > dec::kTcN) return DASH_ERR_SHAPE;
+  if (EPI == dec::kGvQkv && (gp.hd > dec::kTcRows || dec::kTcRows % gp.hd != 0)) return DASH_ERR_SHAPE;
+  const int blocks = R / dec::kTcRows, ksteps = gp.K / 64;
+  // K ranges per row block: about one item per SM, each range's x slice and a
+  // ring of at least two stages within the shared-memory budget
+  int splits = 1;  // at most one item per SM: a second round on a few SMs would double their time
+  if (blocks < di.num_sms) splits = std::min(ksteps, di.num_sms / blocks);
+  auto slice = [&](int sp) { return static_cast<size_t>((ksteps + sp - 1) / sp) * C::kPanelBytes; };
+  while (splits < ksteps && slice(splits) + 2 * C::kStageBytes > kTcSmemBudget) ++splits;
+  if (slice(splits) + 2 * C::kStageBytes > kTcSmemBudget) return DASH_ERR_SHAPE;
+  if (splits > 1 && blocks * splits > dec::kTcMaxItems) return DASH_ERR_SHAPE;
+  const int stages = static_cast<int>(
+      std::min<size_t>(dec::kTcMaxStages, (kTcSmemBudget - slice(splits)) / C::kStageBytes));
+  const size_t smem = 1024 + static_cast<size_t>(stages) * C::kStageBytes + slice(splits);
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(dec::gemv_tc_kernel<EPI, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(1024 + kTcSmemBudget));
+  });
+  if (attr_err != cudaSuccess) return DASH_ERR_CUDA;
+  constexpr CUtensorMapDataType kMt = Num<DT>::kMapType;
+  dec::TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!make_map(&maps.w, gp.W, static_cast<uint64_t>(R), gp.K, gp.K, dec::kTcRows, kMt)) return DASH_ERR_INVALID_ARG;
+  if (EPI == dec::kGvSwiglu && !make_map(&maps.w2, gp.W2, static_cast<uint64_t>(R), gp.K, gp.K, dec::kTcRows, kMt))
+    return DASH_ERR_INVALID_ARG;
+  dec::TcParams tp;
+  std::memset(&tp, 0, sizeof(tp));
+  tp.x = gp.x;
+  tp.gain = gp.gain;
+  tp.eps = gp.eps;
+  tp.n = gp.n;
+  tp.K = gp.K;
+  tp.blocks = blocks;
+  tp.splits = splits;
+  tp.ksteps = ksteps;
+  tp.stages = stages;
+  tp.part = w.tc_part;
+  tp.counters = w.tc_counters;
+  tp.out = gp.out;
+  tp.ldo = gp.ldo;
+  tp.q = gp.q;
+  tp.hq = gp.hq;
+  tp.hkv = gp.hkv;
+  tp.hd = gp.hd;
+  tp.theta = gp.theta;
+  tp.seq = gp.seq;
+  const int items = blocks * splits;
+  const unsigned grid = static_cast<unsigned>(items < di.num_sms ? items : di.num_sms);
+  TimedLaunch tl(kind, gp.n, n_out, gp.K, st);
+  if (launch_pdl(dec::gemv_tc_kernel<EPI, DT>, grid, dec::kTcThreads, smem, st, maps, tp) != cudaSuccess)
+    return DASH_ERR_CUDA;
+  return launch_status();
+}
+
 template <int EPI, int DT>
 dash_status launch_gemv(const DeviceInfo& di, const dec::GemvParams& gp, int kind, int64_t n_out, cudaStream_t st,
-                        bool preload = false) {
+                        bool preload = false, const DecodeWs* w = nullptr) {
+  // three or more input rows: the tensor-core form when the shape suits it
+  if (w && gp.n >= dec::kTcMinRows && g_gemv_tc) {
+    const dash_status s = launch_gemv_tc<EPI, DT>(di, gp, kind, n_out, *w, st);
+    if (s != DASH_ERR_SHAPE) return s;
+  }
   // o_proj / down whose input rows do not all fit in shared memory: one launch
   // per group of rows that does (the weights are read once per group, at the
   // streaming rate; read from global memory per chunk, x cost ~5x more)
@@ -1193,6 +1269,9 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
   s16* x = reinterpret_cast<s16*>(X);
   const int d = D.d_model, hq = D.n_heads, hkv = D.n_kv_heads, hd = D.head_dim, F = D.ffn_dim;
   const int qd = hq * hd;
+  if (n >= dec::kTcMinRows &&
+      cudaMemsetAsync(w.tc_counters, 0, sizeof(int) * dec::kTcMaxItems, st) != cudaSuccess)
+    return DASH_ERR_CUDA;
 
   for (int l = 0; l < D.n_layers; ++l) {
     g_timing.layer = l;
@@ -1223,7 +1302,9 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     qkv.hkv = hkv;
     qkv.hd = hd;
     qkv.theta = D.rope_theta;
-    if ((s = launch_gemv<dec::kGvQkv, DT>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvQkv, DT>(*di, qkv, DASH_K_DEC_GEMV_QKV, qd + 2 * hkv * hd, st, false, &w)) !=
+        DASH_OK)
+      break;
     // attention over each sequence's cache (including the new row)
     s = hd == 128 ? decode_attention_hd<128, DT>(*di, D, n, len, lc, w, st)
                   : decode_attention_hd<64, DT>(*di, D, n, len, lc, w, st);
@@ -1238,7 +1319,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     o.tasks = d / 2;
     o.out = x;
     o.ldo = d;
-    if ((s = launch_gemv<dec::kGvResid, DT>(*di, o, DASH_K_DEC_GEMV_O, d, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid, DT>(*di, o, DASH_K_DEC_GEMV_O, d, st, false, &w)) != DASH_OK) break;
     // RMSNorm (fused) -> gate/up with SwiGLU
     dec::GemvParams gu;
     std::memset(&gu, 0, sizeof(gu));
@@ -1252,7 +1333,8 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     gu.tasks = F;
     gu.out = w.Act;
     gu.ldo = F;
-    if ((s = launch_gemv<dec::kGvSwiglu, DT>(*di, gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvSwiglu, DT>(*di, gu, DASH_K_DEC_GEMV_GATE_UP, 2 * F, st, false, &w)) != DASH_OK)
+      break;
     // down + residual
     dec::GemvParams dn;
     std::memset(&dn, 0, sizeof(dn));
@@ -1263,7 +1345,7 @@ dash_status decode_impl(const dash_dims* dims, const dash_layer_weights* layers,
     dn.tasks = d / 2;
     dn.out = x;
     dn.ldo = d;
-    if ((s = launch_gemv<dec::kGvResid, DT>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st, true)) != DASH_OK) break;
+    if ((s = launch_gemv<dec::kGvResid, DT>(*di, dn, DASH_K_DEC_GEMV_DOWN, d, st, true, &w)) != DASH_OK) break;
     for (int q = 0; q < n; ++q) caches[static_cast<size_t>(q) * D.n_layers + l].len += 1;
   }
   g_timing.layer = -1;
@@ -1378,6 +1460,12 @@ dash_status dash_rmsnorm(const dash_bf16* X, int64_t M, int32_t d, const dash_bf
   if (!X || !g || !Y || !aligned16(X) || !aligned16(g) || !aligned16(Y)) return DASH_ERR_INVALID_ARG;
   return rmsnorm<kBf16>(reinterpret_cast<const s16*>(X), M, nullptr, M, d, reinterpret_cast<const s16*>(g), eps,
                  reinterpret_cast<s16*>(Y), as_stream(stream));
+}
+
+int32_t dash_set_decode_tensor_cores(int32_t enable) {
+  const bool prev = g_gemv_tc;
+  g_gemv_tc = enable != 0;
+  return prev ? 1 : 0;
 }
 
 int32_t dash_set_gemm_pairs(int32_t enable) { return g_gemm_pairs.exchange(enable != 0 ? 1 : 0); }

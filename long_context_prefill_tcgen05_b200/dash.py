@@ -80,6 +80,7 @@ _SIGS = {
     "dash_rmsnorm": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_f64, c_vp, c_vp]),
     "dash_linear": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_i32, c_vp, c_vp]),
     "dash_set_gemm_pairs": (c_i32, [c_i32]),
+    "dash_set_decode_tensor_cores": (c_i32, [c_i32]),
     "dash_attention": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "dash_prefill_varlen_workspace_size": (c_sz, [ctypes.POINTER(Dims), c_i64, c_i32, ctypes.POINTER(Config)]),
     "dash_prefill_varlen": (c_i32, [ctypes.POINTER(Dims), ctypes.POINTER(LayerWeights), c_vp,
@@ -284,6 +285,13 @@ def set_gemm_pairs(enable):
     """Runs later GEMMs as 256x256 tiles on SM pairs (True, the default) or as
     single-SM tiles (False); returns the previous setting."""
     return bool(lib().dash_set_gemm_pairs(1 if enable else 0))
+
+
+def set_decode_tensor_cores(enable):
+    """Runs later generation steps' projections for 3 or more sequences on the
+    tensor cores (True, the default) or as CUDA-core GEMVs (False); returns
+    the previous setting."""
+    return bool(lib().dash_set_decode_tensor_cores(1 if enable else 0))
 
 
 def exp2_fma(x, stream=None):

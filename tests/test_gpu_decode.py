@@ -207,11 +207,22 @@ def test_decode_qwen_layer_full_size(gpu_lib, T):
     assert row_rel_err(to_np(cv[rows].cpu()), _kv_rows(kv[0][1][rows])) < KV_TOL
 
 
-@pytest.mark.parametrize("nseq", [5, 8])
-def test_decode_qwen_layer_many_sequences(gpu_lib, nseq):
+@pytest.mark.parametrize("tensor_cores", [True, False])
+@pytest.mark.parametrize("nseq", [3, 5, 8])
+def test_decode_qwen_layer_many_sequences(gpu_lib, nseq, tensor_cores):
     # One Qwen2.5-7B-shaped layer, nseq sequences with short caches of seeded
-    # random rows.  The down projection's input rows (nseq x 18944 values)
-    # exceed what its GEMV stages in shared memory, so it runs in groups of 4.
+    # random rows, in both forms of the projections: on the tensor cores
+    # (K split over the SMs for QKV, o_proj and down) and as CUDA-core GEMVs
+    # (where down's input rows, nseq x 18944 values, exceed what the GEMV
+    # stages in shared memory beyond 4 sequences, so it runs in groups of 4).
+    prev = dash.set_decode_tensor_cores(tensor_cores)
+    try:
+        _many_sequences_case(nseq)
+    finally:
+        dash.set_decode_tensor_cores(prev)
+
+
+def _many_sequences_case(nseq):
     dims = inputs.QWEN7B
     layers = inputs.make_layers(dims, seed=3, n_layers=1)
     stack = dash.Stack(dims, _dev_layers(layers))
@@ -239,3 +250,38 @@ def test_decode_qwen_layer_many_sequences(gpu_lib, nseq):
         ck, cv, cp = cache.layer(s, 0)
         assert ck.shape[0] == n + 1 and int(cp[-1]) == n
         assert row_rel_err(to_np(ck[-1:].cpu()), _kv_rows(kv[0][0][-1:])) < KV_TOL, s
+
+
+def test_decode_wide_ffn_more_items_than_sms(gpu_lib):
+    # A narrow model with a wide FFN (38400 = 300 row blocks of 128): the
+    # tensor-core gate/up projection has more items than the device has SMs,
+    # so CTAs take a second item (accumulator and weight-ring reuse).
+    dims = inputs.ModelDims(2, 256, 4, 2, 64, 38400, 1e4)
+    layers = inputs.make_layers(dims, seed=8, n_layers=2)
+    stack = dash.Stack(dims, _dev_layers(layers))
+    nseq, n = 4, 50
+    cache = dash.KVCache(stack, nseq, n + 1)
+    kvd = dims.n_kv_heads * dims.head_dim
+    g = torch.Generator().manual_seed(9)
+    ref_kv = []
+    for s in range(nseq):
+        per_layer = []
+        for l in range(dims.n_layers):
+            k = torch.randn(n, kvd, generator=g).to(torch.bfloat16)
+            v = torch.randn(n, kvd, generator=g).to(torch.bfloat16)
+            i = s * dims.n_layers + l
+            cache.k[i][:n] = k.to(DEV)
+            cache.v[i][:n] = v.to(DEV)
+            cache.pos[i][:n] = torch.arange(n, dtype=torch.int32, device=DEV)
+            cache.desc[i].len = n
+            per_layer.append((to_np(k).reshape(n, dims.n_kv_heads, dims.head_dim),
+                              to_np(v).reshape(n, dims.n_kv_heads, dims.head_dim), np.arange(n)))
+        ref_kv.append(per_layer)
+    x = _new_tokens(nseq, dims.d_model, seed=24)
+    X = x.to(DEV).clone()
+    dash.decode_step(stack, X, [n] * nseq, cache)
+    assert dash.device_error() == 0
+    Ln = layers_np(layers)
+    for s in range(nseq):
+        y, _ = O.dash_decode(to_np(x[s:s + 1]), [n], ref_kv[s], Ln, dims.as_dict())
+        assert row_rel_err(to_np(X[s:s + 1].cpu()), y) < HIDDEN_TOL, s
