@@ -358,9 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = rmax;
       }
       const float neg = m_run == -INFINITY ? 0.f : -m_run;  // fully masked so far: p = 0
-      float ls[8];
+      // row sum of the exponentials: even and odd columns in packed fp32x2 adds
+      float2 ls[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+      for (int k = 0; k < 4; ++k) ls[k] = make_float2(0.f, 0.f);
       float lsum = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // 64 columns at a time keeps pk small
@@ -368,17 +369,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int c = half * 64 + 2 * i;
-          const float e0 = ex2_approx(fmaf(s[c], sc, neg));  // MUFU
-          const float x1 = fmaf(s[c + 1], sc, neg);
+          // s * scale - max for both columns in one packed fp32x2 FMA (two fmaf)
+          const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), make_float2(sc, sc), make_float2(neg, neg));
+          const float e0 = ex2_approx(x.x);  // MUFU
           const float e1 = (kEmuPeriod > 0 && (i % (kEmuPeriod > 0 ? kEmuPeriod : 1)) == kEmuPeriod - 1)
-                               ? ex2_fma(x1)  // FMA pipe
-                               : ex2_approx(x1);
-          ls[i & 7] += e0 + e1;
+                               ? ex2_fma(x.y)  // FMA pipe
+                               : ex2_approx(x.y);
+          ls[i & 3] = __fadd2_rn(ls[i & 3], make_float2(e0, e1));
           pk[i] = Num<DT>::pack(e0, e1);
         }
         tmem_st32(s_addr + BKV / 2 + 32 * half, pk);
       }
-      lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      lsum = ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
       l_run = fmaf(l_run, alpha, lsum);
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
         // P_t(j-1) V_(j-1) is complete (in-order MMAs): O_t may be rescaled.
