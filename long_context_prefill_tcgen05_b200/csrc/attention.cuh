@@ -80,6 +80,12 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 512;
 };
 
+// max of three fp32 values in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -332,22 +338,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BKV / 2; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = s[k];
+      for (int k = 0; k < 8; ++k) mx[k] = fmax3(s[k], s[8 + k], s[16 + k]);
 #pragma unroll
-      for (int c = 8; c < BKV / 2; c += 8)
+      for (int c = 24; c + 16 <= BKV / 2; c += 16)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], s[c + k], s[c + 8 + k]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[BKV / 2 - 8 + k]);
       tmem_ld_wait();
       if (edge) {
 #pragma unroll
         for (int c = BKV / 2; c < BKV; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
       }
 #pragma unroll
-      for (int c = BKV / 2; c < BKV; c += 8)
+      for (int c = BKV / 2; c < BKV; c += 16)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[c + k]);
-      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], s[c + k], s[c + 8 + k]);
+      const float rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sc;
       // Each row moves its own reference (rarely); the warp-wide vote on
       // whether O needs rescaling waits until after the exponentials.
       float alpha = 1.f;
