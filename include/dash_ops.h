@@ -73,10 +73,9 @@ dash_status dash_decode_attention(const dash_bf16* Q, int32_t nseq, const dash_k
                                   int32_t hkv, int32_t hd, dash_bf16* O, void* ws, size_t ws_bytes,
                                   void* stream);
 
-/* An exponential on the FMA pipe, which the attention softmax can take for a
- * fraction of its elements in place of MUFU (a compile-time option, off: it
- * measured slower; no page counterpart; exported so tests can hold it to its
- * error bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
+/* An exponential on the FMA pipe, which the attention softmax takes for one
+ * element in 16 in place of MUFU (a compile-time period; no page
+ * counterpart; exported so tests can hold it to its error bound): y[i] = 2^x[i] via x = round(x) + f, a cubic in f on [-0.5, 0.5]
  * (max relative error 7.5e-5) and an exponent-field add; inputs below -125
  * are clamped (result ~2e-38).  x, y: [n] fp32 device arrays. */
 dash_status dash_exp2_fma(const float* x, int64_t n, float* y, void* stream);

@@ -51,9 +51,10 @@ constexpr int kStages = 2;  // load groups in flight
 constexpr int kThreads = 320;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // One exponential in every 2 * kEmuPeriod columns is computed on the FMA pipe
-// (ex2_fma); the rest use MUFU.  0 disables the FMA path.
+// (ex2_fma); the rest use MUFU, whose 16 per clock per SM match the tensor
+// pipe's rate for this tile shape.  0 disables the FMA path.
 #ifndef DASH_ATTN_EMU_PERIOD
-#define DASH_ATTN_EMU_PERIOD 0
+#define DASH_ATTN_EMU_PERIOD 8
 #endif
 constexpr int kEmuPeriod = DASH_ATTN_EMU_PERIOD;
 
