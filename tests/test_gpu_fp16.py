@@ -281,3 +281,34 @@ def test_fp16_qwen_layer_full_T_sampled_rows(gpu_lib):
     assert _rel(delta.cpu().numpy()[rows], O.delta_scores(u)).max() < DELTA_TOL
     del stack, layers
     torch.cuda.empty_cache()
+
+
+def test_fp16_decode_three_sequences_tensor_cores(tiny16):
+    """Three sequences per step: the projections run on the tensor cores in
+    the fp16 format (QKV, o_proj and down on this stack's shapes)."""
+    dims, h0, stack, L = tiny16
+    nseq, n = 3, 70
+    cache = dash.KVCache(stack, nseq, n + 1)
+    kvd = dims.n_kv_heads * dims.head_dim
+    g = torch.Generator().manual_seed(12)
+    ref_kv = []
+    for s in range(nseq):
+        per_layer = []
+        for l in range(dims.n_layers):
+            k = torch.randn(n, kvd, generator=g).to(F16)
+            v = torch.randn(n, kvd, generator=g).to(F16)
+            i = s * dims.n_layers + l
+            cache.k[i][:n] = k.to(DEV)
+            cache.v[i][:n] = v.to(DEV)
+            cache.pos[i][:n] = torch.arange(n, dtype=torch.int32, device=DEV)
+            cache.desc[i].len = n
+            per_layer.append((to_np(k).reshape(n, dims.n_kv_heads, dims.head_dim),
+                              to_np(v).reshape(n, dims.n_kv_heads, dims.head_dim), np.arange(n)))
+        ref_kv.append(per_layer)
+    x = inputs.make_hidden(nseq, dims.d_model, seed=14)[0].to(F16)
+    X = x.to(DEV).clone()
+    dash.decode_step(stack, X, [n] * nseq, cache)
+    assert dash.device_error() == 0
+    for s in range(nseq):
+        y, _ = O.dash_decode(to_np(x[s:s + 1]), [n], ref_kv[s], L, dims.as_dict())
+        assert row_rel_err(to_np(X[s:s + 1].cpu()), y) < HIDDEN_TOL, s
