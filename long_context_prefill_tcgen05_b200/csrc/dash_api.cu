@@ -975,8 +975,12 @@ struct DecodeWs {
 
 void carve_decode(const dash_dims& D, int n, Carver& c, DecodeWs& w) {
   const size_t qd = static_cast<size_t>(D.n_heads) * D.head_dim;
-  w.tc_part = c.take<float>(static_cast<size_t>(dec::kTcMaxItems) * dec::kTcRows * 2 * dec::kTcN);
-  w.tc_counters = c.take<int>(dec::kTcMaxItems);
+  w.tc_part = nullptr;  // the tensor-core projections (3 or more sequences) only
+  w.tc_counters = nullptr;
+  if (n >= dec::kTcMinRows) {
+    w.tc_part = c.take<float>(static_cast<size_t>(dec::kTcMaxItems) * dec::kTcRows * 2 * dec::kTcN);
+    w.tc_counters = c.take<int>(dec::kTcMaxItems);
+  }
   w.Q = c.take<s16>(n * qd);
   w.O = c.take<s16>(n * qd);
   w.Act = c.take<s16>(static_cast<size_t>(n) * D.ffn_dim);
