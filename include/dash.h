@@ -360,9 +360,13 @@ size_t dash_decode_workspace_size(const dash_dims* dims, int32_t nseq);
  *   caches HOST array [nseq * n_layers] (sequence-major): each layer appends
  *          the token's key/value (and position) at row len, then len += 1;
  *          every cache needs len < capacity and len + 1 <= 2^31 - 1.
- * Layer l: RMSNorm -> QKV GEMV with RoPE and the cache append -> attention
- * over the cache -> o_proj + residual -> RMSNorm -> gate/up GEMV with SwiGLU
- * -> down + residual.  Requires (n_heads / n_kv_heads) <= 16. */
+ * Layer l: RMSNorm -> QKV projection with RoPE and the cache append ->
+ * attention over the cache -> o_proj + residual -> RMSNorm -> gate/up
+ * projection with SwiGLU -> down + residual.  The projections run as
+ * CUDA-core GEMVs for 1 or 2 sequences and on the tensor cores for 3 or more
+ * when the shapes suit it (dash_set_decode_tensor_cores in dash_ops.h).
+ * Requires (n_heads / n_kv_heads) <= 16.  Results are deterministic: a fixed
+ * summation order for every sequence count. */
 dash_status dash_decode_step(const dash_dims* dims, const dash_layer_weights* layers, dash_bf16* X,
                              int32_t nseq, const int32_t* pos, dash_kv_cache* caches, void* ws, size_t ws_bytes,
                              void* stream);
