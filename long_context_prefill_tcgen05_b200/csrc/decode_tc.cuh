@@ -243,20 +243,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
       // the four epilogue warps take every decision below alike, so that
       // their named barriers always see all 128 threads
       const bool got = named_bar_and(1, 128, mbar_wait(bar_acc, acc_phase & 1u));
-      uint32_t u[C::kAcc][kTcN];
-      if (got) {
-        tc_fence_after();
-        tmem_ld16(tmem + lane_off, u[0]);
-        if (C::kAcc == 2) tmem_ld16(tmem + lane_off + kTcN, u[C::kAcc - 1]);
-        tmem_ld_wait();
-      }
-      tc_fence_before();
-      mbar_arrive(bar_accfree);
       float y[C::kAcc][kTcN];
 #pragma unroll
       for (int a = 0; a < C::kAcc; ++a)
 #pragma unroll
-        for (int m = 0; m < kTcN; ++m) y[a][m] = __uint_as_float(u[a][m]);
+        for (int m = 0; m < kTcN; ++m) y[a][m] = 0.f;
+      if (got) {
+        uint32_t u[C::kAcc][kTcN];
+        tc_fence_after();
+        tmem_ld16(tmem + lane_off, u[0]);
+        if (C::kAcc == 2) tmem_ld16(tmem + lane_off + kTcN, u[C::kAcc - 1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int a = 0; a < C::kAcc; ++a)
+#pragma unroll
+          for (int m = 0; m < kTcN; ++m) y[a][m] = __uint_as_float(u[a][m]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_accfree);
       bool last = got;
       if (p.splits > 1) {
         // this item's partial sums out; the row block's last item adds all of them in split order
