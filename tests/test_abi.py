@@ -124,6 +124,11 @@ def test_workspace_sizes_grow_with_tokens(L):
     # activations for T = 32768 fit well inside one GPU's memory
     assert 1 << 30 < big < 8 << 30
     assert L.dash_layer_workspace_size(ctypes.byref(dims), 100, 50, 100) == 0  # T_kv < M rejected
+    # a decode workspace sized for n sequences serves any fewer (3 or more add the
+    # split-K partial sums of the tensor-core projections)
+    dec = [L.dash_decode_workspace_size(ctypes.byref(qd), n) for n in range(1, 9)]
+    assert all(0 < a <= b for a, b in zip(dec, dec[1:]))
+    assert dec[2] - dec[1] > 8 << 20
 
 
 def _cache_arr(n, k=FAKE, v=FAKE, cap=1024, ln=0):
