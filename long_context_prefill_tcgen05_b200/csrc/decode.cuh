@@ -808,7 +808,7 @@ struct MergeParams {
   int n, hq, hkv, group, hd, items;
   int seg_cta0[kMaxSegs + 1];
 };
-constexpr int kMergeWarps = 4;
+constexpr int kMergeWarps = 1;  // one warp per CTA: the merge's loads spread over more SMs
 
 template <int DT>
 __global__ void __launch_bounds__(32 * kMergeWarps) decode_merge_kernel(const MergeParams p) {
