@@ -1057,8 +1057,8 @@ dash_status launch_gemv_n(const DeviceInfo& di, const dec::GemvParams& gp, int k
   return launch_gemv_ns<EPI, 8, DT>(di, gp, kind, n_out, preload, st);
 }
 
-constexpr size_t kTcSmemBudget = 208 * 1024;
-bool g_gemv_tc = true;  // dash_set_decode_tensor_cores  // weight ring + x slice (dynamic shared memory)
+constexpr size_t kTcSmemBudget = 208 * 1024;  // weight ring + x slice (dynamic shared memory)
+bool g_gemv_tc = true;                         // dash_set_decode_tensor_cores
 
 // The tensor-core form (decode_tc.cuh) for gp.n >= kTcMinRows.  Returns
 // DASH_ERR_SHAPE, before launching anything, when the shape does not suit it.
@@ -1070,9 +1070,10 @@ dash_status launch_gemv_tc(const DeviceInfo& di, const dec::GemvParams& gp, int 
   if (R % dec::kTcRows != 0 || gp.K % 64 != 0 || gp.n > dec::kTcN) return DASH_ERR_SHAPE;
   if (EPI == dec::kGvQkv && (gp.hd > dec::kTcRows || dec::kTcRows % gp.hd != 0)) return DASH_ERR_SHAPE;
   const int blocks = R / dec::kTcRows, ksteps = gp.K / 64;
-  // K ranges per row block: about one item per SM, each range's x slice and a
-  // ring of at least two stages within the shared-memory budget
-  int splits = 1;  // at most one item per SM: a second round on a few SMs would double their time
+  // K ranges per row block: at most one item per SM (a second round on a few
+  // SMs would double their time), each range's x slice and a ring of at least
+  // two stages within the shared-memory budget
+  int splits = 1;
   if (blocks < di.num_sms) splits = std::min(ksteps, di.num_sms / blocks);
   auto slice = [&](int sp) { return static_cast<size_t>((ksteps + sp - 1) / sp) * C::kPanelBytes; };
   while (splits < ksteps && slice(splits) + 2 * C::kStageBytes > kTcSmemBudget) ++splits;
